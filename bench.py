@@ -1,0 +1,429 @@
+#!/usr/bin/env python
+"""Benchmark of the Hyper-Connections step on B200.
+
+A step is one pass of the whole hot path over one batch: the fused mHC call
+(per-token Sinkhorn projection of the 4x4 mixing logits, write mix, read-weight
+softmax, read mix, pre-norm RMSNorm) on T = 16384 tokens, n = 4 streams,
+d = 7168, bf16 storage, K = 20 -- one hc_write_then_read launch. Inputs are
+synthetic (seeded, drawn on the device) and resident in HBM; the stream state
+ping-pongs between two buffers, so every step reads and writes 2.35 GB, far
+more than the 126 MB L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0). Multi-GPU runs (torchrun, one process per GPU)
+are weak scaling: every rank runs its own batch; the step has no collective
+(tokens are independent), NCCL is used only for the barrier and the max-over-
+ranks timing.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOAD = dict(name="mhc_per_token_sinkhorn_fused", T=16384, n=4, d=7168, dtype="bf16", K=20,
+                eps=1e-6, cfg=3)
+METRIC = "HC step tokens/sec at n=4, d=7168 (bf16); achieved HBM GB/s vs ~8 TB/s peak"
+UNIT = "tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def _source_hash():
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "hyper_connections_stream_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode())
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _profiled_traffic(kernel_key: str):
+    """ncu DRAM bytes per launch committed under profiles/, if the kernel
+    sources have not changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            entry = json.load(f)[kernel_key]
+    except Exception:
+        return None
+    if entry.get("source_sha") != _source_hash():
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+            self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "100"]
+            if self.uuid:
+                cmd += ["-i", self.uuid]
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(cmd, stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return None
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    rows.append((float(parts[0]), float(parts[1]), parts[4:8]))
+                except ValueError:
+                    continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, st in rows for i, s in enumerate(st)
+                          if s.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+BAD_REASONS = {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}
+
+
+# ----------------------------------------------------------------------------
+# the GPU arm
+# ----------------------------------------------------------------------------
+
+def _dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _max_over_ranks(value: float, ws: int, device) -> float:
+    if ws == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def make_inputs(w, rank, device):
+    import torch
+    import hc_inputs as gen
+    T, n, d, cfg = w["T"], w["n"], w["d"], w["cfg"]
+    sd = 7919 * rank
+    H = gen.device_normal(gen.SEED_H + cfg + sd, (T, n, d), torch.bfloat16, device)
+    y = gen.device_normal(gen.SEED_Y + cfg + sd, (T, d), torch.bfloat16, device)
+    L = gen.device_normal(gen.SEED_L + cfg + sd, (T, n, n), torch.float32, device)
+    rl = gen.device_normal(gen.SEED_L + 100 + cfg + sd, (T, n), torch.float32, device)
+    _, _, b = gen.static_params(cfg, n)
+    return dict(H=H, y=y, L=L, rl=rl, b=torch.from_numpy(b).to(device),
+                g=torch.ones(d, dtype=torch.float32, device=device))
+
+
+def run_ours(args):
+    import torch
+    from hyper_connections_stream_b200 import _lib as hc
+    from hyper_connections_stream_b200 import traffic
+
+    ws, rank, local = _dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    w = WORKLOAD
+    T, n, d, K = w["T"], w["n"], w["d"], w["K"]
+    inp = make_inputs(w, rank, device)
+    H0 = inp["H"]
+    H1 = torch.empty_like(H0)
+    x = torch.empty((T, d), dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(src, dst):
+        hc.write_then_read(src, inp["y"], inp["L"], inp["b"], inp["rl"], inp["g"], eps=w["eps"],
+                           mix=hc.MIX_SINKHORN_LOGITS, K=K, read=hc.READ_SOFTMAX_LOGITS,
+                           out=dst, x_next=x)
+
+    bufs = (H0, H1)
+    for i in range(args.warmup):
+        step(bufs[i % 2], bufs[(i + 1) % 2])
+    torch.cuda.synchronize()
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    except Exception:
+        pass
+
+    def timed():
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        _barrier(ws)
+        torch.cuda.synchronize()
+        with ClockSampler(uuid if rank == 0 else None) as clk:
+            for i in range(args.steps):
+                ev[i][0].record(stream)
+                step(bufs[i % 2], bufs[(i + 1) % 2])
+                ev[i][1].record(stream)
+            torch.cuda.synchronize()
+        _barrier(ws)
+        total_ms = ev[0][0].elapsed_time(ev[-1][1])
+        per_launch = [s.elapsed_time(e) for s, e in ev]
+        return total_ms, per_launch, clk.summary()
+
+    total_ms, per_launch, clocks = timed()
+    if clocks and BAD_REASONS & set(clocks["reasons"]):
+        total_ms, per_launch, clocks = timed()  # re-measured once
+    total_ms = _max_over_ranks(total_ms, ws, device)
+    ms_per_step = total_ms / args.steps
+    value = ws * T * args.steps / (total_ms / 1e3)
+
+    # dominant (only) kernel: algorithmic bytes per launch / mean launch time
+    kern_ms = _max_over_ranks(statistics.mean(per_launch), ws, device)
+    alg_bytes = traffic.step_bytes("fused", T, n, d, "bf16", per_token_mix=True,
+                                   per_token_read=True)
+    peak, peak_kind = _peaks()
+    achieved = alg_bytes / (kern_ms / 1e3) / 1e9
+    prof = _profiled_traffic("fused_mhc_n4_d7168_bf16_T16384")
+
+    # end to end through the public API with host buffers
+    e2e = run_e2e(args, inp, w, device, ws)
+
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w["name"], "T": T, "n": n, "d": d, "K": K, "storage": "bf16",
+                   "accumulate": "fp32", "tokens_per_gpu": T, "global_tokens": ws * T,
+                   "parallelism": f"token-sharded x{ws} (no collective)",
+                   "l2": "inputs larger than L2: 2.35 GB read+written per step vs 126 MB L2; "
+                         "stream state ping-pongs between two buffers"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": prof, "peak_source": peak_kind,
+                     "algorithmic_bytes_per_launch": alg_bytes, "kernel_ms": kern_ms,
+                     "frac_of_8TBs": achieved / 8000.0},
+        "e2e": e2e,
+        "gpu_launches": args.steps * ws,
+        "clocks": clocks,
+    }
+    if ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, target_s=args.cpu_seconds)
+    return line
+
+
+def run_e2e(args, inp, w, device, ws):
+    """Same step through the public API with pinned host buffers: every step
+    copies its inputs host->device, runs the kernel and copies H' and x back;
+    all inside the timed region (CUDA events on the launching stream)."""
+    import torch
+    from hyper_connections_stream_b200 import _lib as hc
+    T, n, d = w["T"], w["n"], w["d"]
+    hH = inp["H"].cpu().pin_memory()
+    hy = inp["y"].cpu().pin_memory()
+    hL = inp["L"].cpu().pin_memory()
+    hrl = inp["rl"].cpu().pin_memory()
+    oH = torch.empty_like(hH).pin_memory()
+    ox = torch.empty((T, d), dtype=torch.bfloat16).pin_memory()
+    dH = torch.empty_like(inp["H"])
+    dy = torch.empty_like(inp["y"])
+    dL = torch.empty_like(inp["L"])
+    drl = torch.empty_like(inp["rl"])
+    dx = torch.empty((T, d), dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        dH.copy_(hH, non_blocking=True)
+        dy.copy_(hy, non_blocking=True)
+        dL.copy_(hL, non_blocking=True)
+        drl.copy_(hrl, non_blocking=True)
+        hc.write_then_read(dH, dy, dL, inp["b"], drl, inp["g"], eps=w["eps"],
+                           mix=hc.MIX_SINKHORN_LOGITS, K=w["K"], read=hc.READ_SOFTMAX_LOGITS,
+                           out=dH, x_next=dx)
+        oH.copy_(dH, non_blocking=True)
+        ox.copy_(dx, non_blocking=True)
+
+    steps = max(3, min(args.e2e_steps, args.steps))
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    _barrier(ws)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        step()
+    e.record(stream)
+    torch.cuda.synchronize()
+    ms = _max_over_ranks(s.elapsed_time(e), ws, device)
+    h2d = hH.numel() * 2 + hy.numel() * 2 + hL.numel() * 4 + hrl.numel() * 4
+    d2h = oH.numel() * 2 + ox.numel() * 2
+    return {"value": ws * T * steps / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": steps, "ms_per_step": ms / steps}
+
+
+# ----------------------------------------------------------------------------
+# the oracle (CPU baseline / reference arm)
+# ----------------------------------------------------------------------------
+
+def _oracle_sample(w, S, seed_shift=0):
+    import numpy as np
+    import hc_inputs as gen
+    n, d, cfg = w["n"], w["d"], w["cfg"]
+    H = gen.streams(cfg + seed_shift, S, n, d, "bf16")
+    y = gen.block_out(cfg + seed_shift, S, d, "bf16")
+    L = gen.mix_logits(cfg + seed_shift, S, n)
+    rl = gen.read_logits(cfg + seed_shift, S, n)
+    _, _, b = gen.static_params(cfg, n)
+    return H, y, L, b, rl, np.ones(d, np.float32)
+
+
+def _oracle_step(w, sample):
+    import oracle
+    H, y, L, b, rl, g = sample
+    oracle.write_then_read(H, y, L, b, rl, g, w["eps"], "bf16", K=w["K"], mix_logits=True,
+                           read_logits=True)
+
+
+def _oracle_rate(w, S):
+    sample = _oracle_sample(w, S)
+    t0 = time.perf_counter()
+    _oracle_step(w, sample)
+    return S / (time.perf_counter() - t0)
+
+
+def cpu_baseline(w, target_s=12.0):
+    """The oracle, as it stands, on the host cores: a bounded token sample of
+    the same workload sized to about target_s seconds of work."""
+    import oracle
+    probe = 64
+    rate = _oracle_rate(w, probe)
+    S = int(max(probe, min(w["T"], rate * target_s)))
+    sample = _oracle_sample(w, S)
+    t0 = time.perf_counter()
+    _oracle_step(w, sample)
+    dt = time.perf_counter() - t0
+    return {"value": S / dt, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{S} of the workload's {w['T']} tokens (same shapes and distributions, "
+                      f"host-generated), one fused step, {dt:.1f} s"}
+
+
+def run_reference(args):
+    ws, rank, _ = _dist_env()
+    if rank != 0:
+        return None
+    import oracle
+    w = WORKLOAD
+    rate = _oracle_rate(w, 32)
+    budget_s = args.ref_seconds
+    S = int(max(1, min(w["T"], rate * budget_s / max(1, args.steps + args.warmup))))
+    sample = _oracle_sample(w, S)
+    for _ in range(args.warmup):
+        _oracle_step(w, sample)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_step(w, sample)
+    dt = time.perf_counter() - t0
+    value = S * args.steps / dt
+    cores = oracle.max_threads()
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": w["name"], "T": w["T"], "n": w["n"], "d": w["d"], "K": w["K"],
+                   "storage": "bf16", "accumulate": "fp32",
+                   "sample_tokens_per_step": S},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{S} tokens of the {w['T']}-token workload per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=8)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-seconds", type=float, default=90.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    if ws != args.gpus and not (ws == 1 and args.gpus == 1):
+        if args.gpus > 1 and ws == 1:
+            ap.error(f"--gpus {args.gpus} needs torchrun with {args.gpus} processes")
+    line = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,193 @@
+"""ctypes binding of libhc_b200.so (include/hc_api.h).
+
+Argument marshalling only: tensors are checked for device, dtype, shape and
+contiguity, turned into raw pointers plus token strides, and the call is
+enqueued on torch's current CUDA stream. Every step of the HC computation runs
+in the library's kernels; there is no fallback. If the library is missing or
+fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhc_b200.so")
+
+HC_OK, HC_ERR_INVALID_ARG, HC_ERR_UNSUPPORTED, HC_ERR_MISALIGNED = 0, 1, 2, 3
+HC_ERR_ALIAS, HC_ERR_CUDA, HC_ERR_DEVICE = 4, 5, 6
+HC_F32, HC_BF16 = 0, 1
+MIX_MATRIX, MIX_SINKHORN_LOGITS = 0, 1
+READ_WEIGHTS, READ_SOFTMAX_LOGITS = 0, 1
+
+_DT = {torch.float32: HC_F32, torch.bfloat16: HC_BF16}
+
+# C signatures of the entry points in include/hc_api.h
+_i64, _i32, _vp, _f32 = C.c_int64, C.c_int, C.c_void_p, C.c_float
+SIGNATURES = {
+    "hc_sinkhorn": ([_vp, _vp, _i64, _i32, _i32, _vp], _i32),
+    "hc_read_rmsnorm": ([_vp, _vp, _i32, _i64, _i32, _i64, _i32, _vp, _i64, _vp, _f32, _vp], _i32),
+    "hc_write_mix": ([_vp, _vp, _vp, _i32, _i64, _i32, _i64, _i32, _vp, _i64, _i32, _vp, _i64,
+                      _vp], _i32),
+    "hc_write_then_read": ([_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i64, _i32, _vp, _i64, _i32,
+                            _vp, _i64, _i32, _vp, _i64, _vp, _f32, _vp], _i32),
+    "hc_status_string": ([_i32], C.c_char_p),
+    "hc_last_error": ([], C.c_char_p),
+    "hc_version": ([], _i32),
+}
+
+
+class HCError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{status_string(status)} ({status}): {detail}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib():
+    """Load libhc_b200.so (raises if it is missing: build it first with
+    `python -m hyper_connections_stream_b200.build`)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libhc_b200.so not found at {LIB_PATH}; build it with "
+                              "`python -m hyper_connections_stream_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        for name, (args, res) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def status_string(st: int) -> str:
+    return lib().hc_status_string(int(st)).decode()
+
+
+def _check(st: int):
+    if st != HC_OK:
+        raise HCError(st, lib().hc_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    return C.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need_cuda(name, t, dtype=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _tok_param(name, p, T, per_shape):
+    """Shared ([*per_shape]) or per-token ([T, *per_shape]) fp32 parameter ->
+    token stride in floats."""
+    _need_cuda(name, p, torch.float32)
+    per = 1
+    for s in per_shape:
+        per *= s
+    if tuple(p.shape) == tuple(per_shape):
+        return 0
+    if tuple(p.shape) == (T, *per_shape):
+        return per
+    raise ValueError(f"{name} must have shape {tuple(per_shape)} or {(T, *per_shape)}, "
+                     f"got {tuple(p.shape)}")
+
+
+def _streams_shape(H):
+    if H.dim() != 3:
+        raise ValueError(f"H must be [T, n, d], got {tuple(H.shape)}")
+    if H.dtype not in _DT:
+        raise ValueError(f"H must be float32 or bfloat16, got {H.dtype}")
+    return H.shape
+
+
+def sinkhorn(logits: torch.Tensor, K: int, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Doubly stochastic projection of [..., n, n] fp32 logits: exp, then K
+    (row, column) normalisation pairs."""
+    _need_cuda("logits", logits, torch.float32)
+    n = logits.shape[-1]
+    if logits.dim() < 2 or logits.shape[-2] != n:
+        raise ValueError("logits must be [..., n, n]")
+    T = logits.numel() // (n * n) if n else 0
+    out = torch.empty_like(logits) if out is None else out
+    _need_cuda("out", out, torch.float32)
+    _check(lib().hc_sinkhorn(_ptr(logits), _ptr(out), T, n, int(K), _stream(logits.device)))
+    return out
+
+
+def read_rmsnorm(H, a, g=None, *, eps: float = 1e-6, read: int = READ_WEIGHTS, x=None):
+    """x = RMSNorm(sum_i a_i H_i) * g. H [T,n,d]; a [n] or [T,n] (weights or,
+    with read=READ_SOFTMAX_LOGITS, logits); g [d] fp32 or None."""
+    _need_cuda("H", H)
+    T, n, d = _streams_shape(H)
+    a_s = _tok_param("a", a, T, (n,))
+    if g is not None:
+        _need_cuda("g", g, torch.float32)
+        if tuple(g.shape) != (d,):
+            raise ValueError("g must be [d]")
+    x = torch.empty((T, d), dtype=H.dtype, device=H.device) if x is None else x
+    _need_cuda("x", x, H.dtype)
+    _check(lib().hc_read_rmsnorm(_ptr(H), _ptr(x), _DT[H.dtype], T, n, d, int(read), _ptr(a),
+                                 a_s, _ptr(g), float(eps), _stream(H.device)))
+    return x
+
+
+def write_mix(H, y, A, b, *, mix: int = MIX_MATRIX, K: int = 0, out=None):
+    """H'_j = sum_i A[i,j] H_i + b_j y. A [n,n] or [T,n,n] (matrix or, with
+    mix=MIX_SINKHORN_LOGITS, logits projected by K Sinkhorn pairs); b [n] or
+    [T,n]. out may be H (in place)."""
+    _need_cuda("H", H)
+    T, n, d = _streams_shape(H)
+    _need_cuda("y", y, H.dtype)
+    if tuple(y.shape) != (T, d):
+        raise ValueError("y must be [T, d]")
+    A_s = _tok_param("A", A, T, (n, n))
+    b_s = _tok_param("b", b, T, (n,))
+    out = torch.empty_like(H) if out is None else out
+    _need_cuda("out", out, H.dtype)
+    _check(lib().hc_write_mix(_ptr(H), _ptr(y), _ptr(out), _DT[H.dtype], T, n, d, int(mix),
+                              _ptr(A), A_s, int(K), _ptr(b), b_s, _stream(H.device)))
+    return out
+
+
+def write_then_read(H, y, A, b, a_next, g_next=None, *, eps: float = 1e-6,
+                    mix: int = MIX_MATRIX, K: int = 0, read: int = READ_WEIGHTS,
+                    out=None, x_next=None):
+    """Fused: layer l's write, then layer l+1's read + RMSNorm of the stored H'.
+    Returns (H', x_next)."""
+    _need_cuda("H", H)
+    T, n, d = _streams_shape(H)
+    _need_cuda("y", y, H.dtype)
+    if tuple(y.shape) != (T, d):
+        raise ValueError("y must be [T, d]")
+    A_s = _tok_param("A", A, T, (n, n))
+    b_s = _tok_param("b", b, T, (n,))
+    a_s = _tok_param("a_next", a_next, T, (n,))
+    if g_next is not None:
+        _need_cuda("g_next", g_next, torch.float32)
+        if tuple(g_next.shape) != (d,):
+            raise ValueError("g_next must be [d]")
+    out = torch.empty_like(H) if out is None else out
+    x_next = torch.empty((T, d), dtype=H.dtype, device=H.device) if x_next is None else x_next
+    _need_cuda("out", out, H.dtype)
+    _need_cuda("x_next", x_next, H.dtype)
+    _check(lib().hc_write_then_read(_ptr(H), _ptr(y), _ptr(out), _ptr(x_next), _DT[H.dtype],
+                                    T, n, d, int(mix), _ptr(A), A_s, int(K), _ptr(b), b_s,
+                                    int(read), _ptr(a_next), a_s, _ptr(g_next), float(eps),
+                                    _stream(H.device)))
+    return out, x_next

@@ -1,0 +1,156 @@
+/*
+ * hc_api.h -- C ABI of libhc_b200.so: the Hyper-Connections residual step on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method ("Hyper-connections (mHC)" glossary entry, hfviewer, definition
+ * paragraph): the transformer's single residual stream x + f(x) is widened to
+ * n parallel streams H[n][d] per token; learned matrices mix the streams
+ * before the block runs (read) and after it (write); the mHC variant makes
+ * the mixing doubly stochastic with a few Sinkhorn iterations. Hy4 uses n = 4
+ * ("Tencent open-sources Hy4 Preview at 770B -- Identity Hyper-Connections",
+ * learnaivisually, TL;DR), and the block normalises its input (pre-norm,
+ * same page, Jargon).
+ *
+ * Equations (the pages print none; these are the readings this library
+ * implements):
+ *   read   x    = RMSNorm(h) * g,  h = sum_i a_i H_i,
+ *                 RMSNorm(h) = h / sqrt(mean_k(h_k^2) + eps)
+ *   write  H'_j = sum_i A[i][j] H_i + b_j * y      (row i = source stream)
+ *   mHC    A    = Sinkhorn_K(exp(L)): K times divide each row by its sum,
+ *                 then each column by its sum (exactly K pairs, no early exit)
+ *          a    = softmax(l) over the n streams (per-token read logits)
+ *
+ * Arithmetic: fp32 accumulation. Each mix is a chain of correctly rounded
+ * fp32 fused multiply-adds in stream order starting from -0.0f; the stored
+ * results (H', x) are rounded once to the storage dtype (bf16: round to
+ * nearest even). The RMSNorm statistic sum_k h_k^2 is accumulated in fp64,
+ * r = (float)(1 / sqrt(ss / d + eps)), and x = (h * r) * g in fp32. The
+ * read of the fused call uses the stored (rounded) H'.
+ *
+ * Layout (row-major, no padding): H, Hout [T][n][d] (a token's n rows are
+ * contiguous); y, x [T][d]; fp32 parameters. Per-token parameters take a
+ * token stride in elements: 0 = one set shared by every token (a per-layer
+ * parameter), otherwise the distance between consecutive tokens' sets
+ * (n*n for A or L, n for a, b or l when densely packed).
+ *
+ * Conventions, all entry points:
+ *  - Every pointer is a DEVICE pointer on the current CUDA device, allocated
+ *    and owned by the caller. The library allocates nothing, frees nothing
+ *    and never synchronises; work is enqueued on `stream` (a cudaStream_t;
+ *    NULL = the legacy default stream) and completes asynchronously.
+ *  - Arguments are validated on the host before anything is launched; on any
+ *    error nothing is launched and the status says why (hc_last_error() has
+ *    the details for the calling thread).
+ *  - T == 0 is a no-op that returns HC_OK once the scalar arguments are valid.
+ *  - Supported: 1 <= n <= 8; d > 0 with d % 8 == 0 (bf16) or d % 4 == 0
+ *    (fp32); d <= 32768 (bf16) or 16384 (fp32) for calls that normalise.
+ *    H, y, Hout, x and g are 16-byte aligned; A, b, a are 4-byte aligned.
+ *  - Hout == H (exact in-place update) is allowed. Any other overlap between
+ *    an output and another buffer returns HC_ERR_ALIAS.
+ *  - NaN and Inf inputs propagate per IEEE 754; they are not checked.
+ */
+#ifndef HC_API_H
+#define HC_API_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HC_API __attribute__((visibility("default")))
+#else
+#define HC_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HC_OK = 0,
+    HC_ERR_INVALID_ARG = 1, /* null pointer, negative size or stride, bad enum, K < 1, eps < 0 */
+    HC_ERR_UNSUPPORTED = 2, /* valid math, outside this library's limits (n > 8, d % 8 ...) */
+    HC_ERR_MISALIGNED = 3,  /* a pointer misses the alignment stated above */
+    HC_ERR_ALIAS = 4,       /* an output overlaps another buffer (other than Hout == H) */
+    HC_ERR_CUDA = 5,        /* the CUDA runtime reported an error at launch */
+    HC_ERR_DEVICE = 6       /* a kernel reported a device-side failure */
+} hc_status;
+
+typedef enum { HC_F32 = 0, HC_BF16 = 1 } hc_dtype;
+
+/* How the write mix gets A: given directly, or as logits L projected per
+ * token by K Sinkhorn iterations (mHC). */
+typedef enum { HC_MIX_MATRIX = 0, HC_MIX_SINKHORN_LOGITS = 1 } hc_mix_mode;
+
+/* How the read gets a: given directly, or as logits turned into weights by a
+ * softmax over the n streams (mHC). */
+typedef enum { HC_READ_WEIGHTS = 0, HC_READ_SOFTMAX_LOGITS = 1 } hc_read_mode;
+
+typedef void *hc_stream; /* cudaStream_t */
+
+/*
+ * Sinkhorn projection ("Hyper-connections (mHC)", definition paragraph: the
+ * mixing is made doubly stochastic with a few Sinkhorn iterations).
+ *   logits [T][n][n] fp32 in, out [T][n][n] fp32 out (may equal logits).
+ *   out = K x (row normalisation, column normalisation) of exp(logits).
+ *   Columns of out sum to 1 (the column pass is last); rows approach 1 as K
+ *   grows. 1 <= n <= 8, K >= 1. Both pointers 4-byte aligned, 16-byte not
+ *   needed. A standalone entry for tests and for callers that keep A.
+ */
+HC_API hc_status hc_sinkhorn(const float *logits, float *out, int64_t T, int n, int K,
+                      hc_stream stream);
+
+/*
+ * Read mix followed by the block's pre-norm RMSNorm ("Hyper-connections
+ * (mHC)": mixing before the block; Hy4 explainer, Jargon "Pre-norm").
+ *   H [T][n][d] in (dtype dt), x [T][d] out (dtype dt).
+ *   rm == HC_READ_WEIGHTS: a holds weights; HC_READ_SOFTMAX_LOGITS: logits.
+ *   a_tok_stride: 0 = one set of n for all tokens, else floats per token.
+ *   g: [d] fp32 per-channel gain, or NULL for a gain of 1.
+ *   eps >= 0, added to the mean square inside the square root.
+ */
+HC_API hc_status hc_read_rmsnorm(const void *H, void *x, hc_dtype dt, int64_t T, int n, int64_t d,
+                          hc_read_mode rm, const float *a, int64_t a_tok_stride,
+                          const float *g, float eps, hc_stream stream);
+
+/*
+ * Write mix ("Hyper-connections (mHC)": mixing after the block; Hy4 explainer,
+ * TL;DR: a block can write to one stream and leave the others intact).
+ *   H [T][n][d] and y [T][d] in, Hout [T][n][d] out, all dtype dt.
+ *   H'_j = sum_i A[i][j] H_i + b_j y.
+ *   mm == HC_MIX_MATRIX: A holds the n x n matrix (row-major, row = source);
+ *   HC_MIX_SINKHORN_LOGITS: A holds logits and K >= 1 Sinkhorn pairs project
+ *   them per token in registers (the matrix never goes to memory).
+ *   A_tok_stride / b_tok_stride: 0 = shared by all tokens, else floats per token.
+ *   Hout may equal H.
+ */
+HC_API hc_status hc_write_mix(const void *H, const void *y, void *Hout, hc_dtype dt, int64_t T, int n,
+                       int64_t d, hc_mix_mode mm, const float *A, int64_t A_tok_stride, int K,
+                       const float *b, int64_t b_tok_stride, hc_stream stream);
+
+/*
+ * Fused step: layer l's write followed by layer l+1's read + RMSNorm in one
+ * pass over HBM, so H' is not read back. Same arguments as the two calls
+ * above; the read uses the stored (rounded) H'. Hout may equal H; x_next must
+ * not overlap H, Hout or y.
+ */
+HC_API hc_status hc_write_then_read(const void *H, const void *y, void *Hout, void *x_next,
+                             hc_dtype dt, int64_t T, int n, int64_t d, hc_mix_mode mm,
+                             const float *A, int64_t A_tok_stride, int K, const float *b,
+                             int64_t b_tok_stride, hc_read_mode rm, const float *a_next,
+                             int64_t a_tok_stride, const float *g_next, float eps,
+                             hc_stream stream);
+
+/* Static English text for a status code. */
+HC_API const char *hc_status_string(hc_status st);
+
+/* Details of the calling thread's most recent failed call ("" if none). The
+ * pointer stays valid until the thread's next call into the library. */
+HC_API const char *hc_last_error(void);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+HC_API int hc_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HC_API_H */

@@ -1,0 +1,148 @@
+"""Host-side checks of the C ABI (no GPU needed):
+  - libhc_b200.so builds for sm_100a, loads, and exports every entry point
+    declared in include/*.h with the binding's signatures;
+  - argument validation refuses bad calls with the documented status before
+    anything is launched.
+The validation calls use fake device addresses, so they run in a child process
+with CUDA_VISIBLE_DEVICES="" -- even a validation bug could not launch a kernel.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import glob
+import os
+import re
+import subprocess
+import sys
+import textwrap
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _built_lib():
+    from hyper_connections_stream_b200 import build
+    return build.build()
+
+
+def _declared_entry_points():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        names |= set(re.findall(r"HC_API\s+[\w\s\*]+?\b(hc_\w+)\s*\(", src))
+    return names
+
+
+def test_library_exports_every_declared_entry_point():
+    path = _built_lib()
+    lib = C.CDLL(path)
+    declared = _declared_entry_points()
+    assert {"hc_sinkhorn", "hc_read_rmsnorm", "hc_write_mix", "hc_write_then_read",
+            "hc_status_string", "hc_last_error", "hc_version"} <= declared
+    for name in declared:
+        assert hasattr(lib, name), name
+    from hyper_connections_stream_b200 import _lib
+    assert declared <= set(_lib.SIGNATURES), declared - set(_lib.SIGNATURES)
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\sT\s(hc_\w+)", out))
+    assert exported == declared, exported ^ declared
+
+
+def test_library_is_built_for_sm100a():
+    path = _built_lib()
+    out = subprocess.run(["/usr/local/cuda/bin/cuobjdump", "--list-elf", path],
+                         capture_output=True, text=True)
+    assert "sm_100a" in out.stdout, out.stdout + out.stderr
+
+
+_CHILD = textwrap.dedent(r"""
+    import ctypes as C, json, math
+    from hyper_connections_stream_b200 import _lib as B
+    L = B.lib()
+    A16 = 0x10000          # fake, 16-byte aligned device addresses (never dereferenced)
+    def buf(i): return A16 * (i + 1) * 4096
+    res = {}
+    def call(tag, fn, *args):
+        res[tag] = (getattr(L, fn)(*args), L.hc_last_error().decode())
+    T, n, d = 8, 4, 1024
+    H, y, Ho, x, A, b, a, g = (buf(i) for i in range(8))
+    bf = B.HC_BF16
+    call("ok_T0", "hc_write_then_read", None, None, None, None, bf, 0, n, d, 0, None, 0, 0,
+         None, 0, 0, None, 0, None, 1e-6, None)
+    call("T_neg", "hc_write_mix", H, y, Ho, bf, -1, n, d, 0, A, 0, 0, b, 0, None)
+    call("n0", "hc_write_mix", H, y, Ho, bf, T, 0, d, 0, A, 0, 0, b, 0, None)
+    call("n9", "hc_write_mix", H, y, Ho, bf, T, 9, d, 0, A, 0, 0, b, 0, None)
+    call("d_ragged", "hc_write_mix", H, y, Ho, bf, T, n, 12, 0, A, 0, 0, b, 0, None)
+    call("d_f32_ok_but_null", "hc_write_mix", None, y, Ho, B.HC_F32, T, n, 12, 0, A, 0, 0, b, 0, None)
+    call("d_too_big", "hc_read_rmsnorm", H, x, bf, T, n, 32768 + 8, 0, a, 0, None, 1e-6, None)
+    call("dtype", "hc_write_mix", H, y, Ho, 7, T, n, d, 0, A, 0, 0, b, 0, None)
+    call("mixmode", "hc_write_mix", H, y, Ho, bf, T, n, d, 5, A, 0, 0, b, 0, None)
+    call("readmode", "hc_read_rmsnorm", H, x, bf, T, n, d, 3, a, 0, None, 1e-6, None)
+    call("K0", "hc_write_mix", H, y, Ho, bf, T, n, d, 1, A, 0, 0, b, 0, None)
+    call("K_huge", "hc_write_mix", H, y, Ho, bf, T, n, d, 1, A, 0, 1 << 20, b, 0, None)
+    call("stride_neg", "hc_write_mix", H, y, Ho, bf, T, n, d, 0, A, -16, 0, b, 0, None)
+    call("eps_neg", "hc_read_rmsnorm", H, x, bf, T, n, d, 0, a, 0, None, -1.0, None)
+    call("eps_nan", "hc_read_rmsnorm", H, x, bf, T, n, d, 0, a, 0, None, float("nan"), None)
+    call("eps_inf", "hc_read_rmsnorm", H, x, bf, T, n, d, 0, a, 0, None, float("inf"), None)
+    call("null_H", "hc_write_mix", None, y, Ho, bf, T, n, d, 0, A, 0, 0, b, 0, None)
+    call("null_A", "hc_write_mix", H, y, Ho, bf, T, n, d, 0, None, 0, 0, b, 0, None)
+    call("null_b", "hc_write_then_read", H, y, Ho, x, bf, T, n, d, 0, A, 0, 0, None, 0, 0, a, 0, None, 1e-6, None)
+    call("mis_H", "hc_write_mix", H + 8, y, Ho, bf, T, n, d, 0, A, 0, 0, b, 0, None)
+    call("mis_x", "hc_read_rmsnorm", H, x + 4, bf, T, n, d, 0, a, 0, None, 1e-6, None)
+    call("mis_g", "hc_read_rmsnorm", H, x, bf, T, n, d, 0, a, 0, g + 4, 1e-6, None)
+    call("mis_A", "hc_write_mix", H, y, Ho, bf, T, n, d, 0, A + 2, 0, 0, b, 0, None)
+    hb = T * n * d * 2
+    call("alias_partial", "hc_write_mix", H, y, H + 16, bf, T, n, d, 0, A, 0, 0, b, 0, None)
+    call("alias_y", "hc_write_mix", H, y, y - hb + 16, bf, T, n, d, 0, A, 0, 0, b, 0, None)
+    call("alias_x_H", "hc_write_then_read", H, y, Ho, H + hb - 16, bf, T, n, d, 0, A, 0, 0, b, 0, 0, a, 0, None, 1e-6, None)
+    call("alias_x_read", "hc_read_rmsnorm", H, H + 32, bf, T, n, d, 0, a, 0, None, 1e-6, None)
+    call("sk_n0", "hc_sinkhorn", A, A, T, 0, 20, None)
+    call("sk_K0", "hc_sinkhorn", A, A, T, 4, 0, None)
+    call("sk_null", "hc_sinkhorn", None, A, T, 4, 20, None)
+    call("sk_alias", "hc_sinkhorn", A, A + 4, T, 4, 20, None)
+    call("sk_T0", "hc_sinkhorn", None, None, 0, 4, 20, None)
+    print(json.dumps(res))
+""")
+
+
+def test_argument_validation_statuses():
+    _built_lib()
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="", PYTHONPATH=ROOT)
+    out = subprocess.run([sys.executable, "-c", _CHILD], capture_output=True, text=True, env=env,
+                         cwd=ROOT, timeout=300)
+    assert out.returncode == 0, out.stderr
+    import json
+    res = json.loads(out.stdout.strip().splitlines()[-1])
+    OK, INV, UNS, MIS, ALI = 0, 1, 2, 3, 4
+    want = {
+        "ok_T0": OK, "T_neg": INV, "n0": INV, "n9": UNS, "d_ragged": UNS,
+        "d_f32_ok_but_null": INV, "d_too_big": UNS, "dtype": INV, "mixmode": INV,
+        "readmode": INV, "K0": INV, "K_huge": UNS, "stride_neg": INV, "eps_neg": INV,
+        "eps_nan": INV, "eps_inf": INV, "null_H": INV, "null_A": INV, "null_b": INV,
+        "mis_H": MIS, "mis_x": MIS, "mis_g": MIS, "mis_A": MIS, "alias_partial": ALI,
+        "alias_y": ALI, "alias_x_H": ALI, "alias_x_read": ALI, "sk_n0": INV, "sk_K0": INV,
+        "sk_null": INV, "sk_alias": ALI, "sk_T0": OK,
+    }
+    for tag, code in want.items():
+        got, msg = res[tag]
+        assert got == code, (tag, got, code, msg)
+        if code != OK:
+            assert msg, tag  # a reason is recorded for every refusal
+
+
+def test_status_strings_and_version():
+    from hyper_connections_stream_b200 import _lib
+    L = _lib.lib()
+    for st in range(7):
+        assert L.hc_status_string(st).decode() not in ("", "unknown status")
+    assert L.hc_status_string(99).decode() == "unknown status"
+    assert L.hc_version() >= 100
+
+
+def test_binding_refuses_cpu_tensors():
+    """The binding has no CPU path: host tensors are refused, not computed."""
+    import pytest
+    import torch
+    from hyper_connections_stream_b200 import _lib
+    H = torch.zeros((2, 4, 16), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        _lib.read_rmsnorm(H, torch.ones(4))
