@@ -185,12 +185,16 @@ def run_ours(args):
     ws, rank, local = _dist_env()
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
+    hc.set_path({"auto": hc.PATH_AUTO, "pipelined": hc.PATH_PIPELINED,
+                 "register": hc.PATH_REGISTER}[args.path])
     if ws > 1:
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
-    w = WORKLOAD
+    w = dict(WORKLOAD)
+    if args.tokens:
+        w["T"] = args.tokens
     T, n, d, K = w["T"], w["n"], w["d"], w["K"]
     inp = make_inputs(w, rank, device)
     H0 = inp["H"]
@@ -246,7 +250,7 @@ def run_ours(args):
     prof = _profiled_traffic("fused_mhc_n4_d7168_bf16_T16384")
 
     # end to end through the public API with host buffers
-    e2e = run_e2e(args, inp, w, device, ws)
+    e2e = None if args.kernel_only else run_e2e(args, inp, w, device, ws)
 
     if ws > 1:
         import torch.distributed as dist
@@ -268,9 +272,11 @@ def run_ours(args):
                      "frac_of_8TBs": achieved / 8000.0},
         "e2e": e2e,
         "gpu_launches": args.steps * ws,
+        "kernel_path": args.path,
+        "device_fault": hc.device_fault(),
         "clocks": clocks,
     }
-    if ws == 1 and not args.no_cpu_baseline:
+    if ws == 1 and not (args.no_cpu_baseline or args.kernel_only):
         line["cpu_baseline"] = cpu_baseline(w, target_s=args.cpu_seconds)
     return line
 
@@ -413,6 +419,12 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-seconds", type=float, default=90.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-only", action="store_true",
+                    help="device-timed kernel only (no e2e, no CPU baseline): for profiling")
+    ap.add_argument("--path", choices=["auto", "pipelined", "register"], default="auto",
+                    help="kernel family (auto = pipelined wherever it applies)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override T (smaller cases for ncu captures)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

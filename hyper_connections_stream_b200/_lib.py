@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libhc_b200.so")
 HC_OK, HC_ERR_INVALID_ARG, HC_ERR_UNSUPPORTED, HC_ERR_MISALIGNED = 0, 1, 2, 3
 HC_ERR_ALIAS, HC_ERR_CUDA, HC_ERR_DEVICE = 4, 5, 6
 HC_F32, HC_BF16 = 0, 1
+PATH_AUTO, PATH_PIPELINED, PATH_REGISTER = 0, 1, 2
 MIX_MATRIX, MIX_SINKHORN_LOGITS = 0, 1
 READ_WEIGHTS, READ_SOFTMAX_LOGITS = 0, 1
 
@@ -33,6 +34,9 @@ SIGNATURES = {
                       _vp], _i32),
     "hc_write_then_read": ([_vp, _vp, _vp, _vp, _i32, _i64, _i32, _i64, _i32, _vp, _i64, _i32,
                             _vp, _i64, _i32, _vp, _i64, _vp, _f32, _vp], _i32),
+    "hc_set_path": ([_i32], _i32),
+    "hc_get_path": ([], _i32),
+    "hc_device_fault": ([C.POINTER(_i32), _vp], _i32),
     "hc_status_string": ([_i32], C.c_char_p),
     "hc_last_error": ([], C.c_char_p),
     "hc_version": ([], _i32),
@@ -114,6 +118,26 @@ def _streams_shape(H):
     if H.dtype not in _DT:
         raise ValueError(f"H must be float32 or bfloat16, got {H.dtype}")
     return H.shape
+
+
+def set_path(path: int) -> None:
+    """Choose the kernel family process-wide: PATH_AUTO, PATH_PIPELINED (TMA-fed
+    ring) or PATH_REGISTER (register streaming). Results are identical."""
+    _check(lib().hc_set_path(int(path)))
+
+
+def get_path() -> int:
+    return int(lib().hc_get_path())
+
+
+def device_fault(device=None) -> int:
+    """Synchronise the current stream and return (and clear) the device fault
+    word: 0 when no kernel gave up on a bounded wait."""
+    code = C.c_int(0)
+    st = lib().hc_device_fault(C.byref(code), _stream(device))
+    if st not in (HC_OK, HC_ERR_DEVICE):
+        _check(st)
+    return int(code.value)
 
 
 def sinkhorn(logits: torch.Tensor, K: int, out: torch.Tensor | None = None) -> torch.Tensor:

@@ -1,12 +1,14 @@
 """Build libhc_b200.so (the C-ABI CUDA library) in-tree for sm_100a.
 
-    python -m hyper_connections_stream_b200.build [--force] [--verbose]
+    python -m hyper_connections_stream_b200.build [--force] [--verbose] [-j N]
 
-The library links the CUDA runtime statically and exports only the C entry
-points of include/hc_api.h.
+Each translation unit under csrc/ is compiled to an object in parallel
+(nvcc -c), then linked into one shared library that links the CUDA runtime
+statically and exports only the C entry points of include/hc_api.h.
 """
 from __future__ import annotations
 
+import concurrent.futures as cf
 import glob
 import os
 import subprocess
@@ -16,40 +18,58 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
+OBJDIR = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libhc_b200.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 GENCODE = ["-gencode", "arch=compute_100a,code=sm_100a"]
-NVCC_FLAGS = [*GENCODE, "-O3", "-lineinfo", "-std=c++17", "--shared", "-Xcompiler", "-fPIC",
-              "-Xcompiler", "-fvisibility=hidden", "-cudart", "static",
-              "-I", INCLUDE, "-I", CSRC]
+COMMON = [*GENCODE, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
+          "-Xcompiler", "-fvisibility=hidden", "-I", INCLUDE, "-I", CSRC]
 
 
 def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def deps():
-    return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + \
-        sorted(glob.glob(os.path.join(INCLUDE, "*.h")))
+def headers():
+    return sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h"))
+                  + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
 def needs_build() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    return any(os.path.getmtime(f) > t for f in deps())
+    return any(os.path.getmtime(f) > t for f in sources() + headers() + [__file__])
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
+def _compile(src: str, verbose: bool) -> str:
+    obj = os.path.join(OBJDIR, os.path.basename(src)[:-3] + ".o")
+    cmd = [NVCC, *COMMON, *(["-Xptxas", "-v"] if verbose else []), "-c", src, "-o", obj]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError(f"nvcc failed on {src}:\n{r.stdout}\n{r.stderr}")
+    if verbose:
+        sys.stderr.write(r.stderr)
+    return obj
+
+
+def build(force: bool = False, verbose: bool = False, jobs: int | None = None) -> str:
     if not (force or needs_build()):
         return LIB
+    os.makedirs(OBJDIR, exist_ok=True)
+    jobs = jobs or max(1, min(len(sources()), os.cpu_count() or 1))
+    with cf.ThreadPoolExecutor(jobs) as ex:
+        objs = list(ex.map(lambda s: _compile(s, verbose), sources()))
     tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [NVCC, *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []), *sources(), "-o", tmp]
+    cmd = [NVCC, *GENCODE, "--shared", "-cudart", "static", *objs, "-o", tmp]
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)
     return LIB
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))
+    j = None
+    if "-j" in sys.argv:
+        j = int(sys.argv[sys.argv.index("-j") + 1])
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv, jobs=j))

@@ -13,14 +13,23 @@
 #include <cstdio>
 #include <cstring>
 
+#include <atomic>
+
 #include "hc_api.h"
-#include "hc_stream_kernels.cuh"
+#include "hc_launch.h"
+
+// The library's device fault word (one per device that loads the library).
+// Pipelined kernels OR a fault code into it when a bounded wait runs out.
+__device__ int g_hc_device_fault = 0;
+
+namespace hc {
 
 namespace {
-
 thread_local char g_last_error[512] = "";
+std::atomic<int> g_path{0};
+}  // namespace
 
-hc_status fail(hc_status st, const char *fmt, ...) {
+hc_status set_error(hc_status st, const char *fmt, ...) {
     va_list ap;
     va_start(ap, fmt);
     vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
@@ -28,12 +37,12 @@ hc_status fail(hc_status st, const char *fmt, ...) {
     return st;
 }
 
-hc_status check_launch(const char *what) {
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess)
-        return fail(HC_ERR_CUDA, "%s: launch failed: %s", what, cudaGetErrorString(e));
-    return HC_OK;
-}
+}  // namespace hc
+
+namespace {
+
+using hc::g_last_error;
+#define fail hc::set_error
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -47,24 +56,31 @@ bool overlap(const void *p, int64_t pb, const void *q, int64_t qb) {
 int elem_bytes(hc_dtype dt) { return dt == HC_BF16 ? 2 : 4; }
 int vec_elems(hc_dtype dt) { return dt == HC_BF16 ? 8 : 4; }
 
-struct DeviceInfo {
-    int sms = 0;
-};
-
-hc_status device_info(DeviceInfo &info) {
-    static DeviceInfo cache[64];
+// Per-device launch context: SM count and the address of this device's fault
+// word (looked up once per device, with that device current).
+hc_status launch_ctx(hc::LaunchCtx &ctx) {
+    static int sms_cache[64] = {};
+    static int *fault_cache[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return fail(HC_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
     if (dev < 0 || dev >= 64) return fail(HC_ERR_UNSUPPORTED, "device ordinal %d >= 64", dev);
-    if (cache[dev].sms == 0) {
+    if (sms_cache[dev] == 0) {
         int sms = 0;
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess)
             return fail(HC_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
-        cache[dev].sms = sms;
+        void *addr = nullptr;
+        e = cudaGetSymbolAddress(&addr, g_hc_device_fault);
+        if (e != cudaSuccess)
+            return fail(HC_ERR_CUDA, "cudaGetSymbolAddress(fault word): %s", cudaGetErrorString(e));
+        fault_cache[dev] = static_cast<int *>(addr);
+        sms_cache[dev] = sms;
     }
-    info = cache[dev];
+    ctx.device = dev;
+    ctx.sms = sms_cache[dev];
+    ctx.fault = fault_cache[dev];
+    ctx.path = hc::g_path.load(std::memory_order_relaxed);
     return HC_OK;
 }
 
@@ -131,89 +147,12 @@ hc_status check_K(const char *fn, int K) {
         if (_st != HC_OK) return _st;      \
     } while (0)
 
-// ---- launch of the streaming kernels -----------------------------------------
-
-template <int N, typename S, int KIND, int CPT>
-hc_status launch_stream_cpt(const hc::StepParams &p, int NT, int sms, cudaStream_t st) {
-    auto kern = hc::hc_stream_kernel<N, S, KIND, CPT>;
-    int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NT, 0);
-    if (e != cudaSuccess) return fail(HC_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
-    if (per_sm < 1) per_sm = 1;
-    int64_t grid = (int64_t)sms * per_sm;
-    if (grid > p.T) grid = p.T;
-    kern<<<(unsigned)grid, NT, 0, st>>>(p);
-    return check_launch("hc_stream_kernel");
-}
-
-// Pick threads per CTA (NT) and 16-byte slices per thread (CPT) for a row of
-// nvec slices: the smallest CPT whose NT fits, preferring no idle slices.
-void pick_stream_shape(int64_t nvec, bool normalises, int &NT, int &CPT) {
-    if (!normalises) {
-        // no per-thread state: one pass of up to 256 threads over the row
-        int64_t t = nvec < 256 ? nvec : 256;
-        NT = (int)((t + 31) / 32 * 32);
-        CPT = 1;
-        return;
-    }
-    static const int cpts[] = {1, 2, 4, 8};
-    int best_nt = 0, best_cpt = 8;
-    int64_t best_waste = INT64_MAX;
-    for (int cpt : cpts) {
-        int64_t nt = (nvec + cpt - 1) / cpt;
-        nt = (nt + 31) / 32 * 32;
-        if (nt > hc::kStreamMaxThreads) continue;
-        if (nt < 64 && cpt > 1) continue;  // fewer slices per thread is better here
-        const int64_t waste = nt * cpt - nvec;
-        if (waste < best_waste) {
-            best_waste = waste;
-            best_nt = (int)nt;
-            best_cpt = cpt;
-        }
-    }
-    NT = best_nt;
-    CPT = best_cpt;
-}
-
-template <int N, typename S, int KIND>
-hc_status launch_stream(const hc::StepParams &p, cudaStream_t st) {
-    DeviceInfo info;
-    HC_TRY(device_info(info));
-    constexpr int V = hc::StorageTraits<S>::V;
-    const int64_t nvec = p.d / V;
-    int NT = 0, CPT = 1;
-    pick_stream_shape(nvec, KIND != hc::KIND_WRITE, NT, CPT);
-    if (NT == 0) return fail(HC_ERR_UNSUPPORTED, "no launch shape for d = %lld", (long long)p.d);
-    if constexpr (KIND == hc::KIND_WRITE) {
-        return launch_stream_cpt<N, S, KIND, 1>(p, NT, info.sms, st);
-    } else {
-        switch (CPT) {
-            case 1: return launch_stream_cpt<N, S, KIND, 1>(p, NT, info.sms, st);
-            case 2: return launch_stream_cpt<N, S, KIND, 2>(p, NT, info.sms, st);
-            case 4: return launch_stream_cpt<N, S, KIND, 4>(p, NT, info.sms, st);
-            default: return launch_stream_cpt<N, S, KIND, 8>(p, NT, info.sms, st);
-        }
-    }
-}
-
-template <typename S, int KIND>
-hc_status dispatch_n(int n, const hc::StepParams &p, cudaStream_t st) {
-    switch (n) {
-        case 1: return launch_stream<1, S, KIND>(p, st);
-        case 2: return launch_stream<2, S, KIND>(p, st);
-        case 3: return launch_stream<3, S, KIND>(p, st);
-        case 4: return launch_stream<4, S, KIND>(p, st);
-        case 5: return launch_stream<5, S, KIND>(p, st);
-        case 6: return launch_stream<6, S, KIND>(p, st);
-        case 7: return launch_stream<7, S, KIND>(p, st);
-        default: return launch_stream<8, S, KIND>(p, st);
-    }
-}
-
 template <int KIND>
 hc_status dispatch(hc_dtype dt, int n, const hc::StepParams &p, cudaStream_t st) {
-    if (dt == HC_BF16) return dispatch_n<__nv_bfloat16, KIND>(n, p, st);
-    return dispatch_n<float, KIND>(n, p, st);
+    hc::LaunchCtx ctx{};
+    HC_TRY(launch_ctx(ctx));
+    if (dt == HC_BF16) return hc::launch_kind<__nv_bfloat16, KIND>(n, p, ctx, st);
+    return hc::launch_kind<float, KIND>(n, p, ctx, st);
 }
 
 }  // namespace
@@ -239,6 +178,32 @@ const char *hc_status_string(hc_status st) {
 
 const char *hc_last_error(void) { return g_last_error; }
 
+hc_status hc_set_path(hc_path path) {
+    g_last_error[0] = '\0';
+    if (path != HC_PATH_AUTO && path != HC_PATH_PIPELINED && path != HC_PATH_REGISTER)
+        return fail(HC_ERR_INVALID_ARG, "hc_set_path: bad path %d", (int)path);
+    hc::g_path.store((int)path, std::memory_order_relaxed);
+    return HC_OK;
+}
+
+hc_path hc_get_path(void) { return (hc_path)hc::g_path.load(std::memory_order_relaxed); }
+
+hc_status hc_device_fault(int *code, hc_stream stream) {
+    g_last_error[0] = '\0';
+    if (!code) return fail(HC_ERR_INVALID_ARG, "hc_device_fault: code is NULL");
+    hc::LaunchCtx ctx{};
+    HC_TRY(launch_ctx(ctx));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return fail(HC_ERR_CUDA, "hc_device_fault: %s", cudaGetErrorString(e));
+    int v = 0;
+    e = cudaMemcpy(&v, ctx.fault, sizeof v, cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess && v != 0) e = cudaMemset(ctx.fault, 0, sizeof v);
+    if (e != cudaSuccess) return fail(HC_ERR_CUDA, "hc_device_fault: %s", cudaGetErrorString(e));
+    *code = v;
+    return v ? fail(HC_ERR_DEVICE, "device fault code 0x%x", v) : HC_OK;
+}
+
 hc_status hc_sinkhorn(const float *logits, float *out, int64_t T, int n, int K, hc_stream stream) {
     static const char *fn = "hc_sinkhorn";
     g_last_error[0] = '\0';
@@ -252,33 +217,9 @@ hc_status hc_sinkhorn(const float *logits, float *out, int64_t T, int n, int K, 
     const int64_t bytes = T * n * n * 4;
     if (out != logits && overlap(out, bytes, logits, bytes))
         return fail(HC_ERR_ALIAS, "%s: out partially overlaps logits", fn);
-    DeviceInfo info;
-    HC_TRY(device_info(info));
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int threads = 256;
-    int tpw = 1;
-    switch (n) {
-        case 1: tpw = hc::Group<1>::TPW; break;
-        case 2: tpw = hc::Group<2>::TPW; break;
-        case 3: tpw = hc::Group<3>::TPW; break;
-        case 4: tpw = hc::Group<4>::TPW; break;
-        default: tpw = 1; break;
-    }
-    const int64_t tokens_per_cta = (int64_t)(threads / 32) * tpw;
-    int64_t grid = (T + tokens_per_cta - 1) / tokens_per_cta;
-    const int64_t gmax = (int64_t)info.sms * 8;
-    if (grid > gmax) grid = gmax;
-    switch (n) {
-        case 1: hc::hc_sinkhorn_kernel<1><<<(unsigned)grid, threads, 0, st>>>(logits, out, T, K); break;
-        case 2: hc::hc_sinkhorn_kernel<2><<<(unsigned)grid, threads, 0, st>>>(logits, out, T, K); break;
-        case 3: hc::hc_sinkhorn_kernel<3><<<(unsigned)grid, threads, 0, st>>>(logits, out, T, K); break;
-        case 4: hc::hc_sinkhorn_kernel<4><<<(unsigned)grid, threads, 0, st>>>(logits, out, T, K); break;
-        case 5: hc::hc_sinkhorn_kernel<5><<<(unsigned)grid, threads, 0, st>>>(logits, out, T, K); break;
-        case 6: hc::hc_sinkhorn_kernel<6><<<(unsigned)grid, threads, 0, st>>>(logits, out, T, K); break;
-        case 7: hc::hc_sinkhorn_kernel<7><<<(unsigned)grid, threads, 0, st>>>(logits, out, T, K); break;
-        default: hc::hc_sinkhorn_kernel<8><<<(unsigned)grid, threads, 0, st>>>(logits, out, T, K); break;
-    }
-    return check_launch(fn);
+    hc::LaunchCtx ctx{};
+    HC_TRY(launch_ctx(ctx));
+    return hc::launch_sinkhorn(logits, out, T, n, K, ctx, static_cast<cudaStream_t>(stream));
 }
 
 hc_status hc_read_rmsnorm(const void *H, void *x, hc_dtype dt, int64_t T, int n, int64_t d,

@@ -11,6 +11,12 @@
 namespace hc {
 
 constexpr int kMaxStreams = 8;
+// Largest CTA of the register-streaming kernels; with 8 slices per thread it
+// bounds d of a normalising call at 512 * 8 vectors.
+constexpr int kStreamMaxThreads = 512;
+
+// Step kinds: read + RMSNorm, write mix, fused write then read.
+enum Kind { KIND_READ = 0, KIND_WRITE = 1, KIND_FUSED = 2 };
 
 // ---------------------------------------------------------------------------
 // Storage dtype traits: one 16-byte vector = V elements.

@@ -1,0 +1,157 @@
+// hc_kernels_impl.cuh -- launch-shape selection and dispatch over n for the
+// step kernels. Included by one translation unit per (dtype, kind).
+//
+// Kernel families:
+//   pipelined (hc_pipe_kernels.cuh): TMA-fed ring, warp-specialised; used
+//     whenever at least two ring stages fit in shared memory and, for the
+//     normalising kinds, a token spans at most 8 tiles;
+//   register-streaming (hc_stream_kernels.cuh): no shared-memory staging;
+//     covers the larger d of the normalising kinds and can be forced.
+#pragma once
+
+#include "hc_launch.h"
+#include "hc_pipe_kernels.cuh"
+#include "hc_stream_kernels.cuh"
+
+namespace hc {
+
+// ---- register-streaming family ------------------------------------------------
+
+template <int N, typename S, int KIND, int CPT>
+hc_status launch_stream_cpt(const StepParams &p, int NT, const LaunchCtx &ctx, cudaStream_t st) {
+    auto kern = hc_stream_kernel<N, S, KIND, CPT>;
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NT, 0);
+    if (e != cudaSuccess) return set_error(HC_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
+    if (per_sm < 1) per_sm = 1;
+    int64_t grid = (int64_t)ctx.sms * per_sm;
+    if (grid > p.T) grid = p.T;
+    kern<<<(unsigned)grid, NT, 0, st>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return set_error(HC_ERR_CUDA, "hc_stream_kernel launch: %s", cudaGetErrorString(e));
+    return HC_OK;
+}
+
+// Threads per CTA (NT) and 16-byte slices per thread (CPT) for a row of nvec
+// slices: the least idle slices, then the fewest slices per thread.
+inline void pick_stream_shape(int64_t nvec, bool normalises, int &NT, int &CPT) {
+    if (!normalises) {
+        const int64_t t = nvec < 256 ? nvec : 256;
+        NT = (int)((t + 31) / 32 * 32);
+        CPT = 1;
+        return;
+    }
+    static const int cpts[] = {1, 2, 4, 8};
+    int best_nt = 0, best_cpt = 8;
+    int64_t best_waste = INT64_MAX;
+    for (int cpt : cpts) {
+        int64_t nt = (nvec + cpt - 1) / cpt;
+        nt = (nt + 31) / 32 * 32;
+        if (nt > kStreamMaxThreads) continue;
+        if (nt < 64 && cpt > 1) continue;
+        const int64_t waste = nt * cpt - nvec;
+        if (waste < best_waste) {
+            best_waste = waste;
+            best_nt = (int)nt;
+            best_cpt = cpt;
+        }
+    }
+    NT = best_nt;
+    CPT = best_cpt;
+}
+
+template <int N, typename S, int KIND>
+hc_status launch_stream(const StepParams &p, const LaunchCtx &ctx, cudaStream_t st) {
+    constexpr int V = StorageTraits<S>::V;
+    int NT = 0, CPT = 1;
+    pick_stream_shape(p.d / V, KIND != KIND_WRITE, NT, CPT);
+    if (NT == 0) return set_error(HC_ERR_UNSUPPORTED, "no launch shape for d = %lld", (long long)p.d);
+    if constexpr (KIND == KIND_WRITE) {
+        return launch_stream_cpt<N, S, KIND, 1>(p, NT, ctx, st);
+    } else {
+        switch (CPT) {
+            case 1: return launch_stream_cpt<N, S, KIND, 1>(p, NT, ctx, st);
+            case 2: return launch_stream_cpt<N, S, KIND, 2>(p, NT, ctx, st);
+            case 4: return launch_stream_cpt<N, S, KIND, 4>(p, NT, ctx, st);
+            default: return launch_stream_cpt<N, S, KIND, 8>(p, NT, ctx, st);
+        }
+    }
+}
+
+// ---- pipelined family -------------------------------------------------------------
+
+template <int N, typename S, int KIND>
+bool pipe_shape(const StepParams &p, PipeShape &sh) {
+    constexpr int V = StorageTraits<S>::V;
+    constexpr int ROWS = KIND != KIND_READ ? N + 1 : N;
+    sh.tile = kPipeGroupThreads * V;
+    sh.ntile = (int)((p.d + sh.tile - 1) / sh.tile);
+    sh.stage_bytes = ROWS * sh.tile * (int)sizeof(S);
+    int stages = (kSmemLimit - pipe_fixed_bytes(N, 0)) / (sh.stage_bytes + 16);
+    if (stages > kMaxStages) stages = kMaxStages;
+    sh.stages = stages;
+    if (stages < 2) return false;
+    if (KIND != KIND_WRITE && sh.ntile > 8) return false;
+    return true;
+}
+
+template <int N, typename S, int KIND, int HT>
+hc_status launch_pipe_ht(const StepParams &p, const PipeShape &sh, const LaunchCtx &ctx,
+                         cudaStream_t st) {
+    auto kern = hc_pipe_kernel<N, S, KIND, HT>;
+    const int smem = sh.stages * sh.stage_bytes + pipe_fixed_bytes(N, sh.stages);
+    static int configured[64] = {};  // largest dynamic smem opted in so far, per device
+    if (ctx.device < 0 || ctx.device >= 64)
+        return set_error(HC_ERR_UNSUPPORTED, "device ordinal %d >= 64", ctx.device);
+    if (smem > configured[ctx.device]) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess)
+            return set_error(HC_ERR_CUDA, "cudaFuncSetAttribute(%d B smem): %s", smem,
+                             cudaGetErrorString(e));
+        configured[ctx.device] = smem;
+    }
+    int64_t grid = ctx.sms;
+    if (grid > p.T) grid = p.T;
+    kern<<<(unsigned)grid, kPipeThreads, smem, st>>>(p, sh, ctx.fault);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return set_error(HC_ERR_CUDA, "hc_pipe_kernel launch: %s", cudaGetErrorString(e));
+    return HC_OK;
+}
+
+template <int N, typename S, int KIND>
+hc_status launch_n(const StepParams &p, const LaunchCtx &ctx, cudaStream_t st) {
+    PipeShape sh{};
+    const bool pipe_ok = pipe_shape<N, S, KIND>(p, sh);
+    if (ctx.path == 1 && !pipe_ok)
+        return set_error(HC_ERR_UNSUPPORTED, "pipelined kernels do not cover d = %lld here",
+                         (long long)p.d);
+    if (ctx.path == 2 || !pipe_ok) {
+        if (KIND != KIND_WRITE && p.d > (int64_t)kStreamMaxThreads * 8 * StorageTraits<S>::V)
+            return set_error(HC_ERR_UNSUPPORTED, "d = %lld too large", (long long)p.d);
+        return launch_stream<N, S, KIND>(p, ctx, st);
+    }
+    if constexpr (KIND == KIND_WRITE) {
+        return launch_pipe_ht<N, S, KIND, 1>(p, sh, ctx, st);
+    } else {
+        if (sh.ntile <= 1) return launch_pipe_ht<N, S, KIND, 1>(p, sh, ctx, st);
+        if (sh.ntile <= 2) return launch_pipe_ht<N, S, KIND, 2>(p, sh, ctx, st);
+        if (sh.ntile <= 4) return launch_pipe_ht<N, S, KIND, 4>(p, sh, ctx, st);
+        return launch_pipe_ht<N, S, KIND, 8>(p, sh, ctx, st);
+    }
+}
+
+template <typename S, int KIND>
+hc_status launch_kind(int n, const StepParams &p, const LaunchCtx &ctx, cudaStream_t st) {
+    switch (n) {
+        case 1: return launch_n<1, S, KIND>(p, ctx, st);
+        case 2: return launch_n<2, S, KIND>(p, ctx, st);
+        case 3: return launch_n<3, S, KIND>(p, ctx, st);
+        case 4: return launch_n<4, S, KIND>(p, ctx, st);
+        case 5: return launch_n<5, S, KIND>(p, ctx, st);
+        case 6: return launch_n<6, S, KIND>(p, ctx, st);
+        case 7: return launch_n<7, S, KIND>(p, ctx, st);
+        default: return launch_n<8, S, KIND>(p, ctx, st);
+    }
+}
+
+}  // namespace hc

@@ -19,10 +19,6 @@
 
 namespace hc {
 
-enum Kind { KIND_READ = 0, KIND_WRITE = 1, KIND_FUSED = 2 };
-
-constexpr int kStreamMaxThreads = 512;
-
 // Shared memory of the streaming kernels (static size, bounded by n <= 8).
 constexpr int kPrepTokens = 32;  // parameter slots prepared per batch (max)
 

@@ -1,0 +1,116 @@
+// hc_sync.cuh -- mbarrier, bulk-copy (TMA, non-multicast) and bounded-wait
+// primitives for the pipelined HC kernels (sm_100a, inline PTX).
+//
+// Every wait in these kernels is bounded: it gives up after kWaitLimitNs of
+// %globaltimer time (or as soon as another thread of the CTA has given up),
+// records a fault code in the fault word it was given and lets the caller leave its
+// loop. No wait can hang the GPU.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace hc {
+
+// Fault codes a kernel ORs into the library's device fault word (passed to
+// the kernel as `fault`; the host reads and clears it with hc_device_fault()).
+enum DeviceFault : int {
+    FAULT_WAIT_FULL = 1,    // a consumer waited too long for a tile
+    FAULT_WAIT_EMPTY = 2,   // the producer waited too long for a free stage
+    FAULT_WAIT_PARAM = 4,   // a parameter slot wait ran out
+    FAULT_WAIT_REDUCE = 8,  // a group reduction wait ran out
+    FAULT_WAIT_DRAIN = 16,  // copies still in flight at exit after the limit
+    FAULT_SELFTEST = 32     // the bounded-wait self-test's deliberate time-out
+};
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+
+// Make barrier initialisation visible to the async (bulk-copy) proxy.
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(
+                     smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase of `bar` with the given parity to complete. Returns false
+// if the CTA's abort flag is raised or the time limit passes (then the fault
+// code is recorded and the abort flag raised for the rest of the CTA).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
+                                                  volatile int *abort_flag, int *fault,
+                                                  int fault_code) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 0u) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                atomicOr(fault, fault_code);
+                return false;
+            }
+        }
+    }
+}
+
+// Same, ignoring the abort flag (used to drain copies in flight before exit).
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity, int *fault) {
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 63u && global_timer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(fault, FAULT_WAIT_DRAIN);
+            return false;
+        }
+    }
+}
+
+// Bulk copy global -> shared of `bytes` (multiple of 16, both addresses
+// 16-byte aligned), completing as transaction bytes on `bar`. This is the
+// plain (non-multicast) form: the source is this GPU's own memory.
+__device__ __forceinline__ void bulk_load(void *dst_smem, const void *src_gmem, uint32_t bytes,
+                                          uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_addr(dst_smem)), "l"(src_gmem), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+}  // namespace hc

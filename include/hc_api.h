@@ -139,6 +139,32 @@ HC_API hc_status hc_write_then_read(const void *H, const void *y, void *Hout, vo
                              int64_t a_tok_stride, const float *g_next, float eps,
                              hc_stream stream);
 
+/*
+ * Kernel family used by the step calls (process-wide; default HC_PATH_AUTO).
+ *   HC_PATH_PIPELINED: warp-specialised kernels fed by bulk copies (TMA) into
+ *     a shared-memory ring; the automatic choice wherever it applies (two or
+ *     more ring stages fit and, for calls that normalise, d <= 8 tiles of
+ *     1792 bf16 / 896 fp32 elements). Forcing it where it does not apply
+ *     returns HC_ERR_UNSUPPORTED.
+ *   HC_PATH_REGISTER: register-streaming kernels (no staging); the automatic
+ *     choice for the larger d.
+ * Both families compute bit-identical results.
+ */
+typedef enum { HC_PATH_AUTO = 0, HC_PATH_PIPELINED = 1, HC_PATH_REGISTER = 2 } hc_path;
+HC_API hc_status hc_set_path(hc_path path);
+HC_API hc_path hc_get_path(void);
+
+/*
+ * Device-side failure report. The pipelined kernels bound every wait on
+ * their shared-memory barriers (2 s of GPU time); a wait that runs out makes
+ * the kernel stop, drain its copies in flight and OR a code into the current
+ * device's fault word instead of hanging. This call SYNCHRONISES `stream`,
+ * reads and clears that word into *code, and returns HC_ERR_DEVICE if it was
+ * non-zero (HC_OK otherwise). Codes: 1 tile wait, 2 free-stage wait,
+ * 4 parameter wait, 8 reduction wait, 16 drain at exit, 32 self-test.
+ */
+HC_API hc_status hc_device_fault(int *code, hc_stream stream);
+
 /* Static English text for a status code. */
 HC_API const char *hc_status_string(hc_status st);
 

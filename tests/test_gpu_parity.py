@@ -25,15 +25,22 @@ pytestmark = pytest.mark.gpu
 EPS = 1e-6
 
 
-@pytest.fixture(scope="module")
-def hc():
+@pytest.fixture(scope="module", params=["auto", "register"])
+def hc(request):
+    """The binding, with the kernel family chosen automatically (pipelined
+    wherever it applies) or forced to register streaming. After each family's
+    tests no kernel may have given up on a bounded wait."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from hyper_connections_stream_b200 import build
     build.build()
     import hyper_connections_stream_b200._lib as L
     L.lib()
-    return L
+    L.set_path(L.PATH_AUTO if request.param == "auto" else L.PATH_REGISTER)
+    yield L
+    torch.cuda.synchronize()
+    assert L.device_fault() == 0
+    L.set_path(L.PATH_AUTO)
 
 
 # ---------------------------------------------------------------------------
