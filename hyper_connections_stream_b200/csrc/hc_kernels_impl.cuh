@@ -3,8 +3,8 @@
 //
 // Kernel families:
 //   pipelined (hc_pipe_kernels.cuh): TMA-fed ring, warp-specialised; used
-//     whenever at least two ring stages fit in shared memory and, for the
-//     normalising kinds, a token spans at most 8 tiles;
+//     whenever at least two ring stages fit in shared memory next to the
+//     groups' fp32 rows of h (normalising kinds);
 //   register-streaming (hc_stream_kernels.cuh): no shared-memory staging;
 //     covers the larger d of the normalising kinds and can be forced.
 #pragma once
@@ -81,25 +81,29 @@ hc_status launch_stream(const StepParams &p, const LaunchCtx &ctx, cudaStream_t 
 // ---- pipelined family -------------------------------------------------------------
 
 template <int N, typename S, int KIND>
-bool pipe_shape(const StepParams &p, PipeShape &sh) {
+bool pipe_shape(const StepParams &p, PipeShape &sh, int &smem) {
     constexpr int V = StorageTraits<S>::V;
     constexpr int ROWS = KIND != KIND_READ ? N + 1 : N;
+    const int64_t d_h = KIND != KIND_WRITE ? p.d : 0;
     sh.tile = kPipeGroupThreads * V;
-    sh.ntile = (int)((p.d + sh.tile - 1) / sh.tile);
+    const int64_t ntile = (p.d + sh.tile - 1) / sh.tile;
+    if (ntile > (1 << 20)) return false;
+    sh.ntile = (int)ntile;
     sh.stage_bytes = ROWS * sh.tile * (int)sizeof(S);
-    int stages = (kSmemLimit - pipe_fixed_bytes(N, 0)) / (sh.stage_bytes + 16);
-    if (stages > kMaxStages) stages = kMaxStages;
-    sh.stages = stages;
-    if (stages < 2) return false;
-    if (KIND != KIND_WRITE && sh.ntile > 8) return false;
+    // one ring per consumer group, at least two stages each
+    int64_t per_group = (kSmemLimit - pipe_fixed_bytes(N, 0, d_h)) /
+                        ((int64_t)kPipeGroups * (sh.stage_bytes + 16));
+    if (per_group > kMaxStages / kPipeGroups) per_group = kMaxStages / kPipeGroups;
+    if (per_group < 2) return false;
+    sh.stages = (int)(per_group * kPipeGroups);
+    smem = (int)((int64_t)sh.stages * sh.stage_bytes + pipe_fixed_bytes(N, sh.stages, d_h));
     return true;
 }
 
-template <int N, typename S, int KIND, int HT>
-hc_status launch_pipe_ht(const StepParams &p, const PipeShape &sh, const LaunchCtx &ctx,
-                         cudaStream_t st) {
-    auto kern = hc_pipe_kernel<N, S, KIND, HT>;
-    const int smem = sh.stages * sh.stage_bytes + pipe_fixed_bytes(N, sh.stages);
+template <int N, typename S, int KIND>
+hc_status launch_pipe(const StepParams &p, const PipeShape &sh, int smem, const LaunchCtx &ctx,
+                      cudaStream_t st) {
+    auto kern = hc_pipe_kernel<N, S, KIND>;
     static int configured[64] = {};  // largest dynamic smem opted in so far, per device
     if (ctx.device < 0 || ctx.device >= 64)
         return set_error(HC_ERR_UNSUPPORTED, "device ordinal %d >= 64", ctx.device);
@@ -121,7 +125,8 @@ hc_status launch_pipe_ht(const StepParams &p, const PipeShape &sh, const LaunchC
 template <int N, typename S, int KIND>
 hc_status launch_n(const StepParams &p, const LaunchCtx &ctx, cudaStream_t st) {
     PipeShape sh{};
-    const bool pipe_ok = pipe_shape<N, S, KIND>(p, sh);
+    int smem = 0;
+    const bool pipe_ok = pipe_shape<N, S, KIND>(p, sh, smem);
     if (ctx.path == 1 && !pipe_ok)
         return set_error(HC_ERR_UNSUPPORTED, "pipelined kernels do not cover d = %lld here",
                          (long long)p.d);
@@ -130,14 +135,7 @@ hc_status launch_n(const StepParams &p, const LaunchCtx &ctx, cudaStream_t st) {
             return set_error(HC_ERR_UNSUPPORTED, "d = %lld too large", (long long)p.d);
         return launch_stream<N, S, KIND>(p, ctx, st);
     }
-    if constexpr (KIND == KIND_WRITE) {
-        return launch_pipe_ht<N, S, KIND, 1>(p, sh, ctx, st);
-    } else {
-        if (sh.ntile <= 1) return launch_pipe_ht<N, S, KIND, 1>(p, sh, ctx, st);
-        if (sh.ntile <= 2) return launch_pipe_ht<N, S, KIND, 2>(p, sh, ctx, st);
-        if (sh.ntile <= 4) return launch_pipe_ht<N, S, KIND, 4>(p, sh, ctx, st);
-        return launch_pipe_ht<N, S, KIND, 8>(p, sh, ctx, st);
-    }
+    return launch_pipe<N, S, KIND>(p, sh, smem, ctx, st);
 }
 
 template <typename S, int KIND>

@@ -14,6 +14,9 @@ namespace hc {
 
 // Fault codes a kernel ORs into the library's device fault word (passed to
 // the kernel as `fault`; the host reads and clears it with hc_device_fault()).
+// A parity wait is only meaningful while the waiter is at most one phase
+// ahead of the barrier; the kernels guarantee it by giving every barrier a
+// single consumer that takes the barrier's phases in order.
 enum DeviceFault : int {
     FAULT_WAIT_FULL = 1,    // a consumer waited too long for a tile
     FAULT_WAIT_EMPTY = 2,   // the producer waited too long for a free stage
@@ -62,6 +65,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Non-blocking test: has the phase of `bar` with this parity completed?
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(smem_addr(bar)), "r"(parity)
