@@ -100,12 +100,14 @@ __device__ __forceinline__ void load_gain(const float *g, int64_t k, float (&gv)
 }
 
 // ---------------------------------------------------------------------------
-// Lane groups for the per-token n x n parameters.
+// Per-token n x n parameters, prepared by lane groups.
 //
 // A warp is split into groups of GL lanes; each group owns one token, and
 // lane q of a group holds elements e = q + GL * r (r < EPL) of the row-major
-// n x n matrix. GL is the power of two >= n*n capped at 32, so n <= 4 packs
-// several tokens per warp and n = 6..8 holds two elements per lane.
+// n x n matrix, so every lane performs one (or two) of the n*n divisions of
+// a pass in parallel. Row and column sums read the group's values from a
+// small per-warp shared-memory buffer (kGroupScratch floats), where the n
+// loads of a sum are independent and overlap.
 // ---------------------------------------------------------------------------
 template <int N> struct Group {
     static constexpr int NN = N * N;
@@ -114,83 +116,76 @@ template <int N> struct Group {
     static constexpr int EPL = (NN + GL - 1) / GL;
     static constexpr int TPW = 32 / GL;  // tokens per warp
 };
+constexpr int kGroupScratch = 64;  // floats per warp: TPW * n * n <= 64 for n <= 8
 
-// Value of element `ep` of this lane's group (all 32 lanes must call).
+// Sinkhorn projection of the group's matrix (all 32 lanes call with the same
+// K): M = exp(L); K times { divide every row by its sum; divide every column
+// by its sum }. Sums run in index order starting from +0 and divisions are
+// IEEE (__fdiv_rn), so every element sees a fixed sequence of correctly
+// rounded operations. `scratch` is this warp's kGroupScratch floats.
 template <int N>
-__device__ __forceinline__ float group_fetch(const float (&m)[Group<N>::EPL], int base, int ep) {
-    constexpr int GL = Group<N>::GL;
-    const int src = base + (ep & (GL - 1));
-    float v0 = __shfl_sync(0xffffffffu, m[0], src);
-    if constexpr (Group<N>::EPL == 1) {
-        return v0;
-    } else {
-        float v1 = __shfl_sync(0xffffffffu, m[1], src);
-        return (ep >= GL) ? v1 : v0;
-    }
-}
-
-// Sinkhorn projection of the group's matrix, in place: m = exp(L) on entry
-// is NOT assumed; the caller passes the logits and this computes
-//   M = exp(L); K times { rows /= row sums; columns /= column sums }.
-// Sums run in index order starting from +0, divisions are IEEE (__fdiv_rn),
-// so the operation sequence per element is fixed. All lanes of the warp call
-// this with the same K.
-template <int N>
-__device__ __forceinline__ void group_sinkhorn(float (&m)[Group<N>::EPL], int lane, int K) {
+__device__ __forceinline__ void group_sinkhorn(float (&m)[Group<N>::EPL], float *scratch, int lane,
+                                               int K) {
     constexpr int NN = N * N, GL = Group<N>::GL, EPL = Group<N>::EPL;
     const int q = lane & (GL - 1);
-    const int base = lane & ~(GL - 1);
-#pragma unroll
-    for (int r = 0; r < EPL; ++r) m[r] = expf(m[r]);
-    int row[EPL], col[EPL];
+    float *buf = scratch + (lane / GL) * NN;  // this group's matrix
+    int e[EPL], row[EPL], col[EPL];
+    bool own[EPL];
 #pragma unroll
     for (int r = 0; r < EPL; ++r) {
-        int e = q + GL * r;
-        e = e < NN ? e : NN - 1;  // idle lanes shadow the last element
-        row[r] = e / N;
-        col[r] = e - (e / N) * N;
+        e[r] = q + GL * r;
+        own[r] = e[r] < NN;
+        const int ec = own[r] ? e[r] : NN - 1;  // idle lanes shadow the last element
+        row[r] = ec / N;
+        col[r] = ec - row[r] * N;
+        m[r] = expf(m[r]);
     }
     for (int it = 0; it < K; ++it) {
-        float s[EPL];
 #pragma unroll
-        for (int r = 0; r < EPL; ++r) {
-            float acc = 0.0f;
+        for (int pass = 0; pass < 2; ++pass) {
 #pragma unroll
-            for (int jj = 0; jj < N; ++jj) acc = __fadd_rn(acc, group_fetch<N>(m, base, row[r] * N + jj));
-            s[r] = acc;
+            for (int r = 0; r < EPL; ++r)
+                if (own[r]) buf[e[r]] = m[r];
+            __syncwarp();
+            float s[EPL];
+#pragma unroll
+            for (int r = 0; r < EPL; ++r) {
+                float v[N];
+#pragma unroll
+                for (int k = 0; k < N; ++k) v[k] = pass == 0 ? buf[row[r] * N + k] : buf[k * N + col[r]];
+                float acc = 0.0f;
+#pragma unroll
+                for (int k = 0; k < N; ++k) acc = __fadd_rn(acc, v[k]);
+                s[r] = acc;
+            }
+            __syncwarp();
+#pragma unroll
+            for (int r = 0; r < EPL; ++r) m[r] = __fdiv_rn(m[r], s[r]);
         }
-#pragma unroll
-        for (int r = 0; r < EPL; ++r) m[r] = __fdiv_rn(m[r], s[r]);
-#pragma unroll
-        for (int r = 0; r < EPL; ++r) {
-            float acc = 0.0f;
-#pragma unroll
-            for (int ii = 0; ii < N; ++ii) acc = __fadd_rn(acc, group_fetch<N>(m, base, ii * N + col[r]));
-            s[r] = acc;
-        }
-#pragma unroll
-        for (int r = 0; r < EPL; ++r) m[r] = __fdiv_rn(m[r], s[r]);
     }
 }
 
 // Softmax over the n read logits of the group's token. Lane q < N holds l_q
-// on entry and a_q on exit. Max and sum in index order.
+// on entry and a_q on exit; max and sum in index order.
 template <int N>
-__device__ __forceinline__ float group_softmax(float l, int lane) {
+__device__ __forceinline__ float group_softmax(float l, float *scratch, int lane) {
     constexpr int GL = Group<N>::GL;
     const int q = lane & (GL - 1);
-    const int base = lane & ~(GL - 1);
-    float mx = __shfl_sync(0xffffffffu, l, base);
+    float *buf = scratch + (lane / GL) * N;
+    if (q < N) buf[q] = l;
+    __syncwarp();
+    float v[N];
 #pragma unroll
-    for (int i = 1; i < N; ++i) {
-        float v = __shfl_sync(0xffffffffu, l, base + i);
-        if (v > mx) mx = v;
-    }
-    float ex = (q < N) ? expf(__fsub_rn(l, mx)) : 0.0f;
+    for (int k = 0; k < N; ++k) v[k] = buf[k];
+    __syncwarp();
+    float mx = v[0];
+#pragma unroll
+    for (int k = 1; k < N; ++k)
+        if (v[k] > mx) mx = v[k];
     float s = 0.0f;
 #pragma unroll
-    for (int i = 0; i < N; ++i) s = __fadd_rn(s, __shfl_sync(0xffffffffu, ex, base + i));
-    return __fdiv_rn(ex, s);
+    for (int k = 0; k < N; ++k) s = __fadd_rn(s, expf(__fsub_rn(v[k], mx)));
+    return __fdiv_rn(expf(__fsub_rn(l, mx)), s);
 }
 
 // ---------------------------------------------------------------------------
@@ -217,16 +212,19 @@ struct StepParams {
 };
 
 // Fill the shared-memory parameter block for TB tokens of this CTA's token
-// sequence (token of slot tt = first + tt * step). Every warp takes TPW
-// tokens; lane groups compute Sinkhorn / softmax in registers.
+// sequence (token of slot tt = first + tt * step): every warp takes TPW
+// slots at a time with its lane groups. sA holds A row-major (row = source
+// stream). `scratch` holds kGroupScratch floats per warp.
 template <int N, bool WRITE, bool READ>
 __device__ __forceinline__ void prepare_params(const StepParams &p, int64_t first, int64_t step,
-                                               int TB, float *sA, float *sb, float *sa) {
+                                               int TB, float *sA, float *sb, float *sa,
+                                               float *scratch) {
     constexpr int NN = N * N, GL = Group<N>::GL, EPL = Group<N>::EPL, TPW = Group<N>::TPW;
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int nwarps = blockDim.x >> 5;
     const int q = lane & (GL - 1);
+    float *wscratch = scratch + warp * kGroupScratch;
     for (int slot0 = warp * TPW; slot0 < TB; slot0 += nwarps * TPW) {
         const int tt = slot0 + lane / GL;  // this group's slot
         const int64_t t = first + (int64_t)tt * step;
@@ -238,7 +236,7 @@ __device__ __forceinline__ void prepare_params(const StepParams &p, int64_t firs
                 const int e = q + GL * r;
                 m[r] = (live && e < NN) ? p.A[t * p.A_s + e] : 0.0f;
             }
-            if (p.mix_logits) group_sinkhorn<N>(m, lane, p.K);  // warp-uniform branch
+            if (p.mix_logits) group_sinkhorn<N>(m, wscratch, lane, p.K);  // warp-uniform branch
             if (live) {
 #pragma unroll
                 for (int r = 0; r < EPL; ++r) {
@@ -250,7 +248,7 @@ __device__ __forceinline__ void prepare_params(const StepParams &p, int64_t firs
         }
         if constexpr (READ) {
             float l = (live && q < N) ? p.a[t * p.a_s + q] : 0.0f;
-            if (p.read_logits) l = group_softmax<N>(l, lane);
+            if (p.read_logits) l = group_softmax<N>(l, wscratch, lane);
             if (live && q < N) sa[tt * N + q] = l;
         }
     }

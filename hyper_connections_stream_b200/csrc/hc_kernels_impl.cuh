@@ -82,7 +82,7 @@ hc_status launch_stream(const StepParams &p, const LaunchCtx &ctx, cudaStream_t 
 
 template <int N, typename S, int KIND>
 bool pipe_shape(const StepParams &p, PipeShape &sh, int &smem) {
-    constexpr int V = StorageTraits<S>::V;
+    constexpr int V = pipe_vec_elems<N, S>();
     constexpr int ROWS = KIND != KIND_READ ? N + 1 : N;
     const int64_t d_h = KIND != KIND_WRITE ? p.d : 0;
     sh.tile = kPipeGroupThreads * V;

@@ -37,18 +37,30 @@ namespace hc {
 #ifndef HC_PIPE_GROUP_WARPS
 #define HC_PIPE_GROUP_WARPS 7
 #endif
+#ifndef HC_PIPE_L2_HINT
+#define HC_PIPE_L2_HINT 0
+#endif
 constexpr int kPipeGroups = HC_PIPE_GROUPS;
 constexpr int kPipeGroupWarps = HC_PIPE_GROUP_WARPS;
 constexpr int kPipeGroupThreads = kPipeGroupWarps * 32;
 constexpr int kPipeThreads = 64 + kPipeGroups * kPipeGroupThreads;
-constexpr int kParamSlotsPerGroup = 8;
-constexpr int kParamSlots = kParamSlotsPerGroup * kPipeGroups;
+// The parameter warp prepares one lane group's worth of tokens at a time
+// (32 / GL: 2 for n = 3, 4; 1 for n >= 5); each group's slot ring holds at
+// least 8 of its tokens, and two batches, so preparation runs ahead.
+__host__ __device__ constexpr int pipe_param_batch(int n) {
+    return n * n <= 1 ? 32 : n * n <= 2 ? 16 : n * n <= 4 ? 8 : n * n <= 8 ? 4 : n * n <= 16 ? 2 : 1;
+}
+__host__ __device__ constexpr int pipe_param_slots_per_group(int n) {
+    return (((2 * pipe_param_batch(n) + kPipeGroups - 1) / kPipeGroups > 8
+                 ? (2 * pipe_param_batch(n) + kPipeGroups - 1) / kPipeGroups
+                 : 8) + 1) & ~1;  // even
+}
 constexpr int kMaxStages = 32;
 constexpr int kSmemLimit = 232448;  // 227 KB opt-in dynamic shared memory per CTA
 
 struct PipeShape {
     int stages;       // stages in all (kPipeGroups rings of stages / kPipeGroups)
-    int tile;         // elements of d per tile (= kPipeGroupThreads * V)
+    int tile;         // elements of d per tile (= kPipeGroupThreads * pipe_vec_elems)
     int ntile;        // tiles per token
     int stage_bytes;  // bytes of one stage
 };
@@ -58,35 +70,79 @@ struct PipeShape {
 // normalising kinds, each group's fp32 row h[d] (d_h = d, else 0).
 __host__ __device__ constexpr int64_t pipe_fixed_bytes(int n, int stages, int64_t d_h) {
     return (int64_t)stages * 16                        // full + empty barriers
-           + kParamSlots * 16                          // param full + empty
+           + kPipeGroups * pipe_param_slots_per_group(n) * 16  // param full + empty
            + (kPipeGroups + 1) / 2 * 16                // group reduction barriers
-           + kParamSlots * (n * n + 2 * n) * 4         // parameter slots
+           + kPipeGroups * pipe_param_slots_per_group(n) * (n * n + 2 * n) * 4  // slots
            + kPipeGroups * 2 * kPipeGroupWarps * 8     // reduction partials
            + 16                                        // abort flag (padded)
+           + kGroupScratch * 4                         // parameter warp scratch
            + (int64_t)kPipeGroups * ((d_h * 4 + 15) / 16 * 16);  // h rows
 }
 
-template <typename S> struct SmemVec;
-template <> struct SmemVec<float> {
-    static __device__ __forceinline__ void load(const unsigned char *p, float (&v)[4]) {
+// Elements of d one consumer thread handles per tile: a 16-byte vector, or
+// half of one (8 bytes) for bf16 with n > 4, which keeps the n widened input
+// rows within the register budget.
+template <int N, typename S>
+__host__ __device__ constexpr int pipe_vec_elems() {
+    return (sizeof(S) == 2 && N > 4) ? 4 : StorageTraits<S>::V;
+}
+
+// Shared-memory loads and streaming global stores of VE storage elements.
+template <typename S, int VE> struct VecIO;
+template <> struct VecIO<float, 4> {
+    static __device__ __forceinline__ void load_smem(const unsigned char *p, float (&v)[4]) {
         const float4 q = *reinterpret_cast<const float4 *>(p);
         v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
     }
+    static __device__ __forceinline__ void store(float *p, const float (&v)[4], float (&stored)[4]) {
+        store_vec_cs(p, v, stored);
+    }
+    static __device__ __forceinline__ void store(float *p, const float (&v)[4]) { store_vec_cs(p, v); }
 };
-template <> struct SmemVec<__nv_bfloat16> {
-    static __device__ __forceinline__ void load(const unsigned char *p, float (&v)[8]) {
+template <> struct VecIO<__nv_bfloat16, 8> {
+    static __device__ __forceinline__ void load_smem(const unsigned char *p, float (&v)[8]) {
         const uint4 q = *reinterpret_cast<const uint4 *>(p);
         widen_bf16x2(q.x, v[0], v[1]);
         widen_bf16x2(q.y, v[2], v[3]);
         widen_bf16x2(q.z, v[4], v[5]);
         widen_bf16x2(q.w, v[6], v[7]);
     }
+    static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float (&v)[8],
+                                                 float (&stored)[8]) {
+        store_vec_cs(p, v, stored);
+    }
+    static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float (&v)[8]) {
+        store_vec_cs(p, v);
+    }
+};
+template <> struct VecIO<__nv_bfloat16, 4> {
+    static __device__ __forceinline__ void load_smem(const unsigned char *p, float (&v)[4]) {
+        const uint2 q = *reinterpret_cast<const uint2 *>(p);
+        widen_bf16x2(q.x, v[0], v[1]);
+        widen_bf16x2(q.y, v[2], v[3]);
+    }
+    static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float (&v)[4],
+                                                 float (&stored)[4]) {
+        uint2 q;
+        q.x = pack_bf16x2_rn(v[0], v[1]);
+        q.y = pack_bf16x2_rn(v[2], v[3]);
+        __stcs(reinterpret_cast<uint2 *>(p), q);
+        widen_bf16x2(q.x, stored[0], stored[1]);
+        widen_bf16x2(q.y, stored[2], stored[3]);
+    }
+    static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float (&v)[4]) {
+        uint2 q;
+        q.x = pack_bf16x2_rn(v[0], v[1]);
+        q.y = pack_bf16x2_rn(v[2], v[3]);
+        __stcs(reinterpret_cast<uint2 *>(p), q);
+    }
 };
 
 template <int N, typename S, int KIND>
 __global__ void __launch_bounds__(kPipeThreads, 1)
 hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
-    constexpr int V = StorageTraits<S>::V;
+    constexpr int V = pipe_vec_elems<N, S>();
+    constexpr int VB = V * (int)sizeof(S);  // bytes per thread per row of a tile
     constexpr int NN = N * N;
     constexpr bool WRITE = KIND != KIND_READ;
     constexpr bool READ = KIND != KIND_WRITE;
@@ -94,7 +150,9 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
     constexpr int PSTRIDE = NN + 2 * N;  // A transposed (column j at j*N) | b | a
     constexpr int GW = kPipeGroupWarps;
     constexpr int NG = kPipeGroups;
-    constexpr int PSG = kParamSlotsPerGroup;
+    constexpr int PSG = pipe_param_slots_per_group(N);
+    constexpr int kParamSlots = NG * PSG;
+    constexpr int PB = pipe_param_batch(N);
 
     extern __shared__ __align__(128) unsigned char smem[];
     unsigned char *ring = smem;
@@ -107,7 +165,8 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
     double *sred = reinterpret_cast<double *>(params + kParamSlots * PSTRIDE);
     int *abort_word = reinterpret_cast<int *>(sred + NG * 2 * GW);
     volatile int *abort_flag = abort_word;
-    float *hrow_base = reinterpret_cast<float *>(abort_word + 4);  // 16-byte aligned
+    float *pscratch = reinterpret_cast<float *>(abort_word + 4);  // parameter warp scratch
+    float *hrow_base = pscratch + kGroupScratch;                   // 16-byte aligned
     const int64_t d = p.d;
     const int64_t hrow_stride = READ ? (d + 3) / 4 * 4 : 0;  // floats per group row
     const int SG = sh.stages / NG;  // stages per group ring
@@ -140,56 +199,74 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
         if (lane != 0) return;
         const S *H = static_cast<const S *>(p.H);
         const S *Y = static_cast<const S *>(p.y);
-        int64_t nq[NG], qend[NG];  // tiles issued / to issue, per group ring
+        // per group ring: tiles issued, tiles to issue, and the ring position,
+        // the phase and the (token ordinal, tile) of the next tile
+        int64_t nq[NG], qend[NG], mr[NG];
+        int slot_r[NG], tile_r[NG];
+        uint32_t ph_r[NG];
 #pragma unroll
         for (int r = 0; r < NG; ++r) {
             nq[r] = 0;
             qend[r] = (M > r ? (M - 1 - r) / NG + 1 : 0) * (int64_t)ntile;
+            mr[r] = r;
+            slot_r[r] = 0;
+            tile_r[r] = 0;
+            ph_r[r] = 0;
         }
         uint64_t idle_since = 0;
-        uint32_t idle_spins = 0;
+        uint32_t backoff = 32;
+        [[maybe_unused]] const uint64_t policy = HC_PIPE_L2_HINT ? l2_policy_evict_first() : 0;
+        auto load = [&](void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+            if constexpr (HC_PIPE_L2_HINT) bulk_load_hint(dst, src, bytes, bar, policy);
+            else bulk_load(dst, src, bytes, bar);
+        };
         for (;;) {
             bool pending = false, progressed = false;
 #pragma unroll
             for (int r = 0; r < NG; ++r) {
-                const int64_t qr = nq[r];
-                if (qr >= qend[r]) continue;
+                if (nq[r] >= qend[r]) continue;
                 pending = true;
-                const int s = r * SG + (int)(qr % SG);
-                if (qr >= SG && !mbar_test_wait(&empty[s], (uint32_t)(((qr / SG) & 1) ^ 1))) continue;
-                const int64_t m = r + (qr / ntile) * NG;  // token ordinal within the CTA
-                const int j = (int)(qr % ntile);
-                const int64_t t = blockIdx.x + m * G;
-                const int64_t k0 = (int64_t)j * tile;
+                const int s = r * SG + slot_r[r];
+                if (nq[r] >= SG && !mbar_test_wait(&empty[s], ph_r[r] ^ 1u)) continue;
+                const int64_t t = blockIdx.x + mr[r] * G;
+                const int64_t k0 = (int64_t)tile_r[r] * tile;
                 const int64_t w = (d - k0) < tile ? (d - k0) : tile;
                 const uint32_t rb = (uint32_t)(w * (int64_t)sizeof(S));
                 unsigned char *st = ring + (size_t)s * sh.stage_bytes;
                 mbar_arrive_expect_tx(&full[s], rb * ROWS);
                 const S *src = H + t * N * d + k0;
 #pragma unroll
-                for (int i = 0; i < N; ++i) bulk_load(st + i * row_bytes, src + i * d, rb, &full[s]);
-                if constexpr (WRITE) bulk_load(st + N * row_bytes, Y + t * d + k0, rb, &full[s]);
-                nq[r] = qr + 1;
+                for (int i = 0; i < N; ++i) load(st + i * row_bytes, src + i * d, rb, &full[s]);
+                if constexpr (WRITE) load(st + N * row_bytes, Y + t * d + k0, rb, &full[s]);
+                ++nq[r];
+                if (++slot_r[r] == SG) {
+                    slot_r[r] = 0;
+                    ph_r[r] ^= 1u;
+                }
+                if (++tile_r[r] == ntile) {
+                    tile_r[r] = 0;
+                    mr[r] += NG;
+                }
                 progressed = true;
             }
             if (!pending) break;
             if (progressed) {
                 idle_since = 0;
+                backoff = 32;
                 continue;
             }
-            // every ring is full: back off; give up only after the time limit
+            // every ring is full: back off (up to ~1 us); give up only after the limit
             if (*abort_flag) break;
-            if ((++idle_spins & 31u) == 0u) {
-                const uint64_t now = global_timer_ns();
-                if (idle_since == 0) {
-                    idle_since = now;
-                } else if (now - idle_since > kWaitLimitNs) {
-                    *abort_flag = 1;
-                    atomicOr(fault, FAULT_WAIT_EMPTY);
-                    break;
-                }
+            const uint64_t now = global_timer_ns();
+            if (idle_since == 0) {
+                idle_since = now;
+            } else if (now - idle_since > kWaitLimitNs) {
+                *abort_flag = 1;
+                atomicOr(fault, FAULT_WAIT_EMPTY);
+                break;
             }
-            __nanosleep(32);
+            __nanosleep(backoff);
+            if (backoff < 1024) backoff <<= 1;
         }
         // every issued copy lands before the CTA may exit (normally already done)
 #pragma unroll
@@ -201,9 +278,11 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
 
     if (warp == 1) {
         // ---------------- per-token parameters ----------------
-        constexpr int GL = Group<N>::GL, EPL = Group<N>::EPL, TPW = Group<N>::TPW;
+        // lane group q of each batch prepares token m0 + lane / GL
+        constexpr int GL = Group<N>::GL, EPL = Group<N>::EPL;
+        static_assert(Group<N>::TPW == PB, "one batch is one warp of lane groups");
         const int q = lane & (GL - 1);
-        for (int64_t m0 = 0; m0 < M; m0 += TPW) {
+        for (int64_t m0 = 0; m0 < M; m0 += PB) {
             const int64_t m = m0 + lane / GL;
             const bool live = m < M;
             const int64_t t = blockIdx.x + m * G;
@@ -222,7 +301,7 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
                     const int e = q + GL * r;
                     mv[r] = (live && e < NN) ? p.A[t * p.A_s + e] : 0.0f;
                 }
-                if (p.mix_logits) group_sinkhorn<N>(mv, lane, p.K);
+                if (p.mix_logits) group_sinkhorn<N>(mv, pscratch, lane, p.K);
                 if (live) {
 #pragma unroll
                     for (int r = 0; r < EPL; ++r) {
@@ -234,7 +313,7 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
             }
             if constexpr (READ) {
                 float l = (live && q < N) ? p.a[t * p.a_s + q] : 0.0f;
-                if (p.read_logits) l = group_softmax<N>(l, lane);
+                if (p.read_logits) l = group_softmax<N>(l, pscratch, lane);
                 if (live && q < N) P[NN + N + q] = l;
             }
             __syncwarp();
@@ -254,7 +333,8 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
     unsigned char *gring = ring + (size_t)g * SG * sh.stage_bytes;
     S *Ho = static_cast<S *>(p.Hout);
     S *X = static_cast<S *>(p.x);
-    int64_t q = 0;  // tiles this group has consumed
+    int slot = 0;      // ring position of this group's next tile
+    uint32_t ph = 0;   // its phase parity
 
     for (int64_t m = g, i = 0; m < M; m += NG, ++i) {
         const int64_t t = blockIdx.x + m * G;
@@ -275,25 +355,28 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
         bool ok = true;
         double ss = 0.0;
         S *Hot = Ho + t * N * d;
-        for (int j = 0; j < ntile; ++j, ++q) {
-            const int slot = (int)(q % SG);
-            const uint32_t ph = (uint32_t)((q / SG) & 1);
-            const bool w = mbar_wait_bounded(&gfull[slot], ph, abort_flag, fault, FAULT_WAIT_FULL);
+        for (int j = 0; j < ntile; ++j) {
+            const int cur = slot;
+            const bool w = mbar_wait_bounded(&gfull[cur], ph, abort_flag, fault, FAULT_WAIT_FULL);
             if (!__all_sync(0xffffffffu, w)) {
                 ok = false;
                 break;
             }
-            const unsigned char *st = gring + (size_t)slot * sh.stage_bytes + (size_t)gt * 16;
+            if (++slot == SG) {
+                slot = 0;
+                ph ^= 1u;
+            }
+            const unsigned char *st = gring + (size_t)cur * sh.stage_bytes + (size_t)gt * VB;
             const int64_t k = (int64_t)j * tile + (int64_t)gt * V;
             const bool active = k < d;
             float h[N][V], yv[V];
             if (active) {
 #pragma unroll
-                for (int ii = 0; ii < N; ++ii) SmemVec<S>::load(st + ii * row_bytes, h[ii]);
-                if constexpr (WRITE) SmemVec<S>::load(st + N * row_bytes, yv);
+                for (int ii = 0; ii < N; ++ii) VecIO<S, V>::load_smem(st + ii * row_bytes, h[ii]);
+                if constexpr (WRITE) VecIO<S, V>::load_smem(st + N * row_bytes, yv);
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&gempty[slot]);  // stage data is in registers
+            if (lane == 0) mbar_arrive(&gempty[cur]);  // stage data is in registers
             if (!active) continue;
             float hr[V];
             if constexpr (WRITE) {
@@ -313,7 +396,7 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
                     }
 #pragma unroll
                     for (int e = 0; e < V; ++e) acc[e] = __fmaf_rn(bv[jj], yv[e], acc[e]);
-                    store_vec_cs(Hot + jj * d + k, acc, stored);
+                    VecIO<S, V>::store(Hot + jj * d + k, acc, stored);
                     if constexpr (READ) {
                         if (jj == 0) {
 #pragma unroll
@@ -366,20 +449,44 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
             for (int ii = 0; ii < GW; ++ii) tot += part[ii];
             const float r = __double2float_rn(1.0 / sqrt(tot / (double)d + (double)p.eps));
             S *Xt = X + t * d;
+            // x = (h * r) * g, one slice per tile; the next slice's gain and h
+            // are loaded before the current slice is stored
+            int64_t k = (int64_t)gt * V;
+            bool have = k < d;
+            float gv[V], hv[V];
+            if (have) {
+                load_gain<V>(p.g, k, gv);
+#pragma unroll
+                for (int e = 0; e < V; e += 4) {
+                    const float4 f = *reinterpret_cast<const float4 *>(hrow + k + e);
+                    hv[e] = f.x; hv[e + 1] = f.y; hv[e + 2] = f.z; hv[e + 3] = f.w;
+                }
+            }
             for (int j = 0; j < ntile; ++j) {
-                const int64_t k = (int64_t)j * tile + (int64_t)gt * V;
-                if (k < d) {
-                    float gv[V], hv[V], xv[V];
-                    load_gain<V>(p.g, k, gv);
+                const int64_t kn = k + tile;
+                const bool have_n = (j + 1 < ntile) && kn < d;
+                float gn[V], hn[V];
+                if (have_n) {
+                    load_gain<V>(p.g, kn, gn);
 #pragma unroll
                     for (int e = 0; e < V; e += 4) {
-                        const float4 f = *reinterpret_cast<const float4 *>(hrow + k + e);
-                        hv[e] = f.x; hv[e + 1] = f.y; hv[e + 2] = f.z; hv[e + 3] = f.w;
+                        const float4 f = *reinterpret_cast<const float4 *>(hrow + kn + e);
+                        hn[e] = f.x; hn[e + 1] = f.y; hn[e + 2] = f.z; hn[e + 3] = f.w;
                     }
+                }
+                if (have) {
+                    float xv[V];
 #pragma unroll
                     for (int e = 0; e < V; ++e) xv[e] = __fmul_rn(__fmul_rn(hv[e], r), gv[e]);
-                    store_vec_cs(Xt + k, xv);
+                    VecIO<S, V>::store(Xt + k, xv);
                 }
+#pragma unroll
+                for (int e = 0; e < V; ++e) {
+                    gv[e] = gn[e];
+                    hv[e] = hn[e];
+                }
+                k = kn;
+                have = have_n;
             }
         }
     }

@@ -35,6 +35,7 @@ hc_stream_kernel(StepParams p) {
     __shared__ float sb[TB_MAX * N];
     __shared__ float sa[TB_MAX * N];
     __shared__ double sred[2][kStreamMaxThreads / 32];
+    __shared__ float swork[kStreamMaxThreads / 32 * kGroupScratch];
 
     const int tid = threadIdx.x;
     const int NT = blockDim.x;
@@ -56,7 +57,7 @@ hc_stream_kernel(StepParams p) {
         const int64_t first = blockIdx.x + m0 * G;
         if (first >= p.T) break;
         __syncthreads();  // previous batch's parameters no longer read
-        prepare_params<N, WRITE, READ>(p, first, G, TB, sA, sb, sa);
+        prepare_params<N, WRITE, READ>(p, first, G, TB, sA, sb, sa, swork);
         __syncthreads();
 
         for (int tt = 0; tt < TB; ++tt) {
@@ -173,8 +174,10 @@ template <int N>
 __global__ void __launch_bounds__(256)
 hc_sinkhorn_kernel(const float *L, float *out, int64_t T, int K) {
     constexpr int NN = N * N, GL = Group<N>::GL, EPL = Group<N>::EPL, TPW = Group<N>::TPW;
+    __shared__ float swork[256 / 32 * kGroupScratch];
     const int lane = threadIdx.x & 31;
     const int q = lane & (GL - 1);
+    float *wscratch = swork + (threadIdx.x >> 5) * kGroupScratch;
     const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps_global = ((int64_t)gridDim.x * blockDim.x) >> 5;
     for (int64_t t0 = warp_global * TPW; t0 < T; t0 += nwarps_global * TPW) {
@@ -186,7 +189,7 @@ hc_sinkhorn_kernel(const float *L, float *out, int64_t T, int K) {
             const int e = q + GL * r;
             m[r] = (live && e < NN) ? L[t * NN + e] : 0.0f;
         }
-        group_sinkhorn<N>(m, lane, K);
+        group_sinkhorn<N>(m, wscratch, lane, K);
         if (live) {
 #pragma unroll
             for (int r = 0; r < EPL; ++r) {
