@@ -1,0 +1,95 @@
+"""Multi-rank path on CPU: two gloo ranks run the bench's sharding and timing
+helpers. Each rank steps its own batch of tokens through the oracle; the
+shards, concatenated, must equal one oracle call over all tokens (the step
+has no cross-token coupling, so sharding needs no collective), and the timing
+reduction must return the slowest rank's value."""
+from __future__ import annotations
+
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_inputs(rank, T, n, d):
+    import hc_inputs as gen
+    from hyper_connections_stream_b200 import dist as hd
+    off = hd.seed_offset(rank)
+    H = gen.to_storage(gen.normal(gen.SEED_H + off, (T, n, d)), "bf16")
+    y = gen.to_storage(gen.normal(gen.SEED_Y + off, (T, d)), "bf16")
+    L = gen.normal(gen.SEED_L + off, (T, n, n))
+    rl = gen.normal(gen.SEED_L + 100 + off, (T, n))
+    return H, y, L, rl
+
+
+def _worker(rank, world, port, T, n, d, out_dir):
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    import oracle
+    from hyper_connections_stream_b200 import dist as hd
+    oracle.set_threads(1)
+    ws, r, _ = hd.env()
+    assert (ws, r) == (world, rank)
+    H, y, L, rl = _rank_inputs(rank, T, n, d)
+    b = np.ones(n, np.float32)
+    hd.barrier(ws)
+    H2, x2 = oracle.write_then_read(H, y, L, b, rl, None, 1e-6, "bf16", K=20,
+                                    mix_logits=True, read_logits=True)
+    slowest = hd.max_over_ranks(float(rank + 1) * 0.25, ws)
+    outs = [torch.zeros(T * n * d, dtype=torch.int32) for _ in range(ws)]
+    dist.all_gather(outs, torch.from_numpy(H2.astype(np.int32).reshape(-1)))
+    xs = [torch.zeros(T * d, dtype=torch.int32) for _ in range(ws)]
+    dist.all_gather(xs, torch.from_numpy(x2.astype(np.int32).reshape(-1)))
+    if rank == 0:
+        np.save(os.path.join(out_dir, "H.npy"), torch.cat(outs).numpy())
+        np.save(os.path.join(out_dir, "x.npy"), torch.cat(xs).numpy())
+        np.save(os.path.join(out_dir, "slowest.npy"), np.array([slowest]))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_shard_tokens_without_a_collective(tmp_path):
+    world, T, n, d = 2, 6, 4, 64
+    mp.spawn(_worker, args=(world, _free_port(), T, n, d, str(tmp_path)), nprocs=world, join=True)
+    import oracle
+    parts = [_rank_inputs(r, T, n, d) for r in range(world)]
+    H = np.concatenate([p[0] for p in parts])
+    y = np.concatenate([p[1] for p in parts])
+    L = np.concatenate([p[2] for p in parts])
+    rl = np.concatenate([p[3] for p in parts])
+    H2, x2 = oracle.write_then_read(H, y, L, np.ones(n, np.float32), rl, None, 1e-6, "bf16",
+                                    K=20, mix_logits=True, read_logits=True)
+    got_H = np.load(tmp_path / "H.npy").astype(np.uint16).reshape(world * T, n, d)
+    got_x = np.load(tmp_path / "x.npy").astype(np.uint16).reshape(world * T, d)
+    assert np.array_equal(got_H, H2) and np.array_equal(got_x, x2)
+    assert float(np.load(tmp_path / "slowest.npy")[0]) == 0.5
+
+
+def test_token_shard_partitions_exactly():
+    from hyper_connections_stream_b200 import dist as hd
+    for T in (0, 1, 7, 16384, 16387):
+        for world in (1, 2, 3, 8):
+            spans = [hd.token_shard(T, r, world) for r in range(world)]
+            assert sum(c for _, c in spans) == T
+            pos = 0
+            for start, count in spans:
+                assert start == pos
+                pos += count
+            assert max(c for _, c in spans) - min(c for _, c in spans) <= 1
