@@ -118,17 +118,18 @@ template <int N> struct Group {
 };
 constexpr int kGroupScratch = 64;  // floats per warp: TPW * n * n <= 64 for n <= 8
 
-// Sinkhorn projection of the group's matrix (all 32 lanes call with the same
-// K): M = exp(L); K times { divide every row by its sum; divide every column
-// by its sum }. Sums run in index order starting from +0 and divisions are
-// IEEE (__fdiv_rn), so every element sees a fixed sequence of correctly
-// rounded operations. `scratch` is this warp's kGroupScratch floats.
-template <int N>
-__device__ __forceinline__ void group_sinkhorn(float (&m)[Group<N>::EPL], float *scratch, int lane,
-                                               int K) {
+// Sinkhorn projection of R independent batches of the warp's lane-group
+// matrices (all 32 lanes call with the same K): M = exp(L); K times { divide
+// every row by its sum; divide every column by its sum }. Sums run in index
+// order starting from +0 and divisions are IEEE (__fdiv_rn), so every element
+// sees a fixed sequence of correctly rounded operations. The R batches share
+// the passes, so their latencies overlap. `scratch` holds R * kGroupScratch
+// floats for this warp.
+template <int N, int R>
+__device__ __forceinline__ void group_sinkhorn(float (&m)[R][Group<N>::EPL], float *scratch,
+                                               int lane, int K) {
     constexpr int NN = N * N, GL = Group<N>::GL, EPL = Group<N>::EPL;
     const int q = lane & (GL - 1);
-    float *buf = scratch + (lane / GL) * NN;  // this group's matrix
     int e[EPL], row[EPL], col[EPL];
     bool own[EPL];
 #pragma unroll
@@ -138,31 +139,58 @@ __device__ __forceinline__ void group_sinkhorn(float (&m)[Group<N>::EPL], float 
         const int ec = own[r] ? e[r] : NN - 1;  // idle lanes shadow the last element
         row[r] = ec / N;
         col[r] = ec - row[r] * N;
-        m[r] = expf(m[r]);
+    }
+#pragma unroll
+    for (int b = 0; b < R; ++b) {
+#pragma unroll
+        for (int r = 0; r < EPL; ++r) m[b][r] = expf(m[b][r]);
     }
     for (int it = 0; it < K; ++it) {
 #pragma unroll
         for (int pass = 0; pass < 2; ++pass) {
 #pragma unroll
-            for (int r = 0; r < EPL; ++r)
-                if (own[r]) buf[e[r]] = m[r];
+            for (int b = 0; b < R; ++b) {
+                float *buf = scratch + b * kGroupScratch + (lane / GL) * NN;
+#pragma unroll
+                for (int r = 0; r < EPL; ++r)
+                    if (own[r]) buf[e[r]] = m[b][r];
+            }
             __syncwarp();
-            float s[EPL];
+            float s[R][EPL];
 #pragma unroll
-            for (int r = 0; r < EPL; ++r) {
-                float v[N];
+            for (int b = 0; b < R; ++b) {
+                const float *buf = scratch + b * kGroupScratch + (lane / GL) * NN;
 #pragma unroll
-                for (int k = 0; k < N; ++k) v[k] = pass == 0 ? buf[row[r] * N + k] : buf[k * N + col[r]];
-                float acc = 0.0f;
+                for (int r = 0; r < EPL; ++r) {
+                    float v[N];
 #pragma unroll
-                for (int k = 0; k < N; ++k) acc = __fadd_rn(acc, v[k]);
-                s[r] = acc;
+                    for (int k = 0; k < N; ++k) v[k] = pass == 0 ? buf[row[r] * N + k] : buf[k * N + col[r]];
+                    float acc = 0.0f;
+#pragma unroll
+                    for (int k = 0; k < N; ++k) acc = __fadd_rn(acc, v[k]);
+                    s[b][r] = acc;
+                }
             }
             __syncwarp();
 #pragma unroll
-            for (int r = 0; r < EPL; ++r) m[r] = __fdiv_rn(m[r], s[r]);
+            for (int b = 0; b < R; ++b) {
+#pragma unroll
+                for (int r = 0; r < EPL; ++r) m[b][r] = __fdiv_rn(m[b][r], s[b][r]);
+            }
         }
     }
+}
+
+// One batch (R = 1).
+template <int N>
+__device__ __forceinline__ void group_sinkhorn(float (&m)[Group<N>::EPL], float *scratch, int lane,
+                                               int K) {
+    float mm[1][Group<N>::EPL];
+#pragma unroll
+    for (int r = 0; r < Group<N>::EPL; ++r) mm[0][r] = m[r];
+    group_sinkhorn<N, 1>(mm, scratch, lane, K);
+#pragma unroll
+    for (int r = 0; r < Group<N>::EPL; ++r) m[r] = mm[0][r];
 }
 
 // Softmax over the n read logits of the group's token. Lane q < N holds l_q

@@ -90,11 +90,16 @@ bool pipe_shape(const StepParams &p, PipeShape &sh, int &smem) {
     if (ntile > (1 << 20)) return false;
     sh.ntile = (int)ntile;
     sh.stage_bytes = ROWS * sh.tile * (int)sizeof(S);
-    // one ring per consumer group, at least two stages each
+    // one ring per consumer group: the pipelined family needs room for two
+    // stages per group; the ring then takes the kind's measured depth
     int64_t per_group = (kSmemLimit - pipe_fixed_bytes(N, 0, d_h)) /
                         ((int64_t)kPipeGroups * (sh.stage_bytes + 16));
-    if (per_group > kMaxStages / kPipeGroups) per_group = kMaxStages / kPipeGroups;
     if (per_group < 2) return false;
+    if (per_group > kMaxStages / kPipeGroups) per_group = kMaxStages / kPipeGroups;
+    const int64_t cap = KIND == KIND_WRITE ? HC_PIPE_SG_WRITE
+                        : KIND == KIND_FUSED ? HC_PIPE_SG_FUSED : HC_PIPE_SG_READ;
+    if (per_group > cap) per_group = cap;
+    if (per_group < 1) per_group = 1;
     sh.stages = (int)(per_group * kPipeGroups);
     smem = (int)((int64_t)sh.stages * sh.stage_bytes + pipe_fixed_bytes(N, sh.stages, d_h));
     return true;

@@ -40,15 +40,32 @@ namespace hc {
 #ifndef HC_PIPE_L2_HINT
 #define HC_PIPE_L2_HINT 0
 #endif
+// Ring stages per consumer group, by kind. Shallow read-ahead keeps DRAM
+// reads and writes balanced for the kinds that write as much as they read
+// (measured on B200 at n = 4, d = 7168, bf16: write 2, fused 3); the read
+// kind writes little and wants the deepest ring that fits.
+#ifndef HC_PIPE_SG_WRITE
+#define HC_PIPE_SG_WRITE 2
+#endif
+#ifndef HC_PIPE_SG_FUSED
+#define HC_PIPE_SG_FUSED 3
+#endif
+#ifndef HC_PIPE_SG_READ
+#define HC_PIPE_SG_READ 16
+#endif
 constexpr int kPipeGroups = HC_PIPE_GROUPS;
 constexpr int kPipeGroupWarps = HC_PIPE_GROUP_WARPS;
 constexpr int kPipeGroupThreads = kPipeGroupWarps * 32;
 constexpr int kPipeThreads = 64 + kPipeGroups * kPipeGroupThreads;
-// The parameter warp prepares one lane group's worth of tokens at a time
-// (32 / GL: 2 for n = 3, 4; 1 for n >= 5); each group's slot ring holds at
+// The parameter warp prepares kParamReplicas warps' worth of lane groups at a
+// time (4 tokens for n = 3, 4; 2 for n >= 5); each group's slot ring holds at
 // least 8 of its tokens, and two batches, so preparation runs ahead.
+// Independent token batches the parameter warp runs through each Sinkhorn
+// pass together (their latencies overlap).
+constexpr int kParamReplicas = 2;
 __host__ __device__ constexpr int pipe_param_batch(int n) {
-    return n * n <= 1 ? 32 : n * n <= 2 ? 16 : n * n <= 4 ? 8 : n * n <= 8 ? 4 : n * n <= 16 ? 2 : 1;
+    return kParamReplicas *
+           (n * n <= 1 ? 32 : n * n <= 2 ? 16 : n * n <= 4 ? 8 : n * n <= 8 ? 4 : n * n <= 16 ? 2 : 1);
 }
 __host__ __device__ constexpr int pipe_param_slots_per_group(int n) {
     return (((2 * pipe_param_batch(n) + kPipeGroups - 1) / kPipeGroups > 8
@@ -67,7 +84,8 @@ struct PipeShape {
 
 // Bytes of everything in shared memory other than the ring: barriers,
 // parameter slots, reduction partials, the abort flag and, for the
-// normalising kinds, each group's fp32 row h[d] (d_h = d, else 0).
+// normalising kinds, two fp32 rows h[d] per group (d_h = d, else 0): the
+// current token's and the previous token's, whose x is written meanwhile.
 __host__ __device__ constexpr int64_t pipe_fixed_bytes(int n, int stages, int64_t d_h) {
     return (int64_t)stages * 16                        // full + empty barriers
            + kPipeGroups * pipe_param_slots_per_group(n) * 16  // param full + empty
@@ -75,8 +93,8 @@ __host__ __device__ constexpr int64_t pipe_fixed_bytes(int n, int stages, int64_
            + kPipeGroups * pipe_param_slots_per_group(n) * (n * n + 2 * n) * 4  // slots
            + kPipeGroups * 2 * kPipeGroupWarps * 8     // reduction partials
            + 16                                        // abort flag (padded)
-           + kGroupScratch * 4                         // parameter warp scratch
-           + (int64_t)kPipeGroups * ((d_h * 4 + 15) / 16 * 16);  // h rows
+           + kParamReplicas * kGroupScratch * 4        // parameter warp scratch
+           + (int64_t)kPipeGroups * 2 * ((d_h * 4 + 15) / 16 * 16);  // h rows (2 per group)
 }
 
 // Elements of d one consumer thread handles per tile: a 16-byte vector, or
@@ -166,7 +184,7 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
     int *abort_word = reinterpret_cast<int *>(sred + NG * 2 * GW);
     volatile int *abort_flag = abort_word;
     float *pscratch = reinterpret_cast<float *>(abort_word + 4);  // parameter warp scratch
-    float *hrow_base = pscratch + kGroupScratch;                   // 16-byte aligned
+    float *hrow_base = pscratch + kParamReplicas * kGroupScratch;  // 16-byte aligned
     const int64_t d = p.d;
     const int64_t hrow_stride = READ ? (d + 3) / 4 * 4 : 0;  // floats per group row
     const int SG = sh.stages / NG;  // stages per group ring
@@ -278,56 +296,102 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
 
     if (warp == 1) {
         // ---------------- per-token parameters ----------------
-        // lane group q of each batch prepares token m0 + lane / GL
-        constexpr int GL = Group<N>::GL, EPL = Group<N>::EPL;
-        static_assert(Group<N>::TPW == PB, "one batch is one warp of lane groups");
+        // Batch replica rb, lane group lane / GL prepares token
+        // m0 + rb * TPW + lane / GL. The next batch's inputs are loaded
+        // before the current batch is projected, hiding their latency.
+        constexpr int GL = Group<N>::GL, EPL = Group<N>::EPL, TPW = Group<N>::TPW;
+        constexpr int R = kParamReplicas;
+        static_assert(R * TPW == PB, "a batch is R warps' worth of lane groups");
         const int q = lane & (GL - 1);
-        for (int64_t m0 = 0; m0 < M; m0 += PB) {
-            const int64_t m = m0 + lane / GL;
-            const bool live = m < M;
-            const int64_t t = blockIdx.x + m * G;
-            const int64_t i = m / NG;  // token ordinal within its group
-            const int ps = (int)(m % NG) * PSG + (int)(i % PSG);
-            bool w = true;
-            if (live && i >= PSG)
-                w = mbar_wait_bounded(&pempty[ps], (uint32_t)(((i / PSG) & 1) ^ 1), abort_flag, fault,
-                                      FAULT_WAIT_PARAM);
-            if (!__all_sync(0xffffffffu, w)) break;
-            float *P = params + ps * PSTRIDE;
-            if constexpr (WRITE) {
-                float mv[EPL];
+        float nmv[R][EPL], nlv[R], nbv[R];
+        auto fetch = [&](int64_t m0) {
+#pragma unroll
+            for (int rb = 0; rb < R; ++rb) {
+                const int64_t m = m0 + rb * TPW + lane / GL;
+                const bool live = m < M;
+                const int64_t t = blockIdx.x + m * G;
 #pragma unroll
                 for (int r = 0; r < EPL; ++r) {
                     const int e = q + GL * r;
-                    mv[r] = (live && e < NN) ? p.A[t * p.A_s + e] : 0.0f;
+                    nmv[rb][r] = (WRITE && live && e < NN) ? p.A[t * p.A_s + e] : 0.0f;
                 }
-                if (p.mix_logits) group_sinkhorn<N>(mv, pscratch, lane, p.K);
-                if (live) {
+                nbv[rb] = (WRITE && live && q < N) ? p.b[t * p.b_s + q] : 0.0f;
+                nlv[rb] = (READ && live && q < N) ? p.a[t * p.a_s + q] : 0.0f;
+            }
+        };
+        fetch(0);
+        for (int64_t m0 = 0; m0 < M; m0 += PB) {
+            float mv[R][EPL], lv[R], bvv[R];
+#pragma unroll
+            for (int rb = 0; rb < R; ++rb) {
+#pragma unroll
+                for (int r = 0; r < EPL; ++r) mv[rb][r] = nmv[rb][r];
+                lv[rb] = nlv[rb];
+                bvv[rb] = nbv[rb];
+            }
+            if (m0 + PB < M) fetch(m0 + PB);
+            bool w = true;
+#pragma unroll
+            for (int rb = 0; rb < R; ++rb) {
+                const int64_t m = m0 + rb * TPW + lane / GL;
+                const int64_t i = m / NG;  // token ordinal within its group
+                const int ps = (int)(m % NG) * PSG + (int)(i % PSG);
+                if (m < M && i >= PSG)
+                    w = w && mbar_wait_bounded(&pempty[ps], (uint32_t)(((i / PSG) & 1) ^ 1), abort_flag,
+                                               fault, FAULT_WAIT_PARAM);
+            }
+            if (!__all_sync(0xffffffffu, w)) break;
+            if constexpr (WRITE) {
+                if (p.mix_logits) group_sinkhorn<N, R>(mv, pscratch, lane, p.K);
+            }
+            if constexpr (READ) {
+                if (p.read_logits) {
+#pragma unroll
+                    for (int rb = 0; rb < R; ++rb) lv[rb] = group_softmax<N>(lv[rb], pscratch, lane);
+                }
+            }
+#pragma unroll
+            for (int rb = 0; rb < R; ++rb) {
+                const int64_t m = m0 + rb * TPW + lane / GL;
+                if (m >= M) continue;
+                const int64_t i = m / NG;
+                const int ps = (int)(m % NG) * PSG + (int)(i % PSG);
+                float *P = params + ps * PSTRIDE;
+                if constexpr (WRITE) {
 #pragma unroll
                     for (int r = 0; r < EPL; ++r) {
                         const int e = q + GL * r;  // A[i][j], i = e / N, j = e % N
-                        if (e < NN) P[(e % N) * N + e / N] = mv[r];
+                        if (e < NN) P[(e % N) * N + e / N] = mv[rb][r];
                     }
-                    if (q < N) P[NN + q] = p.b[t * p.b_s + q];
+                    if (q < N) P[NN + q] = bvv[rb];
+                }
+                if constexpr (READ) {
+                    if (q < N) P[NN + N + q] = lv[rb];
                 }
             }
-            if constexpr (READ) {
-                float l = (live && q < N) ? p.a[t * p.a_s + q] : 0.0f;
-                if (p.read_logits) l = group_softmax<N>(l, pscratch, lane);
-                if (live && q < N) P[NN + N + q] = l;
-            }
             __syncwarp();
-            if (live && q == 0) mbar_arrive(&pfull[ps]);
+#pragma unroll
+            for (int rb = 0; rb < R; ++rb) {
+                const int64_t m = m0 + rb * TPW + lane / GL;
+                if (m < M && q == 0) {
+                    const int64_t i = m / NG;
+                    mbar_arrive(&pfull[(int)(m % NG) * PSG + (int)(i % PSG)]);
+                }
+            }
         }
         return;
     }
 
     // ---------------- consumers ----------------
+    // Group g takes the CTA's tokens g, g + NG, ... (its i-th token is
+    // m = g + i * NG). While it processes token i tile by tile, it also writes
+    // token i-1's x, one tile after each of token i's tiles: a warp arrives at
+    // the group reduction of token i-1 and goes on to token i's first tile
+    // before it waits for the other warps' sums, so the wait overlaps work.
     const int cw = warp - 2;
     const int g = cw / GW;
     const int gw = cw - g * GW;
     const int gt = gw * 32 + lane;
-    float *hrow = hrow_base + g * hrow_stride;  // this group's h[d] (fp32)
     uint64_t *gfull = full + g * SG;
     uint64_t *gempty = empty + g * SG;
     unsigned char *gring = ring + (size_t)g * SG * sh.stage_bytes;
@@ -335,158 +399,152 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
     S *X = static_cast<S *>(p.x);
     int slot = 0;      // ring position of this group's next tile
     uint32_t ph = 0;   // its phase parity
+    const int64_t Mg = M > g ? (M - 1 - g) / NG + 1 : 0;  // tokens of this group
+    float r_prev = 0.0f;
 
-    for (int64_t m = g, i = 0; m < M; m += NG, ++i) {
+    for (int64_t i = 0; i <= Mg; ++i) {
+        const bool cur = i < Mg;                 // token i to mix
+        const bool prev = READ && i > 0;         // token i-1 to normalise
+        const int64_t m = g + i * NG;
         const int64_t t = blockIdx.x + m * G;
+        const int64_t t_prev = t - (int64_t)NG * G;
+        float *hcur = hrow_base + (g * 2 + (int)(i & 1)) * hrow_stride;
+        const float *hprev = hrow_base + (g * 2 + (int)((i + 1) & 1)) * hrow_stride;
         const int ps = g * PSG + (int)(i % PSG);
-        {
+        float bv[N], av[N];
+        const float *P = params + ps * PSTRIDE;
+        if (cur) {
             const bool w = mbar_wait_bounded(&pfull[ps], (uint32_t)((i / PSG) & 1), abort_flag, fault,
                                              FAULT_WAIT_PARAM);
             if (!__all_sync(0xffffffffu, w)) break;
-        }
-        const float *P = params + ps * PSTRIDE;
-        float bv[N], av[N];
 #pragma unroll
-        for (int ii = 0; ii < N; ++ii) {
-            bv[ii] = WRITE ? P[NN + ii] : 0.0f;
-            av[ii] = READ ? P[NN + N + ii] : 0.0f;
+            for (int ii = 0; ii < N; ++ii) {
+                bv[ii] = WRITE ? P[NN + ii] : 0.0f;
+                av[ii] = READ ? P[NN + N + ii] : 0.0f;
+            }
         }
 
         bool ok = true;
         double ss = 0.0;
-        S *Hot = Ho + t * N * d;
         for (int j = 0; j < ntile; ++j) {
-            const int cur = slot;
-            const bool w = mbar_wait_bounded(&gfull[cur], ph, abort_flag, fault, FAULT_WAIT_FULL);
-            if (!__all_sync(0xffffffffu, w)) {
-                ok = false;
-                break;
-            }
-            if (++slot == SG) {
-                slot = 0;
-                ph ^= 1u;
-            }
-            const unsigned char *st = gring + (size_t)cur * sh.stage_bytes + (size_t)gt * VB;
             const int64_t k = (int64_t)j * tile + (int64_t)gt * V;
             const bool active = k < d;
-            float h[N][V], yv[V];
-            if (active) {
+            if (cur) {
+                const int cs = slot;
+                const bool w = mbar_wait_bounded(&gfull[cs], ph, abort_flag, fault, FAULT_WAIT_FULL);
+                if (!__all_sync(0xffffffffu, w)) {
+                    ok = false;
+                    break;
+                }
+                if (++slot == SG) {
+                    slot = 0;
+                    ph ^= 1u;
+                }
+                const unsigned char *st = gring + (size_t)cs * sh.stage_bytes + (size_t)gt * VB;
+                float h[N][V], yv[V];
+                if (active) {
 #pragma unroll
-                for (int ii = 0; ii < N; ++ii) VecIO<S, V>::load_smem(st + ii * row_bytes, h[ii]);
-                if constexpr (WRITE) VecIO<S, V>::load_smem(st + N * row_bytes, yv);
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&gempty[cur]);  // stage data is in registers
-            if (!active) continue;
-            float hr[V];
-            if constexpr (WRITE) {
+                    for (int ii = 0; ii < N; ++ii) VecIO<S, V>::load_smem(st + ii * row_bytes, h[ii]);
+                    if constexpr (WRITE) VecIO<S, V>::load_smem(st + N * row_bytes, yv);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&gempty[cs]);  // stage data is in registers
+                if (active) {
+                    float hr[V];
+                    if constexpr (WRITE) {
+                        S *Hot = Ho + t * N * d + k;
 #pragma unroll
-                for (int jj = 0; jj < N; ++jj) {
-                    // column jj of A: A[0][jj] .. A[N-1][jj]
-                    float col[N];
+                        for (int jj = 0; jj < N; ++jj) {
+                            // column jj of A: A[0][jj] .. A[N-1][jj]
+                            float col[N];
 #pragma unroll
-                    for (int ii = 0; ii < N; ++ii) col[ii] = P[jj * N + ii];
-                    float acc[V], stored[V];
+                            for (int ii = 0; ii < N; ++ii) col[ii] = P[jj * N + ii];
+                            float acc[V], stored[V];
 #pragma unroll
-                    for (int e = 0; e < V; ++e) acc[e] = __fmul_rn(col[0], h[0][e]);
+                            for (int e = 0; e < V; ++e) acc[e] = __fmul_rn(col[0], h[0][e]);
 #pragma unroll
-                    for (int ii = 1; ii < N; ++ii) {
+                            for (int ii = 1; ii < N; ++ii) {
 #pragma unroll
-                        for (int e = 0; e < V; ++e) acc[e] = __fmaf_rn(col[ii], h[ii][e], acc[e]);
-                    }
+                                for (int e = 0; e < V; ++e) acc[e] = __fmaf_rn(col[ii], h[ii][e], acc[e]);
+                            }
 #pragma unroll
-                    for (int e = 0; e < V; ++e) acc[e] = __fmaf_rn(bv[jj], yv[e], acc[e]);
-                    VecIO<S, V>::store(Hot + jj * d + k, acc, stored);
-                    if constexpr (READ) {
-                        if (jj == 0) {
+                            for (int e = 0; e < V; ++e) acc[e] = __fmaf_rn(bv[jj], yv[e], acc[e]);
+                            VecIO<S, V>::store(Hot + jj * d, acc, stored);
+                            if constexpr (READ) {
+                                if (jj == 0) {
 #pragma unroll
-                            for (int e = 0; e < V; ++e) hr[e] = __fmul_rn(av[0], stored[e]);
-                        } else {
+                                    for (int e = 0; e < V; ++e) hr[e] = __fmul_rn(av[0], stored[e]);
+                                } else {
 #pragma unroll
-                            for (int e = 0; e < V; ++e) hr[e] = __fmaf_rn(av[jj], stored[e], hr[e]);
+                                    for (int e = 0; e < V; ++e) hr[e] = __fmaf_rn(av[jj], stored[e], hr[e]);
+                                }
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < V; ++e) hr[e] = __fmul_rn(av[0], h[0][e]);
+#pragma unroll
+                        for (int ii = 1; ii < N; ++ii) {
+#pragma unroll
+                            for (int e = 0; e < V; ++e) hr[e] = __fmaf_rn(av[ii], h[ii][e], hr[e]);
                         }
                     }
-                }
-            } else {
+                    if constexpr (READ) {
 #pragma unroll
-                for (int e = 0; e < V; ++e) hr[e] = __fmul_rn(av[0], h[0][e]);
+                        for (int e = 0; e < V; ++e) {
+                            const double hv = (double)hr[e];
+                            ss = __fma_rn(hv, hv, ss);
+                        }
+                        // keep h for the normalisation (this thread reads it back itself)
 #pragma unroll
-                for (int ii = 1; ii < N; ++ii) {
-#pragma unroll
-                    for (int e = 0; e < V; ++e) hr[e] = __fmaf_rn(av[ii], h[ii][e], hr[e]);
+                        for (int e = 0; e < V; e += 4)
+                            *reinterpret_cast<float4 *>(hcur + k + e) =
+                                make_float4(hr[e], hr[e + 1], hr[e + 2], hr[e + 3]);
+                    }
                 }
             }
             if constexpr (READ) {
+                if (prev) {
+                    if (j == 0) {
+                        // token i-1's sum of squares, reduced over the group's warps
+                        const bool w = mbar_wait_bounded(&redbar[g], (uint32_t)((i - 1) & 1), abort_flag,
+                                                         fault, FAULT_WAIT_REDUCE);
+                        if (!__all_sync(0xffffffffu, w)) {
+                            ok = false;
+                            break;
+                        }
+                        const double *part = sred + (g * 2 + (int)((i - 1) & 1)) * GW;
+                        double tot = 0.0;
 #pragma unroll
-                for (int e = 0; e < V; ++e) {
-                    const double hv = (double)hr[e];
-                    ss = __fma_rn(hv, hv, ss);
+                        for (int ii = 0; ii < GW; ++ii) tot += part[ii];
+                        r_prev = __double2float_rn(1.0 / sqrt(tot / (double)d + (double)p.eps));
+                    }
+                    if (active) {
+                        float gv[V], hv[V], xv[V];
+                        load_gain<V>(p.g, k, gv);
+#pragma unroll
+                        for (int e = 0; e < V; e += 4) {
+                            const float4 f = *reinterpret_cast<const float4 *>(hprev + k + e);
+                            hv[e] = f.x; hv[e + 1] = f.y; hv[e + 2] = f.z; hv[e + 3] = f.w;
+                        }
+#pragma unroll
+                        for (int e = 0; e < V; ++e) xv[e] = __fmul_rn(__fmul_rn(hv[e], r_prev), gv[e]);
+                        VecIO<S, V>::store(X + t_prev * d + k, xv);
+                    }
                 }
-                // keep h for the normalisation (this thread reads it back itself)
-#pragma unroll
-                for (int e = 0; e < V; e += 4)
-                    *reinterpret_cast<float4 *>(hrow + k + e) =
-                        make_float4(hr[e], hr[e + 1], hr[e + 2], hr[e + 3]);
             }
         }
         if (!ok) break;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&pempty[ps]);  // parameters no longer read
-
-        if constexpr (READ) {
+        if (cur) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pempty[ps]);  // parameters no longer read
+            if constexpr (READ) {
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-            double *part = sred + (g * 2 + (int)(i & 1)) * GW;
-            if (lane == 0) {
-                part[gw] = ss;
-                mbar_arrive(&redbar[g]);
-            }
-            const bool w = mbar_wait_bounded(&redbar[g], (uint32_t)(i & 1), abort_flag, fault,
-                                             FAULT_WAIT_REDUCE);
-            if (!__all_sync(0xffffffffu, w)) break;
-            double tot = 0.0;
-#pragma unroll
-            for (int ii = 0; ii < GW; ++ii) tot += part[ii];
-            const float r = __double2float_rn(1.0 / sqrt(tot / (double)d + (double)p.eps));
-            S *Xt = X + t * d;
-            // x = (h * r) * g, one slice per tile; the next slice's gain and h
-            // are loaded before the current slice is stored
-            int64_t k = (int64_t)gt * V;
-            bool have = k < d;
-            float gv[V], hv[V];
-            if (have) {
-                load_gain<V>(p.g, k, gv);
-#pragma unroll
-                for (int e = 0; e < V; e += 4) {
-                    const float4 f = *reinterpret_cast<const float4 *>(hrow + k + e);
-                    hv[e] = f.x; hv[e + 1] = f.y; hv[e + 2] = f.z; hv[e + 3] = f.w;
+                for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                if (lane == 0) {
+                    sred[(g * 2 + (int)(i & 1)) * GW + gw] = ss;
+                    mbar_arrive(&redbar[g]);
                 }
-            }
-            for (int j = 0; j < ntile; ++j) {
-                const int64_t kn = k + tile;
-                const bool have_n = (j + 1 < ntile) && kn < d;
-                float gn[V], hn[V];
-                if (have_n) {
-                    load_gain<V>(p.g, kn, gn);
-#pragma unroll
-                    for (int e = 0; e < V; e += 4) {
-                        const float4 f = *reinterpret_cast<const float4 *>(hrow + kn + e);
-                        hn[e] = f.x; hn[e + 1] = f.y; hn[e + 2] = f.z; hn[e + 3] = f.w;
-                    }
-                }
-                if (have) {
-                    float xv[V];
-#pragma unroll
-                    for (int e = 0; e < V; ++e) xv[e] = __fmul_rn(__fmul_rn(hv[e], r), gv[e]);
-                    VecIO<S, V>::store(Xt + k, xv);
-                }
-#pragma unroll
-                for (int e = 0; e < V; ++e) {
-                    gv[e] = gn[e];
-                    hv[e] = hn[e];
-                }
-                k = kn;
-                have = have_n;
             }
         }
     }
