@@ -84,6 +84,28 @@ __device__ __forceinline__ void store_vec_cs(__nv_bfloat16 *p, const float (&v)[
     __stcs(reinterpret_cast<uint4 *>(p), q);
 }
 
+// Paired fp32 arithmetic (sm_100): one instruction performs the operation on
+// two independent element pairs, each correctly rounded exactly like the
+// scalar __fmaf_rn / __fmul_rn, so results are bit-identical.
+__device__ __forceinline__ float2 ffma2_rn(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 fmul2_rn(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
 // Read-only (L1-cached) load of V fp32 gains.
 template <int V>
 __device__ __forceinline__ void load_gain(const float *g, int64_t k, float (&gv)[V]) {

@@ -105,53 +105,78 @@ __host__ __device__ constexpr int pipe_vec_elems() {
     return (sizeof(S) == 2 && N > 4) ? 4 : StorageTraits<S>::V;
 }
 
-// Shared-memory loads and streaming global stores of VE storage elements.
+// Shared-memory loads and streaming global stores of VE storage elements,
+// held as VE / 2 fp32 pairs (element 2p in .x, 2p + 1 in .y).
 template <typename S, int VE> struct VecIO;
 template <> struct VecIO<float, 4> {
-    static __device__ __forceinline__ void load_smem(const unsigned char *p, float (&v)[4]) {
+    static __device__ __forceinline__ void load_smem(const unsigned char *p, float2 (&v)[2]) {
         const float4 q = *reinterpret_cast<const float4 *>(p);
-        v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+        v[0] = make_float2(q.x, q.y);
+        v[1] = make_float2(q.z, q.w);
     }
-    static __device__ __forceinline__ void store(float *p, const float (&v)[4], float (&stored)[4]) {
-        store_vec_cs(p, v, stored);
+    static __device__ __forceinline__ void store(float *p, const float2 (&v)[2], float2 (&stored)[2]) {
+        __stcs(reinterpret_cast<float4 *>(p), make_float4(v[0].x, v[0].y, v[1].x, v[1].y));
+        stored[0] = v[0];
+        stored[1] = v[1];
     }
-    static __device__ __forceinline__ void store(float *p, const float (&v)[4]) { store_vec_cs(p, v); }
+    static __device__ __forceinline__ void store(float *p, const float2 (&v)[2]) {
+        __stcs(reinterpret_cast<float4 *>(p), make_float4(v[0].x, v[0].y, v[1].x, v[1].y));
+    }
 };
+__device__ __forceinline__ float2 widen_pair(uint32_t w) {
+    float2 f;
+    widen_bf16x2(w, f.x, f.y);
+    return f;
+}
 template <> struct VecIO<__nv_bfloat16, 8> {
-    static __device__ __forceinline__ void load_smem(const unsigned char *p, float (&v)[8]) {
+    static __device__ __forceinline__ void load_smem(const unsigned char *p, float2 (&v)[4]) {
         const uint4 q = *reinterpret_cast<const uint4 *>(p);
-        widen_bf16x2(q.x, v[0], v[1]);
-        widen_bf16x2(q.y, v[2], v[3]);
-        widen_bf16x2(q.z, v[4], v[5]);
-        widen_bf16x2(q.w, v[6], v[7]);
+        v[0] = widen_pair(q.x);
+        v[1] = widen_pair(q.y);
+        v[2] = widen_pair(q.z);
+        v[3] = widen_pair(q.w);
     }
-    static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float (&v)[8],
-                                                 float (&stored)[8]) {
-        store_vec_cs(p, v, stored);
+    static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float2 (&v)[4],
+                                                 float2 (&stored)[4]) {
+        uint4 q;
+        q.x = pack_bf16x2_rn(v[0].x, v[0].y);
+        q.y = pack_bf16x2_rn(v[1].x, v[1].y);
+        q.z = pack_bf16x2_rn(v[2].x, v[2].y);
+        q.w = pack_bf16x2_rn(v[3].x, v[3].y);
+        __stcs(reinterpret_cast<uint4 *>(p), q);
+        stored[0] = widen_pair(q.x);
+        stored[1] = widen_pair(q.y);
+        stored[2] = widen_pair(q.z);
+        stored[3] = widen_pair(q.w);
     }
-    static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float (&v)[8]) {
-        store_vec_cs(p, v);
+    static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float2 (&v)[4]) {
+        uint4 q;
+        q.x = pack_bf16x2_rn(v[0].x, v[0].y);
+        q.y = pack_bf16x2_rn(v[1].x, v[1].y);
+        q.z = pack_bf16x2_rn(v[2].x, v[2].y);
+        q.w = pack_bf16x2_rn(v[3].x, v[3].y);
+        __stcs(reinterpret_cast<uint4 *>(p), q);
     }
 };
 template <> struct VecIO<__nv_bfloat16, 4> {
-    static __device__ __forceinline__ void load_smem(const unsigned char *p, float (&v)[4]) {
+    static __device__ __forceinline__ void load_smem(const unsigned char *p, float2 (&v)[2]) {
         const uint2 q = *reinterpret_cast<const uint2 *>(p);
-        widen_bf16x2(q.x, v[0], v[1]);
-        widen_bf16x2(q.y, v[2], v[3]);
+        v[0] = widen_pair(q.x);
+        v[1] = widen_pair(q.y);
     }
-    static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float (&v)[4],
-                                                 float (&stored)[4]) {
+    static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float2 (&v)[2],
+                                                 float2 (&stored)[2]) {
         uint2 q;
-        q.x = pack_bf16x2_rn(v[0], v[1]);
-        q.y = pack_bf16x2_rn(v[2], v[3]);
+        q.x = pack_bf16x2_rn(v[0].x, v[0].y);
+        q.y = pack_bf16x2_rn(v[1].x, v[1].y);
         __stcs(reinterpret_cast<uint2 *>(p), q);
-        widen_bf16x2(q.x, stored[0], stored[1]);
-        widen_bf16x2(q.y, stored[2], stored[3]);
+        stored[0] = widen_pair(q.x);
+        stored[1] = widen_pair(q.y);
     }
-    static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float (&v)[4]) {
+    static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float2 (&v)[2]) {
         uint2 q;
-        q.x = pack_bf16x2_rn(v[0], v[1]);
-        q.y = pack_bf16x2_rn(v[2], v[3]);
+        q.x = pack_bf16x2_rn(v[0].x, v[0].y);
+        q.y = pack_bf16x2_rn(v[1].x, v[1].y);
         __stcs(reinterpret_cast<uint2 *>(p), q);
     }
 };
@@ -441,7 +466,8 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
                     ph ^= 1u;
                 }
                 const unsigned char *st = gring + (size_t)cs * sh.stage_bytes + (size_t)gt * VB;
-                float h[N][V], yv[V];
+                constexpr int VP = V / 2;  // element pairs per thread
+                float2 h[N][VP], yv[VP];
                 if (active) {
 #pragma unroll
                     for (int ii = 0; ii < N; ++ii) VecIO<S, V>::load_smem(st + ii * row_bytes, h[ii]);
@@ -450,7 +476,7 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&gempty[cs]);  // stage data is in registers
                 if (active) {
-                    float hr[V];
+                    float2 hr[VP];
                     if constexpr (WRITE) {
                         S *Hot = Ho + t * N * d + k;
 #pragma unroll
@@ -459,47 +485,54 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
                             float col[N];
 #pragma unroll
                             for (int ii = 0; ii < N; ++ii) col[ii] = P[jj * N + ii];
-                            float acc[V], stored[V];
+                            float2 acc[VP], stored[VP];
+                            const float2 c0 = make_float2(col[0], col[0]);
 #pragma unroll
-                            for (int e = 0; e < V; ++e) acc[e] = __fmul_rn(col[0], h[0][e]);
+                            for (int e = 0; e < VP; ++e) acc[e] = fmul2_rn(c0, h[0][e]);
 #pragma unroll
                             for (int ii = 1; ii < N; ++ii) {
+                                const float2 ci = make_float2(col[ii], col[ii]);
 #pragma unroll
-                                for (int e = 0; e < V; ++e) acc[e] = __fmaf_rn(col[ii], h[ii][e], acc[e]);
+                                for (int e = 0; e < VP; ++e) acc[e] = ffma2_rn(ci, h[ii][e], acc[e]);
                             }
+                            const float2 cb = make_float2(bv[jj], bv[jj]);
 #pragma unroll
-                            for (int e = 0; e < V; ++e) acc[e] = __fmaf_rn(bv[jj], yv[e], acc[e]);
+                            for (int e = 0; e < VP; ++e) acc[e] = ffma2_rn(cb, yv[e], acc[e]);
                             VecIO<S, V>::store(Hot + jj * d, acc, stored);
                             if constexpr (READ) {
+                                const float2 ca = make_float2(av[jj], av[jj]);
                                 if (jj == 0) {
 #pragma unroll
-                                    for (int e = 0; e < V; ++e) hr[e] = __fmul_rn(av[0], stored[e]);
+                                    for (int e = 0; e < VP; ++e) hr[e] = fmul2_rn(ca, stored[e]);
                                 } else {
 #pragma unroll
-                                    for (int e = 0; e < V; ++e) hr[e] = __fmaf_rn(av[jj], stored[e], hr[e]);
+                                    for (int e = 0; e < VP; ++e) hr[e] = ffma2_rn(ca, stored[e], hr[e]);
                                 }
                             }
                         }
                     } else {
+                        const float2 c0 = make_float2(av[0], av[0]);
 #pragma unroll
-                        for (int e = 0; e < V; ++e) hr[e] = __fmul_rn(av[0], h[0][e]);
+                        for (int e = 0; e < VP; ++e) hr[e] = fmul2_rn(c0, h[0][e]);
 #pragma unroll
                         for (int ii = 1; ii < N; ++ii) {
+                            const float2 ci = make_float2(av[ii], av[ii]);
 #pragma unroll
-                            for (int e = 0; e < V; ++e) hr[e] = __fmaf_rn(av[ii], h[ii][e], hr[e]);
+                            for (int e = 0; e < VP; ++e) hr[e] = ffma2_rn(ci, h[ii][e], hr[e]);
                         }
                     }
                     if constexpr (READ) {
 #pragma unroll
-                        for (int e = 0; e < V; ++e) {
-                            const double hv = (double)hr[e];
-                            ss = __fma_rn(hv, hv, ss);
+                        for (int e = 0; e < VP; ++e) {
+                            const double hx = (double)hr[e].x, hy = (double)hr[e].y;
+                            ss = __fma_rn(hx, hx, ss);
+                            ss = __fma_rn(hy, hy, ss);
                         }
                         // keep h for the normalisation (this thread reads it back itself)
 #pragma unroll
-                        for (int e = 0; e < V; e += 4)
-                            *reinterpret_cast<float4 *>(hcur + k + e) =
-                                make_float4(hr[e], hr[e + 1], hr[e + 2], hr[e + 3]);
+                        for (int e = 0; e < VP; e += 2)
+                            *reinterpret_cast<float4 *>(hcur + k + 2 * e) =
+                                make_float4(hr[e].x, hr[e].y, hr[e + 1].x, hr[e + 1].y);
                     }
                 }
             }
@@ -520,15 +553,20 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
                         r_prev = __double2float_rn(1.0 / sqrt(tot / (double)d + (double)p.eps));
                     }
                     if (active) {
-                        float gv[V], hv[V], xv[V];
+                        constexpr int VP = V / 2;
+                        float gv[V];
+                        float2 hv[VP], xv[VP];
                         load_gain<V>(p.g, k, gv);
 #pragma unroll
-                        for (int e = 0; e < V; e += 4) {
-                            const float4 f = *reinterpret_cast<const float4 *>(hprev + k + e);
-                            hv[e] = f.x; hv[e + 1] = f.y; hv[e + 2] = f.z; hv[e + 3] = f.w;
+                        for (int e = 0; e < VP; e += 2) {
+                            const float4 f = *reinterpret_cast<const float4 *>(hprev + k + 2 * e);
+                            hv[e] = make_float2(f.x, f.y);
+                            hv[e + 1] = make_float2(f.z, f.w);
                         }
+                        const float2 r2 = make_float2(r_prev, r_prev);
 #pragma unroll
-                        for (int e = 0; e < V; ++e) xv[e] = __fmul_rn(__fmul_rn(hv[e], r_prev), gv[e]);
+                        for (int e = 0; e < VP; ++e)
+                            xv[e] = fmul2_rn(fmul2_rn(hv[e], r2), make_float2(gv[2 * e], gv[2 * e + 1]));
                         VecIO<S, V>::store(X + t_prev * d + k, xv);
                     }
                 }
