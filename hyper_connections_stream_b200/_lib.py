@@ -37,6 +37,7 @@ SIGNATURES = {
     "hc_set_path": ([_i32], _i32),
     "hc_get_path": ([], _i32),
     "hc_device_fault": ([C.POINTER(_i32), _vp], _i32),
+    "hc_selftest_bounded_wait": ([_i32, _vp], _i32),
     "hc_status_string": ([_i32], C.c_char_p),
     "hc_last_error": ([], C.c_char_p),
     "hc_version": ([], _i32),
@@ -138,6 +139,11 @@ def device_fault(device=None) -> int:
     if st not in (HC_OK, HC_ERR_DEVICE):
         _check(st)
     return int(code.value)
+
+
+def selftest_bounded_wait(limit_us: int = 1000, device=None) -> None:
+    """Launch the bounded-wait self-test (see hc_selftest_bounded_wait)."""
+    _check(lib().hc_selftest_bounded_wait(int(limit_us), _stream(device)))
 
 
 def sinkhorn(logits: torch.Tensor, K: int, out: torch.Tensor | None = None) -> torch.Tensor:

@@ -204,6 +204,16 @@ hc_status hc_device_fault(int *code, hc_stream stream) {
     return v ? fail(HC_ERR_DEVICE, "device fault code 0x%x", v) : HC_OK;
 }
 
+hc_status hc_selftest_bounded_wait(int limit_us, hc_stream stream) {
+    g_last_error[0] = '\0';
+    if (limit_us < 1 || limit_us > 100000)
+        return fail(HC_ERR_INVALID_ARG, "hc_selftest_bounded_wait: limit_us = %d not in [1, 100000]",
+                    limit_us);
+    hc::LaunchCtx ctx{};
+    HC_TRY(launch_ctx(ctx));
+    return hc::launch_selftest_wait(limit_us, ctx, static_cast<cudaStream_t>(stream));
+}
+
 hc_status hc_sinkhorn(const float *logits, float *out, int64_t T, int n, int K, hc_stream stream) {
     static const char *fn = "hc_sinkhorn";
     g_last_error[0] = '\0';

@@ -127,9 +127,11 @@ __device__ __forceinline__ void load_gain(const float *g, int64_t k, float (&gv)
 // A warp is split into groups of GL lanes; each group owns one token, and
 // lane q of a group holds elements e = q + GL * r (r < EPL) of the row-major
 // n x n matrix, so every lane performs one (or two) of the n*n divisions of
-// a pass in parallel. Row and column sums read the group's values from a
-// small per-warp shared-memory buffer (kGroupScratch floats), where the n
-// loads of a sum are independent and overlap.
+// a pass in parallel. With one element per lane (n <= 5) a row or column sum
+// gathers its n values with independent shuffles; with two (n = 6..8) it
+// reads them from a small per-warp shared-memory buffer (kGroupScratch
+// floats). Either way the n fetches of a sum overlap and the additions run
+// in index order.
 // ---------------------------------------------------------------------------
 template <int N> struct Group {
     static constexpr int NN = N * N;
@@ -166,6 +168,32 @@ __device__ __forceinline__ void group_sinkhorn(float (&m)[R][Group<N>::EPL], flo
     for (int b = 0; b < R; ++b) {
 #pragma unroll
         for (int r = 0; r < EPL; ++r) m[b][r] = expf(m[b][r]);
+    }
+    if constexpr (EPL == 1) {
+        // one element per lane: the n values of a row (column) are fetched
+        // with independent shuffles and added in index order
+        const int base = lane & ~(GL - 1);
+        for (int it = 0; it < K; ++it) {
+#pragma unroll
+            for (int pass = 0; pass < 2; ++pass) {
+                float s[R];
+#pragma unroll
+                for (int b = 0; b < R; ++b) {
+                    float v[N];
+#pragma unroll
+                    for (int k = 0; k < N; ++k)
+                        v[k] = __shfl_sync(0xffffffffu, m[b][0],
+                                           base + (pass == 0 ? row[0] * N + k : k * N + col[0]));
+                    float acc = 0.0f;
+#pragma unroll
+                    for (int k = 0; k < N; ++k) acc = __fadd_rn(acc, v[k]);
+                    s[b] = acc;
+                }
+#pragma unroll
+                for (int b = 0; b < R; ++b) m[b][0] = __fdiv_rn(m[b][0], s[b]);
+            }
+        }
+        return;
     }
     for (int it = 0; it < K; ++it) {
 #pragma unroll

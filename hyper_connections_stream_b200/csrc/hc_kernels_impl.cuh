@@ -6,7 +6,8 @@
 //     whenever at least two ring stages fit in shared memory next to the
 //     groups' fp32 rows of h (normalising kinds);
 //   register-streaming (hc_stream_kernels.cuh): no shared-memory staging;
-//     covers the larger d of the normalising kinds and can be forced.
+//     covers the larger d of the normalising kinds and small (decode-sized)
+//     calls, and can be forced.
 #pragma once
 
 #include "hc_launch.h"
@@ -135,7 +136,12 @@ hc_status launch_n(const StepParams &p, const LaunchCtx &ctx, cudaStream_t st) {
     if (ctx.path == 1 && !pipe_ok)
         return set_error(HC_ERR_UNSUPPORTED, "pipelined kernels do not cover d = %lld here",
                          (long long)p.d);
-    if (ctx.path == 2 || !pipe_ok) {
+    // Small calls (decode-sized batches) finish sooner without the pipeline's
+    // set-up: below ~64 MiB of stream traffic the register-streaming family
+    // wins on B200 (measured crossover: n = 4, d = 7168 at ~450 tokens;
+    // d = 4096 at ~1000; n = 8 at ~600).
+    const bool small = p.T * (int64_t)N * p.d * (int64_t)sizeof(S) * 2 < (int64_t(64) << 20);
+    if (ctx.path == 2 || !pipe_ok || (ctx.path == 0 && small)) {
         if (KIND != KIND_WRITE && p.d > (int64_t)kStreamMaxThreads * 8 * StorageTraits<S>::V)
             return set_error(HC_ERR_UNSUPPORTED, "d = %lld too large", (long long)p.d);
         return launch_stream<N, S, KIND>(p, ctx, st);

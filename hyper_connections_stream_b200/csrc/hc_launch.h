@@ -23,6 +23,8 @@ hc_status set_error(hc_status st, const char *fmt, ...);
 template <typename S, int KIND>
 hc_status launch_kind(int n, const StepParams &p, const LaunchCtx &ctx, cudaStream_t st);
 
+hc_status launch_selftest_wait(int limit_us, const LaunchCtx &ctx, cudaStream_t st);
+
 hc_status launch_sinkhorn(const float *L, float *out, int64_t T, int n, int K,
                           const LaunchCtx &ctx, cudaStream_t st);
 

@@ -142,12 +142,13 @@ HC_API hc_status hc_write_then_read(const void *H, const void *y, void *Hout, vo
 /*
  * Kernel family used by the step calls (process-wide; default HC_PATH_AUTO).
  *   HC_PATH_PIPELINED: warp-specialised kernels fed by bulk copies (TMA) into
- *     a shared-memory ring; the automatic choice wherever it applies (two or
- *     more ring stages fit and, for calls that normalise, d <= 8 tiles of
- *     1792 bf16 / 896 fp32 elements). Forcing it where it does not apply
- *     returns HC_ERR_UNSUPPORTED.
+ *     shared-memory rings; the automatic choice for calls that move 64 MiB
+ *     or more of stream state, where its rings fit (for calls that normalise,
+ *     two fp32 rows of d per consumer group must fit next to them: d up to
+ *     9880 bf16 at n = 4). Forcing it where it does not fit returns
+ *     HC_ERR_UNSUPPORTED.
  *   HC_PATH_REGISTER: register-streaming kernels (no staging); the automatic
- *     choice for the larger d.
+ *     choice for smaller calls (decode-sized batches) and larger d.
  * Both families compute bit-identical results.
  */
 typedef enum { HC_PATH_AUTO = 0, HC_PATH_PIPELINED = 1, HC_PATH_REGISTER = 2 } hc_path;
@@ -164,6 +165,16 @@ HC_API hc_path hc_get_path(void);
  * 4 parameter wait, 8 reduction wait, 16 drain at exit, 32 self-test.
  */
 HC_API hc_status hc_device_fault(int *code, hc_stream stream);
+
+/*
+ * Self-test of the bounded waits (the mechanism, not the method; the pages
+ * have no counterpart). Launches one tiny kernel whose single wait is on a
+ * barrier that nothing arrives at, limited to limit_us microseconds
+ * (1..100000). The wait gives up, code 32 is ORed into the device fault word
+ * and the kernel returns normally: no trap, no copy in flight, the context
+ * stays usable. Read the result with hc_device_fault(). Asynchronous.
+ */
+HC_API hc_status hc_selftest_bounded_wait(int limit_us, hc_stream stream);
 
 /* Static English text for a status code. */
 HC_API const char *hc_status_string(hc_status st);

@@ -37,7 +37,8 @@ def test_library_exports_every_declared_entry_point():
     lib = C.CDLL(path)
     declared = _declared_entry_points()
     assert {"hc_sinkhorn", "hc_read_rmsnorm", "hc_write_mix", "hc_write_then_read",
-            "hc_status_string", "hc_last_error", "hc_version"} <= declared
+            "hc_status_string", "hc_last_error", "hc_version", "hc_set_path", "hc_get_path",
+            "hc_device_fault", "hc_selftest_bounded_wait"} <= declared
     for name in declared:
         assert hasattr(lib, name), name
     from hyper_connections_stream_b200 import _lib
@@ -100,6 +101,9 @@ _CHILD = textwrap.dedent(r"""
     call("sk_null", "hc_sinkhorn", None, A, T, 4, 20, None)
     call("sk_alias", "hc_sinkhorn", A, A + 4, T, 4, 20, None)
     call("sk_T0", "hc_sinkhorn", None, None, 0, 4, 20, None)
+    call("st_lo", "hc_selftest_bounded_wait", 0, None)
+    call("st_hi", "hc_selftest_bounded_wait", 1000000, None)
+    call("path_bad", "hc_set_path", 7)
     print(json.dumps(res))
 """)
 
@@ -120,7 +124,7 @@ def test_argument_validation_statuses():
         "eps_nan": INV, "eps_inf": INV, "null_H": INV, "null_A": INV, "null_b": INV,
         "mis_H": MIS, "mis_x": MIS, "mis_g": MIS, "mis_A": MIS, "alias_partial": ALI,
         "alias_y": ALI, "alias_x_H": ALI, "alias_x_read": ALI, "sk_n0": INV, "sk_K0": INV,
-        "sk_null": INV, "sk_alias": ALI, "sk_T0": OK,
+        "sk_null": INV, "sk_alias": ALI, "sk_T0": OK, "st_lo": INV, "st_hi": INV, "path_bad": INV,
     }
     for tag, code in want.items():
         got, msg = res[tag]
