@@ -38,6 +38,7 @@ SIGNATURES = {
     "hc_get_path": ([], _i32),
     "hc_device_fault": ([C.POINTER(_i32), _vp], _i32),
     "hc_selftest_bounded_wait": ([_i32, _vp], _i32),
+    "hc_mix_logits": ([_vp, _vp, _vp, _i32, _i64, _i32, _i64, _i32, _f32, _vp], _i32),
     "hc_status_string": ([_i32], C.c_char_p),
     "hc_last_error": ([], C.c_char_p),
     "hc_version": ([], _i32),
@@ -99,16 +100,24 @@ def _need_cuda(name, t, dtype=None):
 
 
 def _tok_param(name, p, T, per_shape):
-    """Shared ([*per_shape]) or per-token ([T, *per_shape]) fp32 parameter ->
-    token stride in floats."""
-    _need_cuda(name, p, torch.float32)
+    """Shared ([*per_shape], contiguous) or per-token ([T, *per_shape]) fp32
+    parameter -> token stride in floats. A per-token parameter may be a view
+    whose tokens are `stride(0)` floats apart as long as each token's set is
+    contiguous (e.g. a slice of the [T, P] output of mix_logits)."""
+    if not isinstance(p, torch.Tensor) or not p.is_cuda or p.dtype != torch.float32:
+        raise ValueError(f"{name} must be a float32 CUDA tensor")
     per = 1
     for s in per_shape:
         per *= s
     if tuple(p.shape) == tuple(per_shape):
+        if not p.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
         return 0
     if tuple(p.shape) == (T, *per_shape):
-        return per
+        inner = p[0] if T > 0 else p.reshape(per_shape)
+        if T > 0 and not inner.is_contiguous():
+            raise ValueError(f"{name}: each token's values must be contiguous")
+        return p.stride(0) if T > 1 else per
     raise ValueError(f"{name} must have shape {tuple(per_shape)} or {(T, *per_shape)}, "
                      f"got {tuple(p.shape)}")
 
@@ -139,6 +148,23 @@ def device_fault(device=None) -> int:
     if st not in (HC_OK, HC_ERR_DEVICE):
         _check(st)
     return int(code.value)
+
+
+def mix_logits(H, W, *, eps: float = 1e-6, out=None):
+    """Per-token mixing logits on the tensor cores: out[t, j] = r_t * (u_t . W[j])
+    with u_t = H[t] flattened and r_t its inverse RMS. H [T, n, d] bf16,
+    W [P, n*d] bf16 -> out [T, P] fp32."""
+    _need_cuda("H", H, torch.bfloat16)
+    T, n, d = _streams_shape(H)
+    _need_cuda("W", W, torch.bfloat16)
+    if W.dim() != 2 or W.shape[1] != n * d:
+        raise ValueError(f"W must be [P, n*d = {n * d}], got {tuple(W.shape)}")
+    P = W.shape[0]
+    out = torch.empty((T, P), dtype=torch.float32, device=H.device) if out is None else out
+    _need_cuda("out", out, torch.float32)
+    _check(lib().hc_mix_logits(_ptr(H), _ptr(W), _ptr(out), HC_BF16, T, n, d, P, float(eps),
+                               _stream(H.device)))
+    return out
 
 
 def selftest_bounded_wait(limit_us: int = 1000, device=None) -> None:

@@ -204,6 +204,30 @@ hc_status hc_device_fault(int *code, hc_stream stream) {
     return v ? fail(HC_ERR_DEVICE, "device fault code 0x%x", v) : HC_OK;
 }
 
+hc_status hc_mix_logits(const void *H, const void *W, float *logits, hc_dtype dt, int64_t T, int n,
+                        int64_t d, int P, float eps, hc_stream stream) {
+    static const char *fn = "hc_mix_logits";
+    g_last_error[0] = '\0';
+    const Shape s{dt, T, n, d};
+    HC_TRY(check_shape(fn, s, false));
+    if (dt != HC_BF16) return fail(HC_ERR_UNSUPPORTED, "%s: only bf16 streams and weights", fn);
+    if (P < 1) return fail(HC_ERR_INVALID_ARG, "%s: P = %d < 1", fn, P);
+    if (P > 256) return fail(HC_ERR_UNSUPPORTED, "%s: P = %d > 256", fn, P);
+    HC_TRY(check_eps(fn, eps));
+    if (T > (int64_t)0x7fffffff || (int64_t)n * d > (int64_t)0x7fffffff)
+        return fail(HC_ERR_UNSUPPORTED, "%s: T or n*d beyond 2^31", fn);
+    if (T == 0) return HC_OK;
+    HC_TRY(check_buf(fn, "H", H));
+    HC_TRY(check_buf(fn, "W", W));
+    HC_TRY(check_param(fn, "logits", logits));
+    const int64_t hb = T * n * d * 2, wb = (int64_t)P * n * d * 2, zb = T * P * 4;
+    if (overlap(logits, zb, H, hb) || overlap(logits, zb, W, wb))
+        return fail(HC_ERR_ALIAS, "%s: logits overlap H or W", fn);
+    hc::LaunchCtx ctx{};
+    HC_TRY(launch_ctx(ctx));
+    return hc::launch_mix_logits(H, W, logits, T, n, d, P, eps, ctx, static_cast<cudaStream_t>(stream));
+}
+
 hc_status hc_selftest_bounded_wait(int limit_us, hc_stream stream) {
     g_last_error[0] = '\0';
     if (limit_us < 1 || limit_us > 100000)

@@ -193,39 +193,39 @@ __device__ __forceinline__ void group_sinkhorn(float (&m)[R][Group<N>::EPL], flo
                 for (int b = 0; b < R; ++b) m[b][0] = __fdiv_rn(m[b][0], s[b]);
             }
         }
-        return;
-    }
-    for (int it = 0; it < K; ++it) {
+    } else {
+        for (int it = 0; it < K; ++it) {
 #pragma unroll
-        for (int pass = 0; pass < 2; ++pass) {
+            for (int pass = 0; pass < 2; ++pass) {
 #pragma unroll
-            for (int b = 0; b < R; ++b) {
-                float *buf = scratch + b * kGroupScratch + (lane / GL) * NN;
+                for (int b = 0; b < R; ++b) {
+                    float *buf = scratch + b * kGroupScratch + (lane / GL) * NN;
 #pragma unroll
-                for (int r = 0; r < EPL; ++r)
-                    if (own[r]) buf[e[r]] = m[b][r];
-            }
-            __syncwarp();
-            float s[R][EPL];
-#pragma unroll
-            for (int b = 0; b < R; ++b) {
-                const float *buf = scratch + b * kGroupScratch + (lane / GL) * NN;
-#pragma unroll
-                for (int r = 0; r < EPL; ++r) {
-                    float v[N];
-#pragma unroll
-                    for (int k = 0; k < N; ++k) v[k] = pass == 0 ? buf[row[r] * N + k] : buf[k * N + col[r]];
-                    float acc = 0.0f;
-#pragma unroll
-                    for (int k = 0; k < N; ++k) acc = __fadd_rn(acc, v[k]);
-                    s[b][r] = acc;
+                    for (int r = 0; r < EPL; ++r)
+                        if (own[r]) buf[e[r]] = m[b][r];
                 }
-            }
-            __syncwarp();
+                __syncwarp();
+                float s[R][EPL];
 #pragma unroll
-            for (int b = 0; b < R; ++b) {
+                for (int b = 0; b < R; ++b) {
+                    const float *buf = scratch + b * kGroupScratch + (lane / GL) * NN;
 #pragma unroll
-                for (int r = 0; r < EPL; ++r) m[b][r] = __fdiv_rn(m[b][r], s[b][r]);
+                    for (int r = 0; r < EPL; ++r) {
+                        float v[N];
+#pragma unroll
+                        for (int k = 0; k < N; ++k) v[k] = pass == 0 ? buf[row[r] * N + k] : buf[k * N + col[r]];
+                        float acc = 0.0f;
+#pragma unroll
+                        for (int k = 0; k < N; ++k) acc = __fadd_rn(acc, v[k]);
+                        s[b][r] = acc;
+                    }
+                }
+                __syncwarp();
+#pragma unroll
+                for (int b = 0; b < R; ++b) {
+#pragma unroll
+                    for (int r = 0; r < EPL; ++r) m[b][r] = __fdiv_rn(m[b][r], s[b][r]);
+                }
             }
         }
     }

@@ -176,6 +176,25 @@ HC_API hc_status hc_device_fault(int *code, hc_stream stream);
  */
 HC_API hc_status hc_selftest_bounded_wait(int limit_us, hc_stream stream);
 
+/*
+ * Input-dependent mixing logits (the "learned matrices" of the glossary entry
+ * computed from the streams themselves; reading: an RMS-normalised linear map
+ * of the token's flattened streams). For every token t:
+ *   u_t = H[t] flattened to n*d values,  r_t = 1 / sqrt(mean(u_t^2) + eps),
+ *   logits[t][j] = r_t * sum_k u_t[k] * W[j][k]      (j < P)
+ *   H [T][n][d] bf16, W [P][n*d] bf16 (row j = the weights of logit j),
+ *   logits [T][P] fp32 out. P <= 256; with P = n*n + 2n the three blocks
+ *   [n*n | n | n] can feed hc_write_then_read directly as per-token Sinkhorn
+ *   logits, read logits and write gains (token stride P).
+ * Runs on the 5th-generation tensor cores (bf16 x bf16 -> fp32, TMEM
+ * accumulator) with the sum of squares in fp64; the sum over k is in the
+ * tensor core's order, so results match an exact evaluation within fp32
+ * accumulation error, not bit for bit. H, W 16-byte aligned; logits 4-byte
+ * aligned and disjoint from H and W. bf16 only (HC_ERR_UNSUPPORTED otherwise).
+ */
+HC_API hc_status hc_mix_logits(const void *H, const void *W, float *logits, hc_dtype dt,
+                               int64_t T, int n, int64_t d, int P, float eps, hc_stream stream);
+
 /* Static English text for a status code. */
 HC_API const char *hc_status_string(hc_status st);
 

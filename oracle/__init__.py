@@ -40,6 +40,7 @@ def lib():
             "hco_write_then_read": ([vp, vp, vp, vp, i32, i64, i32, i64, i32, vp, i64, i32,
                                      vp, i64, i32, vp, i64, vp, fp], i32),
             "hco_block_tanh": ([vp, vp, i32, i64], i32),
+            "hco_mix_logits": ([vp, vp, vp, i32, i64, i32, i64, i32, fp], i32),
             "hco_single_stream_layer": ([vp, vp, i32, i64, i64, vp, fp], i32),
         }
         for name, (args, res) in sig.items():
@@ -156,6 +157,18 @@ def write_then_read(H, y, A, b, a, g, eps: float, dt: str, K: int = 0,
                                    _tok_stride(a, T, n), _p(g), float(eps)),
          "write_then_read")
     return Hout, x
+
+
+def mix_logits(H, W, eps: float, dt: str):
+    """fp64 logits z[t, j] = r_t * sum_k u_t[k] W[j, k], u_t = H[t] flattened,
+    r_t = 1 / sqrt(mean(u_t^2) + eps). H [T, n, d]; W [P, n*d]."""
+    H = _arr(H, _NP[dt]); W = _arr(W, _NP[dt])
+    T, n, d = H.shape
+    P = W.shape[0]
+    assert W.shape == (P, n * d)
+    z = np.empty((T, P), dtype=np.float64)
+    _chk(lib().hco_mix_logits(_p(H), _p(W), _p(z), _DT[dt], T, n, d, P, float(eps)), "mix_logits")
+    return z
 
 
 def block_tanh(x, dt: str):

@@ -325,6 +325,36 @@ int hco_write_then_read(const void *H, const void *y, void *Hout, void *x_next, 
     return err;
 }
 
+/*
+ * Input-dependent mixing logits (the step's per-token parameters computed from
+ * the streams themselves; the glossary entry only says the mixing matrices are
+ * learned). Reading: u = the token's n*d stream values flattened, r = 1 /
+ * sqrt(mean(u^2) + eps), z[j] = r * sum_k u[k] * W[j][k] for j < P.
+ * W is [P][n*d] in storage dtype dt (row j = the weights of logit j).
+ * Computed in fp64 (no rounding but the final one to fp64), as a reference.
+ */
+int hco_mix_logits(const void *H, const void *W, double *z, int dt, int64_t T, int n, int64_t d,
+                   int P, float eps) {
+    if (check_common(dt, T, n, d) || P < 1) return HCO_EINVAL;
+    const int64_t K = (int64_t)n * d;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        double ss = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            const double u = (double)load_s(H, dt, t * K + k);
+            ss += u * u;
+        }
+        const double r = 1.0 / sqrt(ss / (double)K + (double)eps);
+        for (int j = 0; j < P; ++j) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += (double)load_s(H, dt, t * K + k) * (double)load_s(W, dt, (int64_t)j * K + k);
+            z[t * P + j] = r * acc;
+        }
+    }
+    return HCO_OK;
+}
+
 /* Harness block stand-in: y = round_s(tanhf(x)). Not part of the HC step. */
 int hco_block_tanh(const void *x, void *y, int dt, int64_t count) {
     if (dt != HCO_F32 && dt != HCO_BF16) return HCO_EINVAL;

@@ -419,3 +419,45 @@ def test_state_size_worked_example():
     assert four == g["n_stream_bytes_per_token"]
     assert four - one == g["extra_bytes_per_token"]
     assert four * g["tokens_in_flight"] == g["live_state_bytes"]
+
+
+# --------------------------------------------------------------------------
+# input-dependent mixing logits
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_mix_logits_against_library_matmul(dt):
+    """z = rms-normalised flattened streams times W^T, checked against the
+    library's fp64 matmul and norm."""
+    T, n, d = 9, 4, 96
+    P = n * n + 2 * n
+    H = gen.to_storage(gen.normal(151, (T, n, d)), dt)
+    W = gen.to_storage(gen.normal(152, (P, n * d), std=0.05), dt)
+    z = oracle.mix_logits(H, W, 1e-6, dt)
+    u = torch.from_numpy(f32_of(H, dt).reshape(T, n * d))
+    Wt = torch.from_numpy(f32_of(W, dt))
+    ref = torch.nn.functional.rms_norm(u, (n * d,), eps=float(np.float32(1e-6))) @ Wt.T
+    assert np.max(np.abs(z - ref.numpy())) < 1e-12 * (1 + np.max(np.abs(ref.numpy())))
+
+
+def test_mix_logits_closed_forms():
+    """A one-hot weight row picks a single stream value times r; a constant
+    token gives z = c / sqrt(c^2 + eps) * sum of the row."""
+    T, n, d = 3, 2, 16
+    K = n * d
+    H = gen.normal(153, (T, n, d))
+    W = np.zeros((3, K), np.float32)
+    W[0, 5] = 1.0          # stream 0, channel 5
+    W[1, d + 2] = -2.0     # stream 1, channel 2
+    W[2, :] = 0.5
+    z = oracle.mix_logits(H, W, 0.0, "f32")
+    u = H.reshape(T, K).astype(np.float64)
+    r = 1.0 / np.sqrt(np.mean(u * u, axis=1))
+    assert np.allclose(z[:, 0], r * u[:, 5], rtol=1e-14)
+    assert np.allclose(z[:, 1], -2.0 * r * u[:, d + 2], rtol=1e-14)
+    c = np.full((1, n, d), 0.75, np.float32)
+    zc = oracle.mix_logits(c, W, 0.25, "f32")
+    want = 0.75 / math.sqrt(0.75 ** 2 + 0.25) * np.array([0.0, 0.0, 0.5 * K])
+    want[0] = 0.75 / math.sqrt(0.75 ** 2 + 0.25)
+    want[1] = -2.0 * 0.75 / math.sqrt(0.75 ** 2 + 0.25)
+    assert np.allclose(zc[0], want, rtol=1e-14)
