@@ -170,6 +170,58 @@ def make_inputs(w, rank, device):
                 g=torch.ones(d, dtype=torch.float32, device=device))
 
 
+def run_logits(args):
+    """The input-dependent mixing logits (tensor-core GEMM with an RMS scale)
+    on the workload's streams: T=16384 tokens, n=4, d=7168, P=24 logits.
+    Kernel-only, device-timed; one launch per step."""
+    import numpy as np
+    import torch
+    import hc_inputs as gen
+    from hyper_connections_stream_b200 import _lib as hc
+    ws, rank, local = _dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = dict(WORKLOAD)
+    if args.tokens:
+        w["T"] = args.tokens
+    T, n, d = w["T"], w["n"], w["d"]
+    P, K = n * n + 2 * n, n * d
+    H = gen.device_normal(gen.SEED_H + w["cfg"], (T, n, d), torch.bfloat16, device)
+    W = gen.device_normal(503, (P, K), torch.bfloat16, device, std=1.0 / np.sqrt(K))
+    z = torch.empty((T, P), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    for _ in range(args.warmup):
+        hc.mix_logits(H, W, eps=w["eps"], out=z)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        hc.mix_logits(H, W, eps=w["eps"], out=z)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    per = [s.elapsed_time(e) for s, e in ev]
+    total_ms = ev[0][0].elapsed_time(ev[-1][1])
+    kern_ms = statistics.mean(per)
+    alg_bytes = T * K * 2 + P * K * 2 + T * P * 4
+    flops = 2 * T * K * P
+    peak, peak_kind = _peaks()
+    achieved = alg_bytes / (kern_ms / 1e3) / 1e9
+    return {
+        "metric": "mixing-logits tokens/sec at n=4, d=7168 (bf16 streams, P=24, tensor cores)",
+        "value": T * args.steps / (total_ms / 1e3), "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "mix_logits", "T": T, "n": n, "d": d, "P": P},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "peak_source": peak_kind,
+                     "algorithmic_bytes_per_launch": alg_bytes, "kernel_ms": kern_ms,
+                     "tensor_tflops": flops / (kern_ms / 1e3) / 1e12},
+        "gpu_launches": args.steps, "device_fault": hc.device_fault(),
+    }
+
+
 def run_ours(args):
     import torch
     from hyper_connections_stream_b200 import _lib as hc
@@ -414,6 +466,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-only", action="store_true",
                     help="device-timed kernel only (no e2e, no CPU baseline): for profiling")
+    ap.add_argument("--op", choices=["step", "logits"], default="step",
+                    help="step: the fused HC step (the metric); logits: the tensor-core "
+                         "mixing-logits kernel on the same streams")
     ap.add_argument("--path", choices=["auto", "pipelined", "register"], default="auto",
                     help="kernel family (auto = pipelined wherever it applies)")
     ap.add_argument("--tokens", type=int, default=0,
@@ -425,7 +480,12 @@ def main(argv=None):
     if ws != args.gpus and not (ws == 1 and args.gpus == 1):
         if args.gpus > 1 and ws == 1:
             ap.error(f"--gpus {args.gpus} needs torchrun with {args.gpus} processes")
-    line = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if args.impl == "reference":
+        line = run_reference(args)
+    elif args.op == "logits":
+        line = run_logits(args)
+    else:
+        line = run_ours(args)
     if line is not None:
         print(json.dumps(line), flush=True)
 

@@ -5,8 +5,10 @@
 //
 // a GEMM [T x nd] x [nd x P] with a per-row RMS scale. Each CTA owns a tile of
 // `rows` tokens (<= 128; chosen so every SM gets one tile) and the whole K:
-//   warp 0      TMA producer: 128B-swizzled tiles of H (rows x 64) and W
-//               (Npad x 64) per k-step into a ring of shared-memory stages;
+//   warp 0      TMA producer: per k-step of 256, four adjacent 128B-swizzled
+//               sub-tiles of H (rows x 64) and of W (Npad x 64), so each
+//               token row is fetched 512 contiguous bytes at a time, into a
+//               ring of shared-memory stages;
 //   warp 1      allocates TMEM; one lane issues tcgen05.mma (M = 128, N = Npad,
 //               K = 16 per instruction, bf16 x bf16 -> fp32 in TMEM) and
 //               commits each stage back to the producer;
@@ -26,9 +28,11 @@ namespace hc {
 namespace {
 
 constexpr int kLgThreads = 192;
-constexpr int kLgKStep = 64;  // bf16 elements per k-step (one 128-byte swizzle row)
+constexpr int kLgKSub = 64;   // bf16 elements per sub-tile (one 128-byte swizzle row)
+constexpr int kLgSubs = 4;    // sub-tiles per stage: 512 contiguous bytes of each row
+constexpr int kLgKStep = kLgKSub * kLgSubs;
 constexpr int kLgM = 128;     // MMA rows (TMEM lanes)
-constexpr int kLgMaxStages = 8;
+constexpr int kLgMaxStages = 6;
 
 struct LogitsParams {
     float *z;
@@ -37,6 +41,7 @@ struct LogitsParams {
     int P;           // logits per token
     int Npad;        // P rounded up to 16 (MMA N)
     int rows;        // tokens per CTA tile (<= 128, multiple of 8)
+    int a_bytes;     // A region of a stage: kLgSubs sub-tiles of rows x 128 B + MMA read pad
     int nk;          // k-steps
     int stages;
     uint32_t tmem_cols;
@@ -50,8 +55,10 @@ hc_logits_kernel(const __grid_constant__ CUtensorMap mapH, const __grid_constant
     // 1024-byte aligned base for the swizzle atoms
     unsigned char *smem = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int a_bytes = kLgM * 128;
-    const int stage_bytes = a_bytes + p.Npad * 128;
+    const int a_bytes = p.a_bytes;
+    const int a_sub = p.rows * 128;   // bytes of one A sub-tile (1024-aligned: rows % 8 == 0)
+    const int b_sub = p.Npad * 128;
+    const int stage_bytes = a_bytes + kLgSubs * b_sub;
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + (size_t)p.stages * stage_bytes);
     uint64_t *empty = full + p.stages;
     uint64_t *accum = empty + p.stages;
@@ -88,7 +95,7 @@ hc_logits_kernel(const __grid_constant__ CUtensorMap mapH, const __grid_constant
     if (warp == 0) {
         // ---------------- producer ----------------
         if (lane == 0) {
-            const uint32_t tx = (uint32_t)(p.rows * 128 + p.Npad * 128);
+            const uint32_t tx = (uint32_t)(kLgSubs * (a_sub + b_sub));
             int s = 0;
             uint32_t ph = 0;
             int ks = 0;
@@ -97,8 +104,12 @@ hc_logits_kernel(const __grid_constant__ CUtensorMap mapH, const __grid_constant
                     break;
                 unsigned char *st = smem + (size_t)s * stage_bytes;
                 mbar_arrive_expect_tx(&full[s], tx);
-                tma_load_2d(st, &mapH, ks * kLgKStep, (int32_t)row0, &full[s]);
-                tma_load_2d(st + a_bytes, &mapW, ks * kLgKStep, 0, &full[s]);
+#pragma unroll
+                for (int c = 0; c < kLgSubs; ++c)
+                    tma_load_2d(st + c * a_sub, &mapH, ks * kLgKStep + c * kLgKSub, (int32_t)row0, &full[s]);
+#pragma unroll
+                for (int c = 0; c < kLgSubs; ++c)
+                    tma_load_2d(st + a_bytes + c * b_sub, &mapW, ks * kLgKStep + c * kLgKSub, 0, &full[s]);
                 if (++s == S) {
                     s = 0;
                     ph ^= 1u;
@@ -122,10 +133,14 @@ hc_logits_kernel(const __grid_constant__ CUtensorMap mapH, const __grid_constant
                 const uint32_t a0 = smem_addr(smem + (size_t)s * stage_bytes);
                 const uint32_t b0 = a0 + (uint32_t)a_bytes;
 #pragma unroll
-                for (int kk = 0; kk < kLgKStep / 16; ++kk) {
-                    // +32 bytes along K per 16-element MMA step inside the swizzle atom
-                    umma_bf16(tmem_d, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32),
-                              idesc, (ks | kk) != 0);
+                for (int c = 0; c < kLgSubs; ++c) {
+#pragma unroll
+                    for (int kk = 0; kk < kLgKSub / 16; ++kk) {
+                        // +32 bytes along K per 16-element MMA step inside the swizzle atom
+                        umma_bf16(tmem_d, umma_desc_sw128(a0 + c * a_sub + kk * 32),
+                                  umma_desc_sw128(b0 + c * b_sub + kk * 32), idesc,
+                                  (ks | c | kk) != 0);
+                    }
                 }
                 umma_commit(&empty[s]);  // stage free once these MMAs have read it
                 if (++s == S) {
@@ -161,25 +176,29 @@ hc_logits_kernel(const __grid_constant__ CUtensorMap mapH, const __grid_constant
                 break;
             }
             if (live) {
-                // the row's 128 bytes (64 bf16) sit in one 128-byte line, the
-                // 16-byte chunks permuted by the swizzle: order is irrelevant here
-                const uint4 *row = reinterpret_cast<const uint4 *>(smem + (size_t)s * stage_bytes +
-                                                                   (size_t)r * 128);
-                float2 acc = make_float2(0.0f, 0.0f);
+                // In each sub-tile the row's 128 bytes (64 bf16) fill one
+                // 128-byte line, its 16-byte chunks permuted by the swizzle;
+                // the sum takes them in any order. Starting each row at
+                // physical chunk (row & 7) keeps the eight rows a quarter-warp
+                // reads on distinct banks.
+                const unsigned char *rowp = smem + (size_t)s * stage_bytes + (size_t)r * 128;
+                const int rot = r & 7;
+                float2 acc0 = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint4 q = row[c];
+                for (int c = 0; c < 8 * kLgSubs; ++c) {
+                    const uint4 q = *reinterpret_cast<const uint4 *>(
+                        rowp + (size_t)(c >> 3) * a_sub + (size_t)(((c & 7) ^ rot) * 16));
                     float2 v;
                     widen_bf16x2(q.x, v.x, v.y);
-                    acc = ffma2_rn(v, v, acc);
+                    acc0 = ffma2_rn(v, v, acc0);
                     widen_bf16x2(q.y, v.x, v.y);
-                    acc = ffma2_rn(v, v, acc);
+                    acc1 = ffma2_rn(v, v, acc1);
                     widen_bf16x2(q.z, v.x, v.y);
-                    acc = ffma2_rn(v, v, acc);
+                    acc0 = ffma2_rn(v, v, acc0);
                     widen_bf16x2(q.w, v.x, v.y);
-                    acc = ffma2_rn(v, v, acc);
+                    acc1 = ffma2_rn(v, v, acc1);
                 }
-                ss += (double)acc.x + (double)acc.y;
+                ss += ((double)acc0.x + (double)acc0.y) + ((double)acc1.x + (double)acc1.y);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
@@ -266,7 +285,11 @@ hc_status launch_mix_logits(const void *H, const void *W, float *z, int64_t T, i
     uint32_t cols = 32;
     while (cols < (uint32_t)lp.Npad) cols <<= 1;
     lp.tmem_cols = cols;
-    const int stage_bytes = kLgM * 128 + lp.Npad * 128;
+    // the M = 128 MMA reads 128 rows from each sub-tile base: pad the A region
+    // so the last sub-tile's read stays inside the stage (rows beyond `rows`
+    // feed TMEM lanes the epilogue ignores)
+    lp.a_bytes = kLgSubs * lp.rows * 128 + (kLgM - lp.rows) * 128;
+    const int stage_bytes = lp.a_bytes + kLgSubs * lp.Npad * 128;
     const int fixed = 1024 /* alignment slack */ + 2 * kLgMaxStages * 8 + 16 + 16;
     int stages = (kSmemLimitLogits - fixed) / stage_bytes;
     if (stages > kLgMaxStages) stages = kLgMaxStages;
@@ -275,9 +298,9 @@ hc_status launch_mix_logits(const void *H, const void *W, float *z, int64_t T, i
     const int smem = fixed + stages * stage_bytes;
 
     CUtensorMap mapH, mapW;
-    hc_status ms = make_map(&mapH, H, (uint64_t)lp.K, (uint64_t)T, kLgKStep, (uint32_t)lp.rows);
+    hc_status ms = make_map(&mapH, H, (uint64_t)lp.K, (uint64_t)T, kLgKSub, (uint32_t)lp.rows);
     if (ms != HC_OK) return ms;
-    ms = make_map(&mapW, W, (uint64_t)lp.K, (uint64_t)P, kLgKStep, (uint32_t)lp.Npad);
+    ms = make_map(&mapW, W, (uint64_t)lp.K, (uint64_t)P, kLgKSub, (uint32_t)lp.Npad);
     if (ms != HC_OK) return ms;
 
     static int configured[64] = {};
