@@ -222,6 +222,71 @@ def run_logits(args):
     }
 
 
+def run_ends(args):
+    """The stack ends on the workload's shape (T=16384, n=4, d=7168, bf16):
+    --op expand_read times hc_expand_then_read (one row in -> four copies and
+    layer 0's RMS-normalised block input out); --op collapse times hc_collapse
+    (four streams in -> one weighted row out). Kernel-only, device-timed, one
+    launch per step; outputs ping-pong so consecutive launches do not share
+    buffers in L2."""
+    import numpy as np
+    import torch
+    import hc_inputs as gen
+    from hyper_connections_stream_b200 import _lib as hc
+    ws, rank, local = _dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = dict(WORKLOAD)
+    if args.tokens:
+        w["T"] = args.tokens
+    T, n, d = w["T"], w["n"], w["d"]
+    s = 2
+    g = torch.from_numpy(gen.uniform(3500 + w["cfg"], (d,), 0.5, 1.5)).to(device)
+    a = torch.full((n,), 1.0 / n, device=device)
+    if args.op == "expand_read":
+        xs = [gen.device_normal(gen.SEED_Y + w["cfg"] + i, (T, d), torch.bfloat16, device) for i in range(2)]
+        Hs = [torch.empty((T, n, d), dtype=torch.bfloat16, device=device) for _ in range(2)]
+        xr = [torch.empty((T, d), dtype=torch.bfloat16, device=device) for _ in range(2)]
+        def launch(i):
+            hc.expand_then_read(xs[i % 2], n, a, g, eps=w["eps"], out=Hs[i % 2], x_read=xr[i % 2])
+        alg_bytes = T * d * s * (n + 2) + d * 4
+        what = "expand + layer-0 read (hc_expand_then_read)"
+    else:
+        Hs = [gen.device_normal(gen.SEED_H + w["cfg"] + i, (T, n, d), torch.bfloat16, device) for i in range(2)]
+        outs = [torch.empty((T, d), dtype=torch.bfloat16, device=device) for _ in range(2)]
+        def launch(i):
+            hc.collapse(Hs[i % 2], a, out=outs[i % 2])
+        alg_bytes = T * d * s * (n + 1)
+        what = "collapse (hc_collapse)"
+    stream = torch.cuda.current_stream(device)
+    for i in range(args.warmup):
+        launch(i)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        launch(i)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    kern_ms = statistics.mean(s_.elapsed_time(e) for s_, e in ev)
+    total_ms = ev[0][0].elapsed_time(ev[-1][1])
+    peak, peak_kind = _peaks()
+    achieved = alg_bytes / (kern_ms / 1e3) / 1e9
+    return {
+        "metric": f"stack-end tokens/sec at n=4, d=7168 (bf16): {what}",
+        "value": T * args.steps / (total_ms / 1e3), "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.op, "T": T, "n": n, "d": d, "l2": "inputs and outputs > L2"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "peak_source": peak_kind,
+                     "algorithmic_bytes_per_launch": alg_bytes, "kernel_ms": kern_ms},
+        "gpu_launches": args.steps, "device_fault": hc.device_fault(),
+    }
+
+
 def run_ours(args):
     import torch
     from hyper_connections_stream_b200 import _lib as hc
@@ -466,9 +531,10 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-only", action="store_true",
                     help="device-timed kernel only (no e2e, no CPU baseline): for profiling")
-    ap.add_argument("--op", choices=["step", "logits"], default="step",
+    ap.add_argument("--op", choices=["step", "logits", "expand_read", "collapse"], default="step",
                     help="step: the fused HC step (the metric); logits: the tensor-core "
-                         "mixing-logits kernel on the same streams")
+                         "mixing-logits kernel on the same streams; expand_read / collapse: "
+                         "the stack ends on the same shape")
     ap.add_argument("--path", choices=["auto", "pipelined", "register"], default="auto",
                     help="kernel family (auto = pipelined wherever it applies)")
     ap.add_argument("--tokens", type=int, default=0,
@@ -484,6 +550,8 @@ def main(argv=None):
         line = run_reference(args)
     elif args.op == "logits":
         line = run_logits(args)
+    elif args.op in ("expand_read", "collapse"):
+        line = run_ends(args)
     else:
         line = run_ours(args)
     if line is not None:

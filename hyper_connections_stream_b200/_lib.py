@@ -39,6 +39,10 @@ SIGNATURES = {
     "hc_device_fault": ([C.POINTER(_i32), _vp], _i32),
     "hc_selftest_bounded_wait": ([_i32, _vp], _i32),
     "hc_mix_logits": ([_vp, _vp, _vp, _i32, _i64, _i32, _i64, _i32, _f32, _vp], _i32),
+    "hc_expand": ([_vp, _vp, _i32, _i64, _i32, _i64, _vp], _i32),
+    "hc_expand_then_read": ([_vp, _vp, _vp, _i32, _i64, _i32, _i64, _i32, _vp, _i64, _vp, _f32,
+                             _vp], _i32),
+    "hc_collapse": ([_vp, _vp, _i32, _i64, _i32, _i64, _i32, _vp, _i64, _vp], _i32),
     "hc_status_string": ([_i32], C.c_char_p),
     "hc_last_error": ([], C.c_char_p),
     "hc_version": ([], _i32),
@@ -97,6 +101,21 @@ def _need_cuda(name, t, dtype=None):
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _need_out(name, t, shape, dtype):
+    """An output tensor: CUDA, contiguous, of exactly this shape and dtype (the
+    library writes shape-many elements through the raw pointer)."""
+    _need_cuda(name, t, dtype)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must be {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _need_gain(name, g, d):
+    if g is not None:
+        _need_cuda(name, g, torch.float32)
+        if tuple(g.shape) != (d,):
+            raise ValueError(f"{name} must be [d]")
 
 
 def _tok_param(name, p, T, per_shape):
@@ -161,7 +180,7 @@ def mix_logits(H, W, *, eps: float = 1e-6, out=None):
         raise ValueError(f"W must be [P, n*d = {n * d}], got {tuple(W.shape)}")
     P = W.shape[0]
     out = torch.empty((T, P), dtype=torch.float32, device=H.device) if out is None else out
-    _need_cuda("out", out, torch.float32)
+    _need_out("out", out, (T, P), torch.float32)
     _check(lib().hc_mix_logits(_ptr(H), _ptr(W), _ptr(out), HC_BF16, T, n, d, P, float(eps),
                                _stream(H.device)))
     return out
@@ -181,7 +200,7 @@ def sinkhorn(logits: torch.Tensor, K: int, out: torch.Tensor | None = None) -> t
         raise ValueError("logits must be [..., n, n]")
     T = logits.numel() // (n * n) if n else 0
     out = torch.empty_like(logits) if out is None else out
-    _need_cuda("out", out, torch.float32)
+    _need_out("out", out, tuple(logits.shape), torch.float32)
     _check(lib().hc_sinkhorn(_ptr(logits), _ptr(out), T, n, int(K), _stream(logits.device)))
     return out
 
@@ -197,7 +216,7 @@ def read_rmsnorm(H, a, g=None, *, eps: float = 1e-6, read: int = READ_WEIGHTS, x
         if tuple(g.shape) != (d,):
             raise ValueError("g must be [d]")
     x = torch.empty((T, d), dtype=H.dtype, device=H.device) if x is None else x
-    _need_cuda("x", x, H.dtype)
+    _need_out("x", x, (T, d), H.dtype)
     _check(lib().hc_read_rmsnorm(_ptr(H), _ptr(x), _DT[H.dtype], T, n, d, int(read), _ptr(a),
                                  a_s, _ptr(g), float(eps), _stream(H.device)))
     return x
@@ -215,7 +234,7 @@ def write_mix(H, y, A, b, *, mix: int = MIX_MATRIX, K: int = 0, out=None):
     A_s = _tok_param("A", A, T, (n, n))
     b_s = _tok_param("b", b, T, (n,))
     out = torch.empty_like(H) if out is None else out
-    _need_cuda("out", out, H.dtype)
+    _need_out("out", out, (T, n, d), H.dtype)
     _check(lib().hc_write_mix(_ptr(H), _ptr(y), _ptr(out), _DT[H.dtype], T, n, d, int(mix),
                               _ptr(A), A_s, int(K), _ptr(b), b_s, _stream(H.device)))
     return out
@@ -240,10 +259,55 @@ def write_then_read(H, y, A, b, a_next, g_next=None, *, eps: float = 1e-6,
             raise ValueError("g_next must be [d]")
     out = torch.empty_like(H) if out is None else out
     x_next = torch.empty((T, d), dtype=H.dtype, device=H.device) if x_next is None else x_next
-    _need_cuda("out", out, H.dtype)
-    _need_cuda("x_next", x_next, H.dtype)
+    _need_out("out", out, (T, n, d), H.dtype)
+    _need_out("x_next", x_next, (T, d), H.dtype)
     _check(lib().hc_write_then_read(_ptr(H), _ptr(y), _ptr(out), _ptr(x_next), _DT[H.dtype],
                                     T, n, d, int(mix), _ptr(A), A_s, int(K), _ptr(b), b_s,
                                     int(read), _ptr(a_next), a_s, _ptr(g_next), float(eps),
                                     _stream(H.device)))
     return out, x_next
+
+
+def expand(x, n: int, *, out=None):
+    """Stack entry: H[t, i, :] = x[t, :] for the n streams. x [T, d] -> H [T, n, d]."""
+    _need_cuda("x", x)
+    if x.dim() != 2 or x.dtype not in _DT:
+        raise ValueError("x must be [T, d] float32 or bfloat16")
+    T, d = x.shape
+    out = torch.empty((T, n, d), dtype=x.dtype, device=x.device) if out is None else out
+    _need_out("out", out, (T, n, d), x.dtype)
+    _check(lib().hc_expand(_ptr(x), _ptr(out), _DT[x.dtype], T, int(n), d, _stream(x.device)))
+    return out
+
+
+def expand_then_read(x, n: int, a, g=None, *, eps: float = 1e-6, read: int = READ_WEIGHTS,
+                     out=None, x_read=None):
+    """Stack entry fused with layer 0's read: H = n copies of x, and
+    x_read = RMSNorm(sum_i a_i x) * g. Returns (H, x_read); x_read may be x."""
+    _need_cuda("x", x)
+    if x.dim() != 2 or x.dtype not in _DT:
+        raise ValueError("x must be [T, d] float32 or bfloat16")
+    T, d = x.shape
+    a_s = _tok_param("a", a, T, (int(n),))
+    _need_gain("g", g, d)
+    out = torch.empty((T, n, d), dtype=x.dtype, device=x.device) if out is None else out
+    x_read = torch.empty_like(x) if x_read is None else x_read
+    _need_out("out", out, (T, n, d), x.dtype)
+    _need_out("x_read", x_read, (T, d), x.dtype)
+    _check(lib().hc_expand_then_read(_ptr(x), _ptr(out), _ptr(x_read), _DT[x.dtype], T, int(n), d,
+                                     int(read), _ptr(a), a_s, _ptr(g), float(eps),
+                                     _stream(x.device)))
+    return out, x_read
+
+
+def collapse(H, w, *, read: int = READ_WEIGHTS, out=None):
+    """Stack exit: out = sum_i w_i H_i (no normalisation). w [n] or [T, n]
+    (weights or, with read=READ_SOFTMAX_LOGITS, logits)."""
+    _need_cuda("H", H)
+    T, n, d = _streams_shape(H)
+    w_s = _tok_param("w", w, T, (n,))
+    out = torch.empty((T, d), dtype=H.dtype, device=H.device) if out is None else out
+    _need_out("out", out, (T, d), H.dtype)
+    _check(lib().hc_collapse(_ptr(H), _ptr(out), _DT[H.dtype], T, n, d, int(read), _ptr(w), w_s,
+                             _stream(H.device)))
+    return out

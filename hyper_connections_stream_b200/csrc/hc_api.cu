@@ -353,4 +353,72 @@ hc_status hc_write_then_read(const void *H, const void *y, void *Hout, void *x_n
     return dispatch<hc::KIND_FUSED>(dt, n, p, static_cast<cudaStream_t>(stream));
 }
 
+hc_status hc_expand(const void *x, void *H, hc_dtype dt, int64_t T, int n, int64_t d,
+                    hc_stream stream) {
+    static const char *fn = "hc_expand";
+    g_last_error[0] = '\0';
+    const Shape s{dt, T, n, d};
+    HC_TRY(check_shape(fn, s, false));
+    if (T == 0) return HC_OK;
+    HC_TRY(check_buf(fn, "x", x));
+    HC_TRY(check_buf(fn, "H", H));
+    const int64_t es = elem_bytes(dt);
+    if (overlap(H, T * n * d * es, x, T * d * es)) return fail(HC_ERR_ALIAS, "%s: H overlaps x", fn);
+    hc::StepParams p{};
+    p.y = x; p.Hout = H; p.T = T; p.d = d;
+    return dispatch<hc::KIND_EXPAND>(dt, n, p, static_cast<cudaStream_t>(stream));
+}
+
+hc_status hc_expand_then_read(const void *x, void *H, void *x_read, hc_dtype dt, int64_t T, int n,
+                              int64_t d, hc_read_mode rm, const float *a, int64_t a_tok_stride,
+                              const float *g, float eps, hc_stream stream) {
+    static const char *fn = "hc_expand_then_read";
+    g_last_error[0] = '\0';
+    const Shape s{dt, T, n, d};
+    HC_TRY(check_shape(fn, s, true));
+    if (rm != HC_READ_WEIGHTS && rm != HC_READ_SOFTMAX_LOGITS)
+        return fail(HC_ERR_INVALID_ARG, "%s: bad read mode %d", fn, (int)rm);
+    HC_TRY(check_stride(fn, "a_tok_stride", a_tok_stride));
+    HC_TRY(check_eps(fn, eps));
+    if (T == 0) return HC_OK;
+    HC_TRY(check_buf(fn, "x", x));
+    HC_TRY(check_buf(fn, "H", H));
+    HC_TRY(check_buf(fn, "x_read", x_read));
+    HC_TRY(check_param(fn, "a", a));
+    if (g && !aligned(g, 16)) return fail(HC_ERR_MISALIGNED, "%s: g is not 16-byte aligned", fn);
+    const int64_t es = elem_bytes(dt);
+    const int64_t hb = T * n * d * es, xb = T * d * es;
+    if (overlap(H, hb, x, xb)) return fail(HC_ERR_ALIAS, "%s: H overlaps x", fn);
+    if (overlap(x_read, xb, H, hb)) return fail(HC_ERR_ALIAS, "%s: x_read overlaps H", fn);
+    if (x_read != x && overlap(x_read, xb, x, xb))
+        return fail(HC_ERR_ALIAS, "%s: x_read partially overlaps x", fn);
+    hc::StepParams p{};
+    p.y = x; p.Hout = H; p.x = x_read; p.T = T; p.d = d;
+    p.a = a; p.a_s = a_tok_stride; p.g = g; p.eps = eps;
+    p.read_logits = rm == HC_READ_SOFTMAX_LOGITS;
+    return dispatch<hc::KIND_EXPAND_READ>(dt, n, p, static_cast<cudaStream_t>(stream));
+}
+
+hc_status hc_collapse(const void *H, void *out, hc_dtype dt, int64_t T, int n, int64_t d,
+                      hc_read_mode rm, const float *w, int64_t w_tok_stride, hc_stream stream) {
+    static const char *fn = "hc_collapse";
+    g_last_error[0] = '\0';
+    const Shape s{dt, T, n, d};
+    HC_TRY(check_shape(fn, s, false));
+    if (rm != HC_READ_WEIGHTS && rm != HC_READ_SOFTMAX_LOGITS)
+        return fail(HC_ERR_INVALID_ARG, "%s: bad read mode %d", fn, (int)rm);
+    HC_TRY(check_stride(fn, "w_tok_stride", w_tok_stride));
+    if (T == 0) return HC_OK;
+    HC_TRY(check_buf(fn, "H", H));
+    HC_TRY(check_buf(fn, "out", out));
+    HC_TRY(check_param(fn, "w", w));
+    const int64_t es = elem_bytes(dt);
+    if (overlap(out, T * d * es, H, T * n * d * es)) return fail(HC_ERR_ALIAS, "%s: out overlaps H", fn);
+    hc::StepParams p{};
+    p.H = H; p.x = out; p.T = T; p.d = d;
+    p.a = w; p.a_s = w_tok_stride;
+    p.read_logits = rm == HC_READ_SOFTMAX_LOGITS;
+    return dispatch<hc::KIND_COLLAPSE>(dt, n, p, static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

@@ -15,8 +15,23 @@ constexpr int kMaxStreams = 8;
 // bounds d of a normalising call at 512 * 8 vectors.
 constexpr int kStreamMaxThreads = 512;
 
-// Step kinds: read + RMSNorm, write mix, fused write then read.
-enum Kind { KIND_READ = 0, KIND_WRITE = 1, KIND_FUSED = 2 };
+// Step kinds. READ / WRITE / FUSED are the residual step; the last three are
+// the ends of a stack: EXPAND copies one row into the n streams, EXPAND_READ
+// also produces layer 0's block input from them, COLLAPSE mixes the n
+// streams into one row (no normalisation).
+enum Kind {
+    KIND_READ = 0,
+    KIND_WRITE = 1,
+    KIND_FUSED = 2,
+    KIND_EXPAND = 3,
+    KIND_EXPAND_READ = 4,
+    KIND_COLLAPSE = 5
+};
+
+// Kinds that normalise a mixed row (a CTA-wide statistic per token).
+__host__ __device__ constexpr bool kind_normalises(int kind) {
+    return kind == KIND_READ || kind == KIND_FUSED || kind == KIND_EXPAND_READ;
+}
 
 // ---------------------------------------------------------------------------
 // Storage dtype traits: one 16-byte vector = V elements.

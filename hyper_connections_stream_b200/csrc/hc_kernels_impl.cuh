@@ -65,9 +65,9 @@ template <int N, typename S, int KIND>
 hc_status launch_stream(const StepParams &p, const LaunchCtx &ctx, cudaStream_t st) {
     constexpr int V = StorageTraits<S>::V;
     int NT = 0, CPT = 1;
-    pick_stream_shape(p.d / V, KIND != KIND_WRITE, NT, CPT);
+    pick_stream_shape(p.d / V, kind_normalises(KIND), NT, CPT);
     if (NT == 0) return set_error(HC_ERR_UNSUPPORTED, "no launch shape for d = %lld", (long long)p.d);
-    if constexpr (KIND == KIND_WRITE) {
+    if constexpr (!kind_normalises(KIND)) {
         return launch_stream_cpt<N, S, KIND, 1>(p, NT, ctx, st);
     } else {
         switch (CPT) {
@@ -129,7 +129,7 @@ hc_status launch_pipe(const StepParams &p, const PipeShape &sh, int smem, const 
 }
 
 template <int N, typename S, int KIND>
-hc_status launch_n(const StepParams &p, const LaunchCtx &ctx, cudaStream_t st) {
+hc_status launch_step_n(const StepParams &p, const LaunchCtx &ctx, cudaStream_t st) {
     PipeShape sh{};
     int smem = 0;
     const bool pipe_ok = pipe_shape<N, S, KIND>(p, sh, smem);
@@ -142,11 +142,23 @@ hc_status launch_n(const StepParams &p, const LaunchCtx &ctx, cudaStream_t st) {
     // d = 4096 at ~1000; n = 8 at ~600).
     const bool small = p.T * (int64_t)N * p.d * (int64_t)sizeof(S) * 2 < (int64_t(64) << 20);
     if (ctx.path == 2 || !pipe_ok || (ctx.path == 0 && small)) {
-        if (KIND != KIND_WRITE && p.d > (int64_t)kStreamMaxThreads * 8 * StorageTraits<S>::V)
+        if (kind_normalises(KIND) && p.d > (int64_t)kStreamMaxThreads * 8 * StorageTraits<S>::V)
             return set_error(HC_ERR_UNSUPPORTED, "d = %lld too large", (long long)p.d);
         return launch_stream<N, S, KIND>(p, ctx, st);
     }
     return launch_pipe<N, S, KIND>(p, sh, smem, ctx, st);
+}
+
+template <int N, typename S, int KIND>
+hc_status launch_n(const StepParams &p, const LaunchCtx &ctx, cudaStream_t st) {
+    if constexpr (KIND >= KIND_EXPAND) {
+        // the ends of a stack run once per pass: register-streaming family only
+        if (kind_normalises(KIND) && p.d > (int64_t)kStreamMaxThreads * 8 * StorageTraits<S>::V)
+            return set_error(HC_ERR_UNSUPPORTED, "d = %lld too large", (long long)p.d);
+        return launch_stream<N, S, KIND>(p, ctx, st);
+    } else {
+        return launch_step_n<N, S, KIND>(p, ctx, st);
+    }
 }
 
 template <typename S, int KIND>

@@ -10,6 +10,9 @@
 // KIND_WRITE:  H, y -> H'                    (no reduction, no barrier per token)
 // KIND_READ:   H -> x = RMSNorm(a^T H) g
 // KIND_FUSED:  H, y -> H', x = RMSNorm(a^T H') g (H' not read back)
+// KIND_EXPAND:      e -> H' with every stream a copy of e (p.y holds e)
+// KIND_EXPAND_READ: e -> H' as above, x = RMSNorm(a^T H') g (H' not read back)
+// KIND_COLLAPSE:    H -> x = a^T H, stored without normalisation
 // For the normalising kinds a thread keeps its slice of h in registers until
 // the CTA-wide fp64 sum of squares is known (warp shuffles, then one
 // shared-memory exchange per token), so each byte crosses HBM once.
@@ -27,8 +30,8 @@ __global__ void __launch_bounds__(kStreamMaxThreads)
 hc_stream_kernel(StepParams p) {
     constexpr int V = StorageTraits<S>::V;
     constexpr int NN = N * N;
-    constexpr bool WRITE = KIND != KIND_READ;
-    constexpr bool READ = KIND != KIND_WRITE;
+    constexpr bool WRITE = KIND == KIND_WRITE || KIND == KIND_FUSED;  // A, b per token
+    constexpr bool READ = KIND != KIND_WRITE && KIND != KIND_EXPAND;  // a per token
     constexpr int TB_MAX = kPrepTokens;
 
     __shared__ float sA[TB_MAX * NN > 0 ? TB_MAX * NN : 1];
@@ -66,7 +69,32 @@ hc_stream_kernel(StepParams p) {
             const S *Ht = H + t * N * p.d;
             S *Hot = Ho + t * N * p.d;
 
-            if constexpr (KIND == KIND_WRITE) {
+            if constexpr (KIND == KIND_EXPAND) {
+                for (int64_t c = tid; c < nvec; c += NT) {
+                    const int64_t k = c * V;
+                    float e[V];
+                    load_vec_cs(Y + t * p.d + k, e);
+#pragma unroll
+                    for (int j = 0; j < N; ++j) store_vec_cs(Hot + j * p.d + k, e);
+                }
+            } else if constexpr (KIND == KIND_COLLAPSE) {
+                S *Xt = X + t * p.d;
+                for (int64_t c = tid; c < nvec; c += NT) {
+                    const int64_t k = c * V;
+                    float h[N][V], acc[V];
+#pragma unroll
+                    for (int i = 0; i < N; ++i) load_vec_cs(Ht + i * p.d + k, h[i]);
+#pragma unroll
+                    for (int e = 0; e < V; ++e) acc[e] = -0.0f;
+#pragma unroll
+                    for (int i = 0; i < N; ++i) {
+                        const float ai = sa[tt * N + i];
+#pragma unroll
+                        for (int e = 0; e < V; ++e) acc[e] = __fmaf_rn(ai, h[i][e], acc[e]);
+                    }
+                    store_vec_cs(Xt + k, acc);
+                }
+            } else if constexpr (KIND == KIND_WRITE) {
                 for (int64_t c = tid; c < nvec; c += NT) {
                     const int64_t k = c * V;
                     float h[N][V], yv[V];
@@ -99,12 +127,23 @@ hc_stream_kernel(StepParams p) {
                     const int64_t c = tid + (int64_t)u * NT;
                     if (c < nvec) {
                         const int64_t k = c * V;
-                        float h[N][V];
-#pragma unroll
-                        for (int i = 0; i < N; ++i) load_vec_cs(Ht + i * p.d + k, h[i]);
 #pragma unroll
                         for (int e = 0; e < V; ++e) hs[u][e] = -0.0f;
-                        if constexpr (KIND == KIND_FUSED) {
+                        if constexpr (KIND == KIND_EXPAND_READ) {
+                            // every stream holds e: store the n copies, mix e
+                            float ev[V];
+                            load_vec_cs(Y + t * p.d + k, ev);
+#pragma unroll
+                            for (int j = 0; j < N; ++j) {
+                                store_vec_cs(Hot + j * p.d + k, ev);
+                                const float aj = sa[tt * N + j];
+#pragma unroll
+                                for (int e = 0; e < V; ++e) hs[u][e] = __fmaf_rn(aj, ev[e], hs[u][e]);
+                            }
+                        } else if constexpr (KIND == KIND_FUSED) {
+                            float h[N][V];
+#pragma unroll
+                            for (int i = 0; i < N; ++i) load_vec_cs(Ht + i * p.d + k, h[i]);
                             float yv[V];
                             load_vec_cs(Y + t * p.d + k, yv);
 #pragma unroll
@@ -127,6 +166,9 @@ hc_stream_kernel(StepParams p) {
                                 for (int e = 0; e < V; ++e) hs[u][e] = __fmaf_rn(aj, stored[e], hs[u][e]);
                             }
                         } else {
+                            float h[N][V];
+#pragma unroll
+                            for (int i = 0; i < N; ++i) load_vec_cs(Ht + i * p.d + k, h[i]);
 #pragma unroll
                             for (int i = 0; i < N; ++i) {
                                 const float ai = sa[tt * N + i];

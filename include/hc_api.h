@@ -140,6 +140,39 @@ HC_API hc_status hc_write_then_read(const void *H, const void *y, void *Hout, vo
                              hc_stream stream);
 
 /*
+ * Ends of a stack ("Tencent open-sources Hy4 Preview at 770B -- Identity
+ * Hyper-Connections", learnaivisually: TL;DR and the residual-design table --
+ * the n streams start as copies of one; the pages do not say how they are
+ * combined at the top, read here as a learned weighted sum of the streams).
+ *
+ * hc_expand: H[t][i][:] = x[t][:] for every stream i (a bit copy).
+ *   x [T][d] in, H [T][n][d] out, dtype dt, both 16-byte aligned, no overlap.
+ *
+ * hc_expand_then_read: hc_expand fused with layer 0's read + pre-norm
+ *   RMSNorm of the copies (arguments as hc_read_rmsnorm), so H is not read
+ *   back: x_read = RMSNorm(sum_i a_i x) * g, the mix an fp32 fused
+ *   multiply-add chain in stream order. x_read may equal x exactly (in place);
+ *   H must not overlap x or x_read.
+ *
+ * hc_collapse: out[t][:] = sum_i w_i H[t][i][:], an fp32 fused multiply-add
+ *   chain in stream order stored in dtype dt, no normalisation (a final norm
+ *   before the head is hc_read_rmsnorm). rm == HC_READ_SOFTMAX_LOGITS turns w
+ *   into weights with a softmax over the n streams first. w_tok_stride: 0 =
+ *   one set for all tokens, else floats per token. out must not overlap H.
+ *
+ * Same shape limits and error statuses as the step calls; T == 0 is a no-op.
+ */
+HC_API hc_status hc_expand(const void *x, void *H, hc_dtype dt, int64_t T, int n, int64_t d,
+                           hc_stream stream);
+HC_API hc_status hc_expand_then_read(const void *x, void *H, void *x_read, hc_dtype dt, int64_t T,
+                                     int n, int64_t d, hc_read_mode rm, const float *a,
+                                     int64_t a_tok_stride, const float *g, float eps,
+                                     hc_stream stream);
+HC_API hc_status hc_collapse(const void *H, void *out, hc_dtype dt, int64_t T, int n, int64_t d,
+                             hc_read_mode rm, const float *w, int64_t w_tok_stride,
+                             hc_stream stream);
+
+/*
  * Kernel family used by the step calls (process-wide; default HC_PATH_AUTO).
  *   HC_PATH_PIPELINED: warp-specialised kernels fed by bulk copies (TMA) into
  *     shared-memory rings; the automatic choice for calls that move 64 MiB

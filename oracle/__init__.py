@@ -42,6 +42,8 @@ def lib():
             "hco_block_tanh": ([vp, vp, i32, i64], i32),
             "hco_mix_logits": ([vp, vp, vp, i32, i64, i32, i64, i32, fp], i32),
             "hco_single_stream_layer": ([vp, vp, i32, i64, i64, vp, fp], i32),
+            "hco_expand": ([vp, vp, i32, i64, i32, i64], i32),
+            "hco_collapse": ([vp, vp, i32, i64, i32, i64, i32, vp, i64], i32),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -169,6 +171,35 @@ def mix_logits(H, W, eps: float, dt: str):
     z = np.empty((T, P), dtype=np.float64)
     _chk(lib().hco_mix_logits(_p(H), _p(W), _p(z), _DT[dt], T, n, d, P, float(eps)), "mix_logits")
     return z
+
+
+def expand(x, n: int, dt: str):
+    """Stack entry: H[t, i, :] = x[t, :] for i < n. x [T, d] -> H [T, n, d]."""
+    x = _arr(x, _NP[dt])
+    T, d = x.shape
+    H = np.empty((T, n, d), dtype=_NP[dt])
+    _chk(lib().hco_expand(_p(x), _p(H), _DT[dt], T, int(n), d), "expand")
+    return H
+
+
+def expand_then_read(x, n: int, a, g, eps: float, dt: str, read_logits: bool = False):
+    """Stack entry followed by layer 0's read: (expand(x), RMSNorm(sum_i a_i H_i) g)
+    of the expanded streams; with read_logits, a holds softmax logits."""
+    H = expand(x, n, dt)
+    w = softmax(a) if read_logits else a
+    return H, read_rmsnorm(H, w, g, eps, dt)
+
+
+def collapse(H, w, dt: str, read_logits: bool = False):
+    """Stack exit: out[t] = sum_i w_i H[t, i] (fmaf chain, stored in dt).
+    w: [n] or [T, n]; with read_logits, w holds softmax logits."""
+    H = _arr(H, _NP[dt])
+    T, n, d = H.shape
+    w = _arr(w, np.float32)
+    out = np.empty((T, d), dtype=_NP[dt])
+    _chk(lib().hco_collapse(_p(H), _p(out), _DT[dt], T, n, d, int(read_logits), _p(w),
+                            _tok_stride(w, T, n)), "collapse")
+    return out
 
 
 def block_tanh(x, dt: str):

@@ -355,6 +355,44 @@ int hco_mix_logits(const void *H, const void *W, double *z, int dt, int64_t T, i
     return HCO_OK;
 }
 
+/*
+ * Ends of a stack ("Tencent open-sources Hy4 Preview at 770B -- Identity
+ * Hyper-Connections", learnaivisually: TL;DR and the residual-design table,
+ * the n streams start as copies of one). Expansion: every stream of token t
+ * is a copy of x[t]. The pages do not say how the streams are combined at the
+ * top; reading: a weighted sum of the streams, out = sum_i w_i H_i, the same
+ * fmaf chain in stream order as the read mix, stored without normalisation.
+ */
+int hco_expand(const void *x, void *H, int dt, int64_t T, int n, int64_t d) {
+    if (check_common(dt, T, n, d)) return HCO_EINVAL;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t)
+        for (int i = 0; i < n; ++i)
+            for (int64_t k = 0; k < d; ++k)
+                store_s(H, dt, (t * n + i) * d + k, load_s(x, dt, t * d + k));
+    return HCO_OK;
+}
+
+int hco_collapse(const void *H, void *out, int dt, int64_t T, int n, int64_t d, int read_logits,
+                 const float *w, int64_t w_s) {
+    if (check_common(dt, T, n, d) || !w) return HCO_EINVAL;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        float ww[16];
+        const float *wt = tok_ptr(w, w_s, t);
+        if (read_logits) {
+            softmax_one_f32(wt, ww, n);
+            wt = ww;
+        }
+        for (int64_t k = 0; k < d; ++k) {
+            float acc = -0.0f;
+            for (int i = 0; i < n; ++i) acc = fmaf(wt[i], load_s(H, dt, (t * n + i) * d + k), acc);
+            store_s(out, dt, t * d + k, acc);
+        }
+    }
+    return HCO_OK;
+}
+
 /* Harness block stand-in: y = round_s(tanhf(x)). Not part of the HC step. */
 int hco_block_tanh(const void *x, void *y, int dt, int64_t count) {
     if (dt != HCO_F32 && dt != HCO_BF16) return HCO_EINVAL;

@@ -104,6 +104,22 @@ _CHILD = textwrap.dedent(r"""
     call("st_lo", "hc_selftest_bounded_wait", 0, None)
     call("st_hi", "hc_selftest_bounded_wait", 1000000, None)
     call("path_bad", "hc_set_path", 7)
+    xb = T * d * 2
+    call("ex_T0", "hc_expand", None, None, bf, 0, n, d, None)
+    call("ex_n9", "hc_expand", x, H, bf, T, 9, d, None)
+    call("ex_null", "hc_expand", None, H, bf, T, n, d, None)
+    call("ex_mis", "hc_expand", x + 8, H, bf, T, n, d, None)
+    call("ex_alias", "hc_expand", H + hb - 16, H, bf, T, n, d, None)
+    call("er_readmode", "hc_expand_then_read", x, H, y, bf, T, n, d, 4, a, 0, None, 1e-6, None)
+    call("er_null_a", "hc_expand_then_read", x, H, y, bf, T, n, d, 0, None, 0, None, 1e-6, None)
+    call("er_eps", "hc_expand_then_read", x, H, y, bf, T, n, d, 0, a, 0, None, -2.0, None)
+    call("er_alias_xr_H", "hc_expand_then_read", x, H, H + 64, bf, T, n, d, 0, a, 0, None, 1e-6, None)
+    call("er_alias_xr_x", "hc_expand_then_read", x, H, x + 32, bf, T, n, d, 0, a, 0, None, 1e-6, None)
+    call("er_d_too_big", "hc_expand_then_read", x, H, y, bf, T, n, 32768 + 8, 0, a, 0, None, 1e-6, None)
+    call("co_null_w", "hc_collapse", H, x, bf, T, n, d, 0, None, 0, None)
+    call("co_stride", "hc_collapse", H, x, bf, T, n, d, 0, a, -4, None)
+    call("co_alias", "hc_collapse", H, H + hb - xb + 16, bf, T, n, d, 0, a, 0, None)
+    call("co_mis_w", "hc_collapse", H, x, bf, T, n, d, 0, a + 1, 0, None)
     print(json.dumps(res))
 """)
 
@@ -125,6 +141,10 @@ def test_argument_validation_statuses():
         "mis_H": MIS, "mis_x": MIS, "mis_g": MIS, "mis_A": MIS, "alias_partial": ALI,
         "alias_y": ALI, "alias_x_H": ALI, "alias_x_read": ALI, "sk_n0": INV, "sk_K0": INV,
         "sk_null": INV, "sk_alias": ALI, "sk_T0": OK, "st_lo": INV, "st_hi": INV, "path_bad": INV,
+        "ex_T0": OK, "ex_n9": UNS, "ex_null": INV, "ex_mis": MIS, "ex_alias": ALI,
+        "er_readmode": INV, "er_null_a": INV, "er_eps": INV, "er_alias_xr_H": ALI,
+        "er_alias_xr_x": ALI, "er_d_too_big": UNS, "co_null_w": INV, "co_stride": INV,
+        "co_alias": ALI, "co_mis_w": MIS,
     }
     for tag, code in want.items():
         got, msg = res[tag]

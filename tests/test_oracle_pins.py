@@ -461,3 +461,85 @@ def test_mix_logits_closed_forms():
     want[0] = 0.75 / math.sqrt(0.75 ** 2 + 0.25)
     want[1] = -2.0 * 0.75 / math.sqrt(0.75 ** 2 + 0.25)
     assert np.allclose(zc[0], want, rtol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# stack ends: expansion into n copies, collapse by a weighted sum
+# ("Tencent open-sources Hy4 Preview at 770B -- Identity Hyper-Connections",
+# TL;DR and residual-design table: the streams start as copies of one)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_expand_is_n_copies(dt):
+    T, n, d = 5, 3, 24
+    x = gen.to_storage(gen.normal(601, (T, d)), dt)
+    H = oracle.expand(x, n, dt)
+    want = torch.from_numpy(x.view(np.int16) if dt == "bf16" else x).unsqueeze(1).expand(T, n, d)
+    got = torch.from_numpy(H.view(np.int16) if dt == "bf16" else H)
+    assert torch.equal(got, want)
+
+
+@pytest.mark.parametrize("n", [1, 2, 4])
+@pytest.mark.parametrize("dt", ["f32", "bf16"])
+def test_collapse_brute_force_exact_rationals(n, dt):
+    T, d = 3, 16
+    H = gen.to_storage(gen.normal(611 + n, (T, n, d)), dt)
+    w = gen.normal(612 + n, (T, n))
+    out = f32_of(oracle.collapse(H, w, dt), dt)
+    Hv = f32_of(H, dt)
+    for t in range(T):
+        for k in range(d):
+            terms = [Fraction(float(w[t, i])) * Fraction(float(Hv[t, i, k])) for i in range(n)]
+            exact = sum(terms, Fraction(0))
+            mag = float(sum(abs(x) for x in terms))
+            bound = 1.01 * n * U32 * mag
+            if dt == "bf16":
+                bound += 2.0 ** -8 * abs(float(exact)) * 1.01
+            assert abs(float(Fraction(float(out[t, k])) - exact)) <= bound, (t, k)
+
+
+def test_collapse_closed_forms():
+    """One-hot weights return that stream bit for bit; weights (1, 1) return
+    the fp32 sum of the two streams rounded once to bf16 (torch's add and
+    round); expand then a one-hot collapse returns the input."""
+    T, n, d = 4, 4, 32
+    H = gen.to_storage(gen.normal(621, (T, n, d)), "bf16")
+    for k in range(n):
+        w = np.zeros(n, np.float32)
+        w[k] = 1.0
+        assert np.array_equal(oracle.collapse(H, w, "bf16"), H[:, k])
+    H2 = np.ascontiguousarray(H[:, :2])
+    got = oracle.collapse(H2, np.ones(2, np.float32), "bf16")
+    tH = torch.from_numpy(H2.view(np.int16)).view(torch.bfloat16).float()
+    want = (tH[:, 0] + tH[:, 1]).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, want)
+    x = gen.to_storage(gen.normal(622, (T, d)), "bf16")
+    assert np.array_equal(oracle.collapse(oracle.expand(x, 3, "bf16"),
+                                          np.array([0, 1, 0], np.float32), "bf16"), x)
+
+
+def test_collapse_softmax_logits_against_library_softmax():
+    T, n, d = 6, 4, 16
+    H = gen.to_storage(gen.normal(631, (T, n, d)), "f32")
+    l = gen.normal(632, (T, n))
+    got = oracle.collapse(H, l, "f32", read_logits=True).astype(np.float64)
+    w = torch.softmax(torch.from_numpy(l.astype(np.float64)), dim=-1).numpy()
+    want = np.einsum("ti,tik->tk", w, H.astype(np.float64))
+    mag = np.einsum("ti,tik->tk", w, np.abs(H.astype(np.float64)))
+    assert np.all(np.abs(got - want) <= 8 * U32 * mag + 1e-30)
+
+
+def test_expand_then_read_is_prenorm_of_the_input():
+    """Copies of x read with weights summing to 1 in dyadic steps (0.25 each)
+    mix back to x exactly, so layer 0's block input is RMSNorm(x) g: compare
+    with the library's rms_norm in fp64."""
+    T, n, d = 8, 4, 128
+    x = gen.normal(641, (T, d))
+    g = gen.uniform(642, (d,), 0.5, 1.5)
+    a = np.full(n, 0.25, np.float32)
+    H, xr = oracle.expand_then_read(x, n, a, g, 1e-6, "f32")
+    assert np.array_equal(H[:, 3], x)
+    ref = torch.nn.functional.rms_norm(torch.from_numpy(x.astype(np.float64)), (d,),
+                                       weight=torch.from_numpy(g.astype(np.float64)),
+                                       eps=float(np.float32(1e-6))).numpy()
+    assert np.max(np.abs(xr - ref) / (np.abs(ref) + 1e-3)) < 1e-6
