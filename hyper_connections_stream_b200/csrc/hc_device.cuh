@@ -164,7 +164,12 @@ constexpr int kGroupScratch = 64;  // floats per warp: TPW * n * n <= 64 for n <
 // sees a fixed sequence of correctly rounded operations. The R batches share
 // the passes, so their latencies overlap. `scratch` holds R * kGroupScratch
 // floats for this warp.
-template <int N, int R>
+// SHFL selects how a lane gathers the n values of its row (column) when it
+// owns one element (n <= 5): warp shuffles (shortest latency for one batch,
+// the decode-sized calls) or the shared-memory buffer (more batches per unit
+// time: the pipelined kernel's parameter warp, which must keep pace with the
+// streams, measured faster on B200). Results are identical either way.
+template <int N, int R, bool SHFL = true>
 __device__ __forceinline__ void group_sinkhorn(float (&m)[R][Group<N>::EPL], float *scratch,
                                                int lane, int K) {
     constexpr int NN = N * N, GL = Group<N>::GL, EPL = Group<N>::EPL;
@@ -184,7 +189,7 @@ __device__ __forceinline__ void group_sinkhorn(float (&m)[R][Group<N>::EPL], flo
 #pragma unroll
         for (int r = 0; r < EPL; ++r) m[b][r] = expf(m[b][r]);
     }
-    if constexpr (EPL == 1) {
+    if constexpr (EPL == 1 && SHFL) {
         // one element per lane: the n values of a row (column) are fetched
         // with independent shuffles and added in index order
         const int base = lane & ~(GL - 1);

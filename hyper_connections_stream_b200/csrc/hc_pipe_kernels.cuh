@@ -367,7 +367,7 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
             }
             if (!__all_sync(0xffffffffu, w)) break;
             if constexpr (WRITE) {
-                if (p.mix_logits) group_sinkhorn<N, R>(mv, pscratch, lane, p.K);
+                if (p.mix_logits) group_sinkhorn<N, R, false>(mv, pscratch, lane, p.K);
             }
             if constexpr (READ) {
                 if (p.read_logits) {
