@@ -291,6 +291,90 @@ def run_ends(args):
     }
 
 
+def run_linear_write(args):
+    """The block's output projection fused with the write mix
+    (hc_linear_then_write) on the workload's streams: X [T, k=7168] times
+    Wo^T [7168, d=7168] on the tensor cores, then the write of the n=4 streams
+    with per-token Sinkhorn-projected A, y never stored. Device-timed, one
+    launch per step. Also times the unfused pair it replaces (torch.matmul,
+    i.e. cuBLAS, storing y, then hc_write_mix) for context."""
+    import numpy as np
+    import torch
+    import hc_inputs as gen
+    from hyper_connections_stream_b200 import _lib as hc
+    ws, rank, local = _dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = dict(WORKLOAD)
+    if args.tokens:
+        w["T"] = args.tokens
+    T, n, d = w["T"], w["n"], w["d"]
+    k = d
+    X = gen.device_normal(gen.SEED_Y + w["cfg"], (T, k), torch.bfloat16, device)
+    Wo = gen.device_normal(505, (d, k), torch.bfloat16, device, std=1.0 / np.sqrt(k))
+    Hs = [gen.device_normal(gen.SEED_H + w["cfg"], (T, n, d), torch.bfloat16, device),
+          torch.empty((T, n, d), dtype=torch.bfloat16, device=device)]
+    L = gen.device_normal(gen.SEED_L + w["cfg"], (T, n, n), torch.float32, device)
+    A = hc.sinkhorn(L, w["K"])
+    b = torch.from_numpy(gen.normal(gen.SEED_P + w["cfg"], (n,), mean=1.0, std=0.02)).to(device)
+    y = torch.empty((T, d), dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def timed(fn, steps):
+        for i in range(args.warmup):
+            fn(i)
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for i in range(steps):
+            ev[i][0].record(stream)
+            fn(i)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        return (statistics.mean(s_.elapsed_time(e) for s_, e in ev),
+                ev[0][0].elapsed_time(ev[-1][1]))
+
+    def fused(i):
+        hc.linear_then_write(X, Wo, Hs[i % 2], A, b, out=Hs[(i + 1) % 2])
+
+    def unfused(i):
+        torch.matmul(X, Wo.t(), out=y)
+        hc.write_mix(Hs[i % 2], y, A, b, out=Hs[(i + 1) % 2])
+
+    def cublas(i):
+        torch.matmul(X, Wo.t(), out=y)
+
+    kern_ms, total_ms = timed(fused, args.steps)
+    ref_steps = max(3, min(args.steps, 50))
+    unfused_ms, _ = timed(unfused, ref_steps)
+    cublas_ms, _ = timed(cublas, ref_steps)
+    flops = 2.0 * T * k * d
+    tflops = flops / (kern_ms / 1e3) / 1e12
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peak, peak_kind = float(json.load(f)["bf16_tflops"]), "measured (burst)"
+    except Exception:
+        peak, peak_kind = 1590.0, "fallback"
+    hbm_bytes = T * k * 2 + d * k * 2 + T * n * d * 2 * 2 + T * n * n * 4
+    return {
+        "metric": "block output projection + HC write tokens/sec at n=4, d=k=7168 (bf16, tensor cores)",
+        "value": T * args.steps / (total_ms / 1e3), "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "linear_write", "T": T, "n": n, "d": d, "k": k,
+                   "mix": "per-token Sinkhorn-projected A (K=20)", "l2": "inputs and outputs > L2"},
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                     "frac": tflops / peak, "traffic": None, "peak_source": peak_kind,
+                     "flops_per_launch": flops, "kernel_ms": kern_ms,
+                     "hbm_bytes_min": hbm_bytes,
+                     "hbm_gbs_at_min_bytes": hbm_bytes / (kern_ms / 1e3) / 1e9},
+        "unfused": {"ms": unfused_ms, "cublas_matmul_ms": cublas_ms,
+                    "how": "torch.matmul(X, Wo.T, out=y) then hc_write_mix (y stored and re-read)"},
+        "gpu_launches": args.steps, "device_fault": hc.device_fault(),
+    }
+
+
 def run_ours(args):
     import torch
     from hyper_connections_stream_b200 import _lib as hc
@@ -535,10 +619,12 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-only", action="store_true",
                     help="device-timed kernel only (no e2e, no CPU baseline): for profiling")
-    ap.add_argument("--op", choices=["step", "logits", "expand_read", "collapse"], default="step",
+    ap.add_argument("--op", choices=["step", "logits", "expand_read", "collapse", "linear_write"],
+                    default="step",
                     help="step: the fused HC step (the metric); logits: the tensor-core "
                          "mixing-logits kernel on the same streams; expand_read / collapse: "
-                         "the stack ends on the same shape")
+                         "the stack ends on the same shape; linear_write: the block's output "
+                         "projection fused with the write")
     ap.add_argument("--path", choices=["auto", "pipelined", "register"], default="auto",
                     help="kernel family (auto = pipelined wherever it applies)")
     ap.add_argument("--tokens", type=int, default=0,
@@ -556,6 +642,8 @@ def main(argv=None):
         line = run_logits(args)
     elif args.op in ("expand_read", "collapse"):
         line = run_ends(args)
+    elif args.op == "linear_write":
+        line = run_linear_write(args)
     else:
         line = run_ours(args)
     if line is not None:

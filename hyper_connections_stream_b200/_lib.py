@@ -40,6 +40,8 @@ SIGNATURES = {
     "hc_selftest_bounded_wait": ([_i32, _vp], _i32),
     "hc_mix_logits": ([_vp, _vp, _vp, _i32, _i64, _i32, _i64, _i32, _f32, _vp], _i32),
     "hc_expand": ([_vp, _vp, _i32, _i64, _i32, _i64, _vp], _i32),
+    "hc_linear_then_write": ([_vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i64, _i64, _vp, _i64,
+                              _vp, _i64, _vp], _i32),
     "hc_expand_then_read": ([_vp, _vp, _vp, _i32, _i64, _i32, _i64, _i32, _vp, _i64, _vp, _f32,
                              _vp], _i32),
     "hc_collapse": ([_vp, _vp, _i32, _i64, _i32, _i64, _i32, _vp, _i64, _vp], _i32),
@@ -310,4 +312,29 @@ def collapse(H, w, *, read: int = READ_WEIGHTS, out=None):
     _need_out("out", out, (T, d), H.dtype)
     _check(lib().hc_collapse(_ptr(H), _ptr(out), _DT[H.dtype], T, n, d, int(read), _ptr(w), w_s,
                              _stream(H.device)))
+    return out
+
+
+def linear_then_write(X, Wo, H, A, b, *, out=None, y_out=None):
+    """The block's output projection fused with the write mix:
+    y = bf16(X Wo^T) on the tensor cores, H'_j = sum_i A[i,j] H_i + b_j y.
+    X [T, k], Wo [d, k], H [T, n, d], all bf16; A [n, n] or [T, n, n] (a
+    matrix); b [n] or [T, n]. y is stored only if y_out is given. out may be H."""
+    _need_cuda("X", X, torch.bfloat16)
+    _need_cuda("Wo", Wo, torch.bfloat16)
+    _need_cuda("H", H, torch.bfloat16)
+    T, n, d = _streams_shape(H)
+    if X.dim() != 2 or X.shape[0] != T:
+        raise ValueError(f"X must be [T = {T}, k], got {tuple(X.shape)}")
+    k = X.shape[1]
+    if tuple(Wo.shape) != (d, k):
+        raise ValueError(f"Wo must be [d = {d}, k = {k}], got {tuple(Wo.shape)}")
+    A_s = _tok_param("A", A, T, (n, n))
+    b_s = _tok_param("b", b, T, (n,))
+    out = torch.empty_like(H) if out is None else out
+    _need_out("out", out, (T, n, d), torch.bfloat16)
+    if y_out is not None:
+        _need_out("y_out", y_out, (T, d), torch.bfloat16)
+    _check(lib().hc_linear_then_write(_ptr(X), _ptr(Wo), _ptr(H), _ptr(out), _ptr(y_out), HC_BF16,
+                                      T, n, d, k, _ptr(A), A_s, _ptr(b), b_s, _stream(H.device)))
     return out

@@ -421,4 +421,45 @@ hc_status hc_collapse(const void *H, void *out, hc_dtype dt, int64_t T, int n, i
     return dispatch<hc::KIND_COLLAPSE>(dt, n, p, static_cast<cudaStream_t>(stream));
 }
 
+hc_status hc_linear_then_write(const void *X, const void *Wo, const void *H, void *Hout, void *y_out,
+                               hc_dtype dt, int64_t T, int n, int64_t d, int64_t k, const float *A,
+                               int64_t A_tok_stride, const float *b, int64_t b_tok_stride,
+                               hc_stream stream) {
+    static const char *fn = "hc_linear_then_write";
+    g_last_error[0] = '\0';
+    if (dt != HC_BF16) return fail(HC_ERR_UNSUPPORTED, "%s: bf16 storage only (dtype %d)", fn, (int)dt);
+    const Shape s{dt, T, n, d};
+    HC_TRY(check_shape(fn, s, false));
+    if (k < 1) return fail(HC_ERR_INVALID_ARG, "%s: k = %lld < 1", fn, (long long)k);
+    if (k % 8 != 0)
+        return fail(HC_ERR_UNSUPPORTED, "%s: k = %lld is not a multiple of 8 (16-byte rows)", fn,
+                    (long long)k);
+    if (k > (int64_t(1) << 31) || d > (int64_t(1) << 31) || T > (int64_t(1) << 31))
+        return fail(HC_ERR_UNSUPPORTED, "%s: T, d and k must each be below 2^31", fn);
+    HC_TRY(check_stride(fn, "A_tok_stride", A_tok_stride));
+    HC_TRY(check_stride(fn, "b_tok_stride", b_tok_stride));
+    if (T == 0) return HC_OK;
+    HC_TRY(check_buf(fn, "X", X));
+    HC_TRY(check_buf(fn, "Wo", Wo));
+    HC_TRY(check_buf(fn, "H", H));
+    HC_TRY(check_buf(fn, "Hout", Hout));
+    if (y_out && !aligned(y_out, 16)) return fail(HC_ERR_MISALIGNED, "%s: y_out is not 16-byte aligned", fn);
+    HC_TRY(check_param(fn, "A", A));
+    HC_TRY(check_param(fn, "b", b));
+    const int64_t hb = T * n * d * 2, yb = T * d * 2, xb = T * k * 2, wb = d * k * 2;
+    if (Hout != H && overlap(Hout, hb, H, hb)) return fail(HC_ERR_ALIAS, "%s: Hout partially overlaps H", fn);
+    if (overlap(Hout, hb, X, xb) || overlap(Hout, hb, Wo, wb))
+        return fail(HC_ERR_ALIAS, "%s: Hout overlaps X or Wo", fn);
+    if (y_out && (overlap(y_out, yb, H, hb) || overlap(y_out, yb, Hout, hb) ||
+                  overlap(y_out, yb, X, xb) || overlap(y_out, yb, Wo, wb)))
+        return fail(HC_ERR_ALIAS, "%s: y_out overlaps another buffer", fn);
+    hc::LaunchCtx ctx{};
+    HC_TRY(launch_ctx(ctx));
+    hc::LinearWriteArgs la{};
+    la.X = X; la.Wo = Wo; la.H = H; la.Hout = Hout; la.y = y_out;
+    la.T = T; la.d = d; la.k = k; la.n = n;
+    la.A = A; la.A_s = A_tok_stride; la.b = b; la.b_s = b_tok_stride;
+    return hc::launch_linear_write(la, ctx, static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

@@ -2,6 +2,7 @@
 // and the kernel translation units (one per storage dtype and kernel kind).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "hc_api.h"
@@ -25,9 +26,28 @@ hc_status set_error(hc_status st, const char *fmt, ...);
 template <typename S, int KIND>
 hc_status launch_kind(int n, const StepParams &p, const LaunchCtx &ctx, cudaStream_t st);
 
+// 2-D bf16 TMA tensor map over a row-major [outer][inner] array: 128-byte
+// swizzle, zero fill out of bounds, box of box_outer rows x box_inner elements.
+hc_status make_tma_map_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
+                            uint32_t box_inner, uint32_t box_outer);
+
 // Input-dependent mixing logits on the tensor cores (bf16 H and W).
 hc_status launch_mix_logits(const void *H, const void *W, float *z, int64_t T, int n, int64_t d,
                             int P, float eps, const LaunchCtx &ctx, cudaStream_t st);
+
+// The block's output projection fused with the write mix (bf16):
+// y = X Wo^T on the tensor cores, H'_j = sum_i A[i][j] H_i + b_j y.
+struct LinearWriteArgs {
+    const void *X, *Wo, *H;
+    void *Hout, *y;  // y may be null
+    int64_t T, d, k;
+    int n;
+    const float *A;
+    int64_t A_s;
+    const float *b;
+    int64_t b_s;
+};
+hc_status launch_linear_write(const LinearWriteArgs &a, const LaunchCtx &ctx, cudaStream_t st);
 
 hc_status launch_selftest_wait(int limit_us, const LaunchCtx &ctx, cudaStream_t st);
 

@@ -232,9 +232,12 @@ hc_logits_kernel(const __grid_constant__ CUtensorMap mapH, const __grid_constant
     if (lane == 0) mbar_arrive(done);
 }
 
+}  // namespace
+
+// 2-D bf16 tensor map with 128-byte swizzle and zero fill out of bounds.
 // cuTensorMapEncodeTiled through the runtime's driver entry point (the library
 // does not link the driver library directly).
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     if (!fn) {
         void *ptr = nullptr;
@@ -247,8 +250,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-hc_status make_map(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
-                   uint32_t box_inner, uint32_t box_outer) {
+hc_status make_tma_map_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t outer,
+                            uint32_t box_inner, uint32_t box_outer) {
     auto fn = encode_fn();
     if (!fn) return set_error(HC_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
     cuuint64_t gdim[2] = {inner, outer};
@@ -261,8 +264,6 @@ hc_status make_map(CUtensorMap *map, const void *base, uint64_t inner, uint64_t 
     if (r != CUDA_SUCCESS) return set_error(HC_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
     return HC_OK;
 }
-
-}  // namespace
 
 hc_status launch_mix_logits(const void *H, const void *W, float *z, int64_t T, int n, int64_t d,
                             int P, float eps, const LaunchCtx &ctx, cudaStream_t st) {
@@ -298,9 +299,9 @@ hc_status launch_mix_logits(const void *H, const void *W, float *z, int64_t T, i
     const int smem = fixed + stages * stage_bytes;
 
     CUtensorMap mapH, mapW;
-    hc_status ms = make_map(&mapH, H, (uint64_t)lp.K, (uint64_t)T, kLgKSub, (uint32_t)lp.rows);
+    hc_status ms = make_tma_map_bf16(&mapH, H, (uint64_t)lp.K, (uint64_t)T, kLgKSub, (uint32_t)lp.rows);
     if (ms != HC_OK) return ms;
-    ms = make_map(&mapW, W, (uint64_t)lp.K, (uint64_t)P, kLgKSub, (uint32_t)lp.Npad);
+    ms = make_tma_map_bf16(&mapW, W, (uint64_t)lp.K, (uint64_t)P, kLgKSub, (uint32_t)lp.Npad);
     if (ms != HC_OK) return ms;
 
     static int configured[64] = {};

@@ -140,6 +140,28 @@ HC_API hc_status hc_write_then_read(const void *H, const void *y, void *Hout, vo
                              hc_stream stream);
 
 /*
+ * The block's output projection fused with the write mix, so the block output
+ * y never makes a round trip through HBM (Hy4-preview model techniques map,
+ * models.inteligile.com, "inference kernel": kernel fusion used; glossary entry
+ * "Hyper-connections (mHC)": the streams are mixed after each block):
+ *   y[t][c]  = bf16( sum_k X[t][k] * Wo[c][k] )   fp32 accumulation on the tensor
+ *              cores, rounded to bf16 as a stored y would be;
+ *   H'[t][j] = sum_i A[i][j] H[t][i] + b_j y[t]   as hc_write_mix with a given
+ *              matrix (the per-token Sinkhorn form projects its logits first
+ *              with hc_sinkhorn).
+ *   X [T][k], Wo [d][k] (the projection's weight, one row per output channel),
+ *   H and Hout [T][n][d]; bf16 only. k % 8 == 0, d % 8 == 0, 1 <= n <= 8.
+ *   A [n][n] / b [n] per layer (tok_stride 0) or per token (floats per token).
+ *   y_out: if not NULL, y is also stored there ([T][d] bf16), else never.
+ *   Hout may equal H exactly (in place); no other overlap. X, Wo, H, Hout and
+ *   y_out 16-byte aligned. Asynchronous; T == 0 is a no-op.
+ */
+HC_API hc_status hc_linear_then_write(const void *X, const void *Wo, const void *H, void *Hout,
+                                      void *y_out, hc_dtype dt, int64_t T, int n, int64_t d,
+                                      int64_t k, const float *A, int64_t A_tok_stride,
+                                      const float *b, int64_t b_tok_stride, hc_stream stream);
+
+/*
  * Ends of a stack ("Tencent open-sources Hy4 Preview at 770B -- Identity
  * Hyper-Connections", learnaivisually: TL;DR and the residual-design table --
  * the n streams start as copies of one; the pages do not say how they are

@@ -43,6 +43,7 @@ def lib():
             "hco_mix_logits": ([vp, vp, vp, i32, i64, i32, i64, i32, fp], i32),
             "hco_single_stream_layer": ([vp, vp, i32, i64, i64, vp, fp], i32),
             "hco_expand": ([vp, vp, i32, i64, i32, i64], i32),
+            "hco_linear": ([vp, vp, vp, i32, i64, i64, i64], i32),
             "hco_collapse": ([vp, vp, i32, i64, i32, i64, i32, vp, i64], i32),
         }
         for name, (args, res) in sig.items():
@@ -200,6 +201,17 @@ def collapse(H, w, dt: str, read_logits: bool = False):
     _chk(lib().hco_collapse(_p(H), _p(out), _DT[dt], T, n, d, int(read_logits), _p(w),
                             _tok_stride(w, T, n)), "collapse")
     return out
+
+
+def linear(X, W, dt: str):
+    """fp64 y[t, c] = sum_k X[t, k] W[c, k]. X [T, k], W [d, k] storage arrays."""
+    X = _arr(X, _NP[dt]); W = _arr(W, _NP[dt])
+    T, k = X.shape
+    d = W.shape[0]
+    assert W.shape == (d, k)
+    y = np.empty((T, d), dtype=np.float64)
+    _chk(lib().hco_linear(_p(X), _p(W), _p(y), _DT[dt], T, k, d), "linear")
+    return y
 
 
 def block_tanh(x, dt: str):

@@ -393,6 +393,26 @@ int hco_collapse(const void *H, void *out, int dt, int64_t T, int n, int64_t d, 
     return HCO_OK;
 }
 
+/*
+ * The block's output projection (a plain linear map), as a reference for the
+ * fused projection + write: y[t][c] = sum_k X[t][k] * W[c][k], W one row per
+ * output channel. Computed in fp64 (products of bf16 or fp32 values are exact
+ * in fp64; sums in index order), stored as fp64. Not part of the HC step
+ * itself: the write mix of a given y is hco_write_mix.
+ */
+int hco_linear(const void *X, const void *W, double *y, int dt, int64_t T, int64_t k, int64_t d) {
+    if ((dt != HCO_F32 && dt != HCO_BF16) || T < 0 || k < 1 || d < 1) return HCO_EINVAL;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int64_t kk = 0; kk < k; ++kk)
+                acc += (double)load_s(X, dt, t * k + kk) * (double)load_s(W, dt, c * k + kk);
+            y[t * d + c] = acc;
+        }
+    return HCO_OK;
+}
+
 /* Harness block stand-in: y = round_s(tanhf(x)). Not part of the HC step. */
 int hco_block_tanh(const void *x, void *y, int dt, int64_t count) {
     if (dt != HCO_F32 && dt != HCO_BF16) return HCO_EINVAL;

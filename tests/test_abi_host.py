@@ -120,6 +120,15 @@ _CHILD = textwrap.dedent(r"""
     call("co_stride", "hc_collapse", H, x, bf, T, n, d, 0, a, -4, None)
     call("co_alias", "hc_collapse", H, H + hb - xb + 16, bf, T, n, d, 0, a, 0, None)
     call("co_mis_w", "hc_collapse", H, x, bf, T, n, d, 0, a + 1, 0, None)
+    Xl, Wl = buf(20), buf(40)
+    call("lw_f32", "hc_linear_then_write", Xl, Wl, H, Ho, None, B.HC_F32, T, n, d, 64, A, 0, b, 0, None)
+    call("lw_k_ragged", "hc_linear_then_write", Xl, Wl, H, Ho, None, bf, T, n, d, 60, A, 0, b, 0, None)
+    call("lw_k0", "hc_linear_then_write", Xl, Wl, H, Ho, None, bf, T, n, d, 0, A, 0, b, 0, None)
+    call("lw_T0", "hc_linear_then_write", None, None, None, None, None, bf, 0, n, d, 64, None, 0, None, 0, None)
+    call("lw_mis_X", "hc_linear_then_write", Xl + 8, Wl, H, Ho, None, bf, T, n, d, 64, A, 0, b, 0, None)
+    call("lw_null_A", "hc_linear_then_write", Xl, Wl, H, Ho, None, bf, T, n, d, 64, None, 0, b, 0, None)
+    call("lw_alias_y", "hc_linear_then_write", Xl, Wl, H, Ho, Ho + 64, bf, T, n, d, 64, A, 0, b, 0, None)
+    call("lw_alias_X", "hc_linear_then_write", Xl, Wl, H, Xl + 32, None, bf, T, n, d, 64, A, 0, b, 0, None)
     print(json.dumps(res))
 """)
 
@@ -145,6 +154,8 @@ def test_argument_validation_statuses():
         "er_readmode": INV, "er_null_a": INV, "er_eps": INV, "er_alias_xr_H": ALI,
         "er_alias_xr_x": ALI, "er_d_too_big": UNS, "co_null_w": INV, "co_stride": INV,
         "co_alias": ALI, "co_mis_w": MIS,
+        "lw_f32": UNS, "lw_k_ragged": UNS, "lw_k0": INV, "lw_T0": OK, "lw_mis_X": MIS,
+        "lw_null_A": INV, "lw_alias_y": ALI, "lw_alias_X": ALI,
     }
     for tag, code in want.items():
         got, msg = res[tag]

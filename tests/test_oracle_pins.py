@@ -543,3 +543,25 @@ def test_expand_then_read_is_prenorm_of_the_input():
                                        weight=torch.from_numpy(g.astype(np.float64)),
                                        eps=float(np.float32(1e-6))).numpy()
     assert np.max(np.abs(xr - ref) / (np.abs(ref) + 1e-3)) < 1e-6
+
+
+# --------------------------------------------------------------------------
+# the block's output projection (reference for the fused projection + write)
+# --------------------------------------------------------------------------
+
+def test_linear_against_library_matmul_and_closed_forms():
+    T, k, d = 7, 40, 24
+    X = gen.to_storage(gen.normal(801, (T, k)), "bf16")
+    W = gen.to_storage(gen.normal(802, (d, k)), "bf16")
+    y = oracle.linear(X, W, "bf16")
+    ref = torch.from_numpy(f32_of(X, "bf16")) @ torch.from_numpy(f32_of(W, "bf16")).T
+    assert np.max(np.abs(y - ref.numpy())) <= 1e-13 * np.max(np.abs(ref.numpy()))
+    # identity weights return X; a one-hot row picks one input channel
+    I = gen.to_storage(np.eye(k, dtype=np.float32), "bf16")
+    assert np.array_equal(oracle.linear(X, I, "bf16"), f32_of(X, "bf16"))
+    W1 = np.zeros((2, k), np.float32)
+    W1[0, 3] = 1.0
+    W1[1, k - 1] = -2.0
+    y1 = oracle.linear(X, gen.to_storage(W1, "bf16"), "bf16")
+    assert np.array_equal(y1[:, 0], f32_of(X, "bf16")[:, 3])
+    assert np.array_equal(y1[:, 1], -2.0 * f32_of(X, "bf16")[:, k - 1])
