@@ -9,21 +9,27 @@
 // kernel: kernel fusion used"; the glossary entry "Hyper-connections (mHC)":
 // the streams are mixed after each block.)
 //
-// Persistent kernel, one CTA per SM, 192 threads; output tiles of 128 tokens x
-// 256 channels are handed out round-robin:
-//   warp 0      TMA producer: per k-step of 64, the 128B-swizzled X tile
-//               (128 x 64) and Wo tile (256 x 64) into a ring of stages;
-//   warp 1      allocates 512 TMEM columns (two 128 x 256 fp32 accumulators);
-//               one lane issues tcgen05.mma (M = 128, N = 256, K = 16) and
-//               commits each stage back to the producer and each finished
-//               accumulator to the epilogue;
-//   warps 2-5   epilogue, one thread per token row (TMEM lane): tcgen05.ld 16
-//               channels of y, round to bf16, then for each 8-channel half
-//               load the token's n stream slices, mix, store H'. The epilogue
-//               of tile i overlaps the MMAs of tile i+1 (the other
-//               accumulator).
-// Every wait is bounded; on time-out the CTA records a fault, drains its
-// copies and MMAs, frees TMEM and exits.
+// Persistent kernel on CTA pairs (clusters of two, one CTA per SM, 192
+// threads each); output tiles of 256 tokens x 256 channels are handed out
+// round-robin to the pairs. CTA r of a pair stages token rows 128r..128r+127
+// of X and channel rows 128r..128r+127 of Wo, so each SM streams 32 KB per
+// k-step for a 256 x 256 x 64 product (a third less than one CTA per tile):
+//   warp 0      TMA producer: per k-step of 64, the 128B-swizzled X and Wo
+//               halves into a ring of stages; the bytes of both CTAs complete
+//               on the leader's stage barrier;
+//   warp 1      TMEM (512 columns: two 128 x 256 fp32 accumulators per CTA,
+//               allocated for the pair); in the leader one lane issues
+//               tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16) and
+//               commits each stage and each finished accumulator to both CTAs;
+//   warps 2-5   epilogue of this CTA's 128 rows: tcgen05.ld of the
+//               accumulator (one token row per thread), rounded to bf16 and
+//               transposed through shared memory, then the write mix of the
+//               token's n stream slices with coalesced 256-byte loads and
+//               stores; the accumulator is handed back to the leader's MMA as
+//               soon as it has been read, so the epilogue of tile i overlaps
+//               the MMAs of tile i+1.
+// Every wait is bounded; on time-out a CTA records a fault, drains its copies
+// and MMAs and leaves through the closing cluster barrier.
 #include <cuda.h>
 
 #include "hc_launch.h"
@@ -34,15 +40,18 @@ namespace hc {
 namespace {
 
 constexpr int kLwThreads = 192;
-constexpr int kLwM = 128;                    // tokens per tile (TMEM lanes)
+constexpr int kLwM = 128;                    // token rows per CTA (TMEM lanes)
+constexpr int kLwTileM = 2 * kLwM;           // token rows per pair tile (MMA M)
 constexpr int kLwN = 256;                    // channels per tile (MMA N)
+constexpr int kLwBRows = kLwN / 2;           // Wo rows staged per CTA
 constexpr int kLwK = 64;                     // k per stage: one 128-byte swizzle row
 constexpr int kLwABytes = kLwM * kLwK * 2;   // 16 KB
-constexpr int kLwBBytes = kLwN * kLwK * 2;   // 32 KB
+constexpr int kLwBBytes = kLwBRows * kLwK * 2;  // 16 KB
 constexpr int kLwStageBytes = kLwABytes + kLwBBytes;
-constexpr int kLwStages = 4;
+constexpr int kLwStages = 6;
 constexpr uint32_t kLwTmemCols = 2 * kLwN;
-constexpr int kLwSmem = 1024 /* alignment slack */ + kLwStages * kLwStageBytes +
+constexpr int kLwYBufBytes = 32 * (kLwN / 2) * 2;  // one epilogue warp: 32 rows x 128 bf16
+constexpr int kLwSmem = 1024 /* alignment slack */ + kLwStages * kLwStageBytes + 4 * kLwYBufBytes +
                         (2 * kLwStages + 5) * 8 + 16;
 
 struct LinearWriteParams {
@@ -55,25 +64,35 @@ struct LinearWriteParams {
     int64_t b_s;
     int64_t T, d;
     int64_t tiles;
-    int num_n;  // channel tiles
+    int64_t num_m;  // token tiles
+    int num_n;      // channel tiles
     int nk;     // k-steps per tile
 };
 
-__device__ __forceinline__ void load_bf16x8(const __nv_bfloat16 *p, float (&v)[8]) {
-    const uint4 q = *reinterpret_cast<const uint4 *>(p);
-    widen_bf16x2(q.x, v[0], v[1]);
-    widen_bf16x2(q.y, v[2], v[3]);
-    widen_bf16x2(q.z, v[4], v[5]);
-    widen_bf16x2(q.w, v[6], v[7]);
+// Tile order: groups of kLwGroupM token blocks; inside a group the channel
+// block varies slowest, so the ~74 tiles in flight share a few Wo blocks
+// (3.7 MB each at k = 7168) and one group of X rows in L2, and Wo is read from
+// DRAM once per group instead of once per wave.
+constexpr int kLwGroupM = 8;
+
+__device__ __forceinline__ void tile_coords(int64_t tile, int64_t num_m, int num_n, int32_t &m0,
+                                            int32_t &n0) {
+    const int64_t group_tiles = (int64_t)kLwGroupM * num_n;
+    const int64_t g = tile / group_tiles;
+    const int64_t rem = tile - g * group_tiles;
+    const int64_t m_base = g * kLwGroupM;
+    const int64_t gm = num_m - m_base < kLwGroupM ? num_m - m_base : kLwGroupM;
+    m0 = (int32_t)((m_base + rem % gm) * kLwTileM);
+    n0 = (int32_t)((rem / gm) * kLwN);
 }
 
-__device__ __forceinline__ void store_bf16x8(__nv_bfloat16 *p, const float (&v)[8]) {
+__device__ __forceinline__ void store_bf16x8_cs(__nv_bfloat16 *p, const float (&v)[8]) {
     uint4 q;
     q.x = pack_bf16x2_rn(v[0], v[1]);
     q.y = pack_bf16x2_rn(v[2], v[3]);
     q.z = pack_bf16x2_rn(v[4], v[5]);
     q.w = pack_bf16x2_rn(v[6], v[7]);
-    *reinterpret_cast<uint4 *>(p) = q;
+    __stcs(reinterpret_cast<uint4 *>(p), q);
 }
 
 template <int N>
@@ -84,7 +103,7 @@ hc_linear_write_kernel(const __grid_constant__ CUtensorMap mapX,
     unsigned char *smem = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr int S = kLwStages;
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * kLwStageBytes);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + S * kLwStageBytes + 4 * kLwYBufBytes);
     uint64_t *empty = full + S;
     uint64_t *acc_full = empty + S;      // [2]
     uint64_t *acc_empty = acc_full + 2;  // [2]
@@ -94,15 +113,19 @@ hc_linear_write_kernel(const __grid_constant__ CUtensorMap mapX,
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();  // 0: the leader, which issues the MMAs
+    const bool leader = rank == 0;
+    const int64_t pair = blockIdx.x >> 1;
+    const int64_t npairs = gridDim.x >> 1;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);  // the MMA commit
+            mbar_init(&full[s], 1);   // leader: its producer's expect_tx (+ both CTAs' bytes)
+            mbar_init(&empty[s], 1);  // the MMA commit, multicast to both CTAs
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&acc_full[b], 1);   // the MMA commit
-            mbar_init(&acc_empty[b], 4);  // the four epilogue warps
+            mbar_init(&acc_full[b], 1);   // the MMA commit, multicast to both CTAs
+            mbar_init(&acc_empty[b], 8);  // leader: the four epilogue warps of each CTA
         }
         mbar_init(drained, 1);
         *abort_flag = 0;
@@ -111,24 +134,25 @@ hc_linear_write_kernel(const __grid_constant__ CUtensorMap mapX,
         prefetch_tensor_map(&mapW);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_slot, kLwTmemCols);
-        tmem_relinquish();
+        tmem_alloc_pair(tmem_slot, kLwTmemCols);
+        tmem_relinquish_pair();
     }
     tc_fence_before_sync();
-    __syncthreads();
+    cluster_sync_all();  // both CTAs' barriers initialised, TMEM allocated
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ---------------- TMA producer ----------------
+        // ---------------- TMA producer (both CTAs) ----------------
         if (lane == 0) {
+            const uint32_t full_leader = mapa_shared(smem_addr(&full[0]), 0);
             int s = 0;
             uint32_t ph = 0;
             int64_t it = 0;
             bool ok = true;
-            for (int64_t tile = blockIdx.x; ok && tile < p.tiles; tile += gridDim.x) {
-                const int32_t m0 = (int32_t)(tile / p.num_n) * kLwM;
-                const int32_t n0 = (int32_t)(tile % p.num_n) * kLwN;
+            for (int64_t tile = pair; ok && tile < p.tiles; tile += npairs) {
+                int32_t m0, n0;
+                tile_coords(tile, p.num_m, p.num_n, m0, n0);
                 for (int ks = 0; ks < p.nk; ++ks, ++it) {
                     if (it >= S &&
                         !mbar_wait_bounded(&empty[s], ph ^ 1u, abort_flag, fault, FAULT_WAIT_EMPTY)) {
@@ -136,29 +160,33 @@ hc_linear_write_kernel(const __grid_constant__ CUtensorMap mapX,
                         break;
                     }
                     unsigned char *st = smem + s * kLwStageBytes;
-                    mbar_arrive_expect_tx(&full[s], (uint32_t)kLwStageBytes);
-                    tma_load_2d(st, &mapX, ks * kLwK, m0, &full[s]);
-                    tma_load_2d(st + kLwABytes, &mapW, ks * kLwK, n0, &full[s]);
+                    if (leader) mbar_arrive_expect_tx(&full[s], (uint32_t)(2 * kLwStageBytes));
+                    tma_load_2d_pair(st, &mapX, ks * kLwK, m0 + (int32_t)rank * kLwM,
+                                     full_leader + 8u * (uint32_t)s);
+                    tma_load_2d_pair(st + kLwABytes, &mapW, ks * kLwK, n0 + (int32_t)rank * kLwBRows,
+                                     full_leader + 8u * (uint32_t)s);
                     if (++s == S) {
                         s = 0;
                         ph ^= 1u;
                     }
                 }
             }
-            // the copies still in flight land before the CTA exits
-            for (int64_t q = (it > S ? it - S : 0); q < it; ++q)
-                mbar_wait_drain(&full[q % S], (uint32_t)((q / S) & 1), fault);
+            // the copies still in flight (both CTAs' bytes complete on the
+            // leader's barriers) land before the pair leaves
+            if (leader)
+                for (int64_t q = (it > S ? it - S : 0); q < it; ++q)
+                    mbar_wait_drain(&full[q % S], (uint32_t)((q / S) & 1), fault);
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
-        if (lane == 0) {
-            const uint32_t idesc = umma_idesc_bf16_f32(kLwM, kLwN);
+        // ---------------- MMA issuer (the leader) ----------------
+        if (lane == 0 && leader) {
+            const uint32_t idesc = umma_idesc_bf16_f32(kLwTileM, kLwN);
             int s = 0;
             uint32_t ph = 0;
             int lt = 0;
             bool ok = true;
-            for (int64_t tile = blockIdx.x; ok && tile < p.tiles; tile += gridDim.x, ++lt) {
+            for (int64_t tile = pair; ok && tile < p.tiles; tile += npairs, ++lt) {
                 const int buf = lt & 1;
                 if (lt >= 2 && !mbar_wait_bounded(&acc_empty[buf], (uint32_t)(((lt >> 1) & 1) ^ 1),
                                                   abort_flag, fault, FAULT_WAIT_REDUCE))
@@ -176,109 +204,149 @@ hc_linear_write_kernel(const __grid_constant__ CUtensorMap mapX,
 #pragma unroll
                     for (int kk = 0; kk < kLwK / 16; ++kk) {
                         // +32 bytes along K per 16-element step inside the swizzle atom
-                        umma_bf16(dacc, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32),
-                                  idesc, (ks | kk) != 0);
+                        umma_bf16_pair(dacc, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32),
+                                       idesc, (ks | kk) != 0);
                     }
-                    umma_commit(&empty[s]);  // stage free once these MMAs have read it
+                    umma_commit_pair(&empty[s], 0x3);  // both CTAs' stages are free once read
                     if (++s == S) {
                         s = 0;
                         ph ^= 1u;
                     }
                 }
                 if (!ok) break;
-                umma_commit(&acc_full[buf]);  // accumulator complete
+                umma_commit_pair(&acc_full[buf], 0x3);  // both halves of the accumulator complete
             }
-            umma_commit(drained);  // every MMA issued so far has finished
+            umma_commit_pair(drained, 0x1);  // every MMA issued so far has finished
             mbar_wait_drain(drained, 0, fault);
         }
         __syncwarp();
     } else {
-        // ---------------- epilogue (warps 2..5) ----------------
+        // Warp q owns TMEM lanes (token rows) 32q..32q+31. Per half tile (128
+        // channels): (A) each thread loads its row's 128 accumulators, rounds
+        // them to bf16 and parks them in the warp's 8 KB slice of shared
+        // memory (16-byte chunks XOR-swizzled by row, so neither the row-wise
+        // writes nor the column-wise reads conflict); (B) the warp then walks
+        // its rows two at a time, a half-warp per row, each lane taking 8
+        // channels: the stream loads and H' stores are 256-byte coalesced
+        // runs. The accumulator is released right after the last TMEM load.
         const int quarter = warp & 3;  // TMEM lanes this warp may access
-        const int r = quarter * 32 + lane;
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-        float Am[N][N], bv[N];
-        if (p.A_s == 0) {
-#pragma unroll
-            for (int i = 0; i < N; ++i)
-#pragma unroll
-                for (int j = 0; j < N; ++j) Am[i][j] = p.A[i * N + j];
-        }
-        if (p.b_s == 0) {
-#pragma unroll
-            for (int j = 0; j < N; ++j) bv[j] = p.b[j];
-        }
+        unsigned char *ybuf = smem + S * kLwStageBytes + quarter * kLwYBufBytes;
+        // row pairs per iteration: as many as the registers hold (packed bf16)
+        constexpr int RPI = N <= 1 ? 16 : N <= 2 ? 8 : N <= 4 ? 4 : 1;
+        const int half_lane = lane >> 4;  // which row of the pair
+        const int lc = lane & 15;         // 16-byte chunk of the row (8 channels)
         int lt = 0;
-        for (int64_t tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++lt) {
+        const uint32_t acc_empty_leader = mapa_shared(smem_addr(&acc_empty[0]), 0);
+        for (int64_t tile = pair; tile < p.tiles; tile += npairs, ++lt) {
             const int buf = lt & 1;
             const bool w = mbar_wait_bounded(&acc_full[buf], (uint32_t)((lt >> 1) & 1), abort_flag,
                                              fault, FAULT_WAIT_FULL);
             if (!__all_sync(0xffffffffu, w)) break;
             tc_fence_after_sync();
-            const int64_t t = (tile / p.num_n) * kLwM + r;
-            const int64_t n0 = (tile % p.num_n) * kLwN;
-            const bool live = t < p.T;
-            if (live) {
-                if (p.A_s != 0) {
+            int32_t m0, n0;
+            tile_coords(tile, p.num_m, p.num_n, m0, n0);
+            const int64_t t0 = (int64_t)m0 + (int64_t)rank * kLwM + quarter * 32;  // this warp's first row
+#pragma unroll 1
+            for (int hf = 0; hf < 2; ++hf) {
+                // (A) accumulators -> bf16 -> shared memory (row = lane)
 #pragma unroll
-                    for (int i = 0; i < N; ++i)
-#pragma unroll
-                        for (int j = 0; j < N; ++j) Am[i][j] = p.A[t * p.A_s + i * N + j];
+                for (int c0 = 0; c0 < kLwN / 2; c0 += 16) {
+                    uint32_t v[16];
+                    tmem_ld_32x32b_x16(lane_base + (uint32_t)(buf * kLwN + hf * (kLwN / 2) + c0), v);
+                    tmem_ld_wait();
+                    uint4 q0, q1;
+                    q0.x = pack_bf16x2_rn(__uint_as_float(v[0]), __uint_as_float(v[1]));
+                    q0.y = pack_bf16x2_rn(__uint_as_float(v[2]), __uint_as_float(v[3]));
+                    q0.z = pack_bf16x2_rn(__uint_as_float(v[4]), __uint_as_float(v[5]));
+                    q0.w = pack_bf16x2_rn(__uint_as_float(v[6]), __uint_as_float(v[7]));
+                    q1.x = pack_bf16x2_rn(__uint_as_float(v[8]), __uint_as_float(v[9]));
+                    q1.y = pack_bf16x2_rn(__uint_as_float(v[10]), __uint_as_float(v[11]));
+                    q1.z = pack_bf16x2_rn(__uint_as_float(v[12]), __uint_as_float(v[13]));
+                    q1.w = pack_bf16x2_rn(__uint_as_float(v[14]), __uint_as_float(v[15]));
+                    const int ch = c0 >> 3;  // logical chunk (even)
+                    *reinterpret_cast<uint4 *>(ybuf + lane * 256 + ((ch ^ (lane & 7)) << 4)) = q0;
+                    *reinterpret_cast<uint4 *>(ybuf + lane * 256 + (((ch + 1) ^ (lane & 7)) << 4)) = q1;
                 }
-                if (p.b_s != 0) {
-#pragma unroll
-                    for (int j = 0; j < N; ++j) bv[j] = p.b[t * p.b_s + j];
+                if (hf == 1) {
+                    // every accumulator of this tile is in registers or shared memory
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(acc_empty_leader + 8u * (uint32_t)buf);
                 }
-            }
-            const __nv_bfloat16 *Ht = p.H + t * N * p.d;
-            __nv_bfloat16 *Hot = p.Hout + t * N * p.d;
-            for (int c0 = 0; c0 < kLwN; c0 += 16) {
-                uint32_t v[16];
-                tmem_ld_32x32b_x16(lane_base + (uint32_t)(buf * kLwN + c0), v);
-                tmem_ld_wait();
+                __syncwarp();
+                // (B) rows in pairs, coalesced along the channels. The stream
+                // slices of RPI row pairs are loaded (packed bf16) before any
+                // is mixed, so each iteration keeps RPI * n * 512 bytes per
+                // warp in flight.
+                const int64_t c = n0 + hf * (kLwN / 2) + lc * 8;
+                for (int rr = 0; rr < 32; rr += 2 * RPI) {
+                    uint4 hraw[RPI][N], yraw[RPI];
+                    bool live[RPI];
+                    int64_t t[RPI];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int64_t c = n0 + c0 + 8 * h;
-                    if (!live || c >= p.d) continue;
-                    // y as a stored bf16 value would hold it
-                    float yv[8];
+                    for (int u = 0; u < RPI; ++u) {
+                        const int row = rr + 2 * u + half_lane;
+                        t[u] = t0 + row;
+                        live[u] = t[u] < p.T && c < p.d;
+                        yraw[u] = *reinterpret_cast<const uint4 *>(ybuf + row * 256 + ((lc ^ (row & 7)) << 4));
+                        if (live[u]) {
+                            const __nv_bfloat16 *Ht = p.H + t[u] * N * p.d + c;
 #pragma unroll
-                    for (int e = 0; e < 8; e += 2) {
-                        const uint32_t q =
-                            pack_bf16x2_rn(__uint_as_float(v[8 * h + e]), __uint_as_float(v[8 * h + e + 1]));
-                        widen_bf16x2(q, yv[e], yv[e + 1]);
+                            for (int i = 0; i < N; ++i)
+                                hraw[u][i] = __ldcs(reinterpret_cast<const uint4 *>(Ht + i * p.d));
+                        }
                     }
-                    if (p.y) store_bf16x8(p.y + t * p.d + c, yv);
-                    float hv[N][8];
 #pragma unroll
-                    for (int i = 0; i < N; ++i) load_bf16x8(Ht + i * p.d + c, hv[i]);
+                    for (int u = 0; u < RPI; ++u) {
+                        if (!live[u]) continue;
+                        if (p.y) *reinterpret_cast<uint4 *>(p.y + t[u] * p.d + c) = yraw[u];
+                        float hv[N][8], yv[8];
 #pragma unroll
-                    for (int j = 0; j < N; ++j) {
-                        float acc[8];
+                        for (int i = 0; i < N; ++i) {
+                            widen_bf16x2(hraw[u][i].x, hv[i][0], hv[i][1]);
+                            widen_bf16x2(hraw[u][i].y, hv[i][2], hv[i][3]);
+                            widen_bf16x2(hraw[u][i].z, hv[i][4], hv[i][5]);
+                            widen_bf16x2(hraw[u][i].w, hv[i][6], hv[i][7]);
+                        }
+                        widen_bf16x2(yraw[u].x, yv[0], yv[1]);
+                        widen_bf16x2(yraw[u].y, yv[2], yv[3]);
+                        widen_bf16x2(yraw[u].z, yv[4], yv[5]);
+                        widen_bf16x2(yraw[u].w, yv[6], yv[7]);
+                        // the row's parameters (stride 0: shared by all tokens), L1 broadcasts
+                        const float *Ap = p.A + t[u] * p.A_s;
+                        const float *bp = p.b + t[u] * p.b_s;
+                        __nv_bfloat16 *Hot = p.Hout + t[u] * N * p.d + c;
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) acc[e] = -0.0f;
+                        for (int j = 0; j < N; ++j) {
+                            float acc[8];
 #pragma unroll
-                        for (int i = 0; i < N; ++i)
+                            for (int e = 0; e < 8; ++e) acc[e] = -0.0f;
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) acc[e] = __fmaf_rn(Am[i][j], hv[i][e], acc[e]);
+                            for (int i = 0; i < N; ++i) {
+                                const float aij = Ap[i * N + j];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) acc[e] = __fmaf_rn(bv[j], yv[e], acc[e]);
-                        store_bf16x8(Hot + j * p.d + c, acc);
+                                for (int e = 0; e < 8; ++e) acc[e] = __fmaf_rn(aij, hv[i][e], acc[e]);
+                            }
+                            const float bj = bp[j];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) acc[e] = __fmaf_rn(bj, yv[e], acc[e]);
+                            store_bf16x8_cs(Hot + j * p.d, acc);
+                        }
                     }
                 }
+                __syncwarp();  // the slice is rewritten by the next half / tile
             }
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[buf]);  // this accumulator may be refilled
         }
     }
 
-    // every role has finished with TMEM (the MMA lane drained its MMAs)
+    // every role of both CTAs has finished with TMEM and with the peer's
+    // shared memory (the leader drained its MMAs and the pair's copies)
     tc_fence_before_sync();
-    __syncthreads();
+    cluster_sync_all();
     if (warp == 1) {
         tc_fence_after_sync();
-        tmem_dealloc(tmem, kLwTmemCols);
+        tmem_dealloc_pair(tmem, kLwTmemCols);
     }
 }
 
@@ -296,10 +364,24 @@ hc_status launch_n_lw(const CUtensorMap &mapX, const CUtensorMap &mapW, const Li
                              cudaGetErrorString(e));
         configured[ctx.device] = true;
     }
-    int64_t grid = ctx.sms;
-    if (grid > lp.tiles) grid = lp.tiles;
-    kern<<<(unsigned)grid, kLwThreads, kLwSmem, st>>>(mapX, mapW, lp, ctx.fault);
-    cudaError_t e = cudaGetLastError();
+    // one CTA pair (a cluster of two) per two SMs, at most one pair per tile
+    int64_t pairs = ctx.sms / 2;
+    if (pairs > lp.tiles) pairs = lp.tiles;
+    if (pairs < 1) pairs = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+    cfg.blockDim = dim3(kLwThreads, 1, 1);
+    cfg.dynamicSmemBytes = kLwSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mapX, mapW, lp, ctx.fault);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess)
         return set_error(HC_ERR_CUDA, "hc_linear_write_kernel launch: %s", cudaGetErrorString(e));
     return HC_OK;
@@ -319,19 +401,20 @@ hc_status launch_linear_write(const LinearWriteArgs &a, const LaunchCtx &ctx, cu
     lp.b_s = a.b_s;
     lp.T = a.T;
     lp.d = a.d;
-    const int64_t num_m = (a.T + kLwM - 1) / kLwM;
+    const int64_t num_m = (a.T + kLwTileM - 1) / kLwTileM;
     const int64_t num_n = (a.d + kLwN - 1) / kLwN;
     const int64_t nk = (a.k + kLwK - 1) / kLwK;
-    if (num_m > (int64_t(1) << 31) / kLwM || num_n > INT32_MAX || nk > INT32_MAX)
+    if (num_m > (int64_t(1) << 31) / kLwTileM || num_n > INT32_MAX / kLwN || nk > INT32_MAX / kLwK)
         return set_error(HC_ERR_UNSUPPORTED, "shape too large for the tile grid");
     lp.num_n = (int)num_n;
+    lp.num_m = num_m;
     lp.tiles = num_m * num_n;
     lp.nk = (int)nk;
 
     CUtensorMap mapX, mapW;
     hc_status ms = make_tma_map_bf16(&mapX, a.X, (uint64_t)a.k, (uint64_t)a.T, kLwK, kLwM);
     if (ms != HC_OK) return ms;
-    ms = make_tma_map_bf16(&mapW, a.Wo, (uint64_t)a.k, (uint64_t)a.d, kLwK, kLwN);
+    ms = make_tma_map_bf16(&mapW, a.Wo, (uint64_t)a.k, (uint64_t)a.d, kLwK, kLwBRows);
     if (ms != HC_OK) return ms;
     switch (a.n) {
         case 1: return launch_n_lw<1>(mapX, mapW, lp, ctx, st);
