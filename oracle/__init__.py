@@ -44,6 +44,10 @@ def lib():
             "hco_single_stream_layer": ([vp, vp, i32, i64, i64, vp, fp], i32),
             "hco_expand": ([vp, vp, i32, i64, i32, i64], i32),
             "hco_linear": ([vp, vp, vp, i32, i64, i64, i64], i32),
+            "hco_sinkhorn_backward": ([vp, vp, vp, i64, i32, i32], i32),
+            "hco_write_then_read_backward": ([vp, vp, i32, i64, i32, i64, i32, vp, i64, i32, vp, i64,
+                                              i32, vp, i64, vp, fp, vp, vp, vp, vp, vp, vp, vp, vp],
+                                             i32),
             "hco_collapse": ([vp, vp, i32, i64, i32, i64, i32, vp, i64], i32),
         }
         for name, (args, res) in sig.items():
@@ -212,6 +216,42 @@ def linear(X, W, dt: str):
     y = np.empty((T, d), dtype=np.float64)
     _chk(lib().hco_linear(_p(X), _p(W), _p(y), _DT[dt], T, k, d), "linear")
     return y
+
+
+def sinkhorn_backward(L, dA, K: int):
+    """fp64 gradient w.r.t. the logits L [..., n, n] of the Sinkhorn projection
+    (exp, then K row/column pairs), given the gradient dA w.r.t. its output."""
+    L = _arr(L, np.float32)
+    dA = _arr(dA, np.float64)
+    n = L.shape[-1]
+    T = L.size // (n * n)
+    dL = np.empty(L.shape, dtype=np.float64)
+    _chk(lib().hco_sinkhorn_backward(_p(L), _p(dA), _p(dL), T, n, int(K)), "sinkhorn_backward")
+    return dL
+
+
+def write_then_read_backward(H, y, A, b, a, g, eps: float, dt: str, dHout, dx, K: int = 0,
+                             mix_logits: bool = False, read_logits: bool = False, want_dg=True):
+    """fp64 gradients of the fused step (straight through the storage rounding).
+    dHout [T, n, d] (or None) and dx [T, d] are the upstream gradients. Returns
+    dict(dH, dy, dA, db, da, dg): dA / db / da per token ([T, n, n], [T, n],
+    [T, n]; with mix_logits / read_logits, w.r.t. the logits); dg [d] summed
+    over tokens (None if g is None or not want_dg)."""
+    H = _arr(H, _NP[dt]); y = _arr(y, _NP[dt])
+    T, n, d = H.shape
+    A = _arr(A, np.float32); b = _arr(b, np.float32); a = _arr(a, np.float32)
+    g = None if g is None else _arr(g, np.float32)
+    dHout = None if dHout is None else _arr(dHout, np.float64)
+    dx = _arr(dx, np.float64)
+    out = dict(dH=np.empty((T, n, d)), dy=np.empty((T, d)), dA=np.empty((T, n, n)),
+               db=np.empty((T, n)), da=np.empty((T, n)),
+               dg=np.empty(d) if (g is not None and want_dg) else None)
+    _chk(lib().hco_write_then_read_backward(
+        _p(H), _p(y), _DT[dt], T, n, d, int(mix_logits), _p(A), _tok_stride(A, T, n * n), int(K),
+        _p(b), _tok_stride(b, T, n), int(read_logits), _p(a), _tok_stride(a, T, n), _p(g),
+        float(eps), _p(dHout), _p(dx), _p(out["dH"]), _p(out["dy"]), _p(out["dA"]), _p(out["db"]),
+        _p(out["da"]), _p(out["dg"])), "write_then_read_backward")
+    return out
 
 
 def block_tanh(x, dt: str):

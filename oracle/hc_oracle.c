@@ -413,6 +413,196 @@ int hco_linear(const void *X, const void *W, double *y, int dt, int64_t T, int64
     return HCO_OK;
 }
 
+/*
+ * Backward pass of the fused step (training). The forward is hco_write_then_read;
+ * storage rounding is treated as the identity for gradients (its derivative
+ * almost everywhere), so the gradients are those of the exact-arithmetic step
+ * evaluated at the stored forward values (H' as stored, h as the fp32 chain,
+ * r as rounded to fp32). All backward arithmetic is fp64:
+ *   x_k  = h_k r g_k,  r = (sum h^2 / d + eps)^(-1/2)
+ *   dh_k = r g_k dx_k - (r^3 / d) h_k sum_m g_m dx_m h_m      (RMSNorm)
+ *   dg_k = sum_t dx_k h_k r                                  (over tokens)
+ *   G_j  = dH'_j + a_j dh                                    (into stream j of H')
+ *   dH_i = sum_j A[i][j] G_j,  dy = sum_j b_j G_j
+ *   dA[i][j] = sum_k H_i,k G_j,k,  db_j = sum_k y_k G_j,k,  da_j = sum_k dh_k H'_j,k
+ * then, per token, through the softmax of the read logits
+ *   dl_j = a_j (da_j - sum_m a_m da_m)
+ * and through the Sinkhorn projection: the K (row, column) pairs are re-run
+ * in fp64 keeping every intermediate, then each normalisation M' = M / s is
+ * undone in reverse order with dM = (dM' - sum(dM' * M') over the same row or
+ * column) / s, and finally dL = dM * exp(L).
+ * dHout may be NULL (no gradient arrives at H'); dg may be NULL.
+ */
+static void sinkhorn_backward_f64(const float *L, const double *dA, double *dL, int n, int K,
+                                  double *hist /* (2K+1) n*n */) {
+    const int nn = n * n;
+    for (int e = 0; e < nn; ++e) hist[e] = exp((double)L[e]);
+    for (int p = 0; p < 2 * K; ++p) {
+        const double *in = hist + (int64_t)p * nn;
+        double *out = hist + (int64_t)(p + 1) * nn;
+        for (int q = 0; q < n; ++q) {
+            double s = 0.0;
+            for (int k = 0; k < n; ++k) s += (p % 2 == 0) ? in[q * n + k] : in[k * n + q];
+            for (int k = 0; k < n; ++k) {
+                const int e = (p % 2 == 0) ? q * n + k : k * n + q;
+                out[e] = in[e] / s;
+            }
+        }
+    }
+    double gcur[256], gnext[256];
+    for (int e = 0; e < nn; ++e) gcur[e] = dA[e];
+    for (int p = 2 * K - 1; p >= 0; --p) {
+        const double *in = hist + (int64_t)p * nn;
+        const double *out = hist + (int64_t)(p + 1) * nn;
+        for (int q = 0; q < n; ++q) {
+            double s = 0.0, t = 0.0;
+            for (int k = 0; k < n; ++k) {
+                const int e = (p % 2 == 0) ? q * n + k : k * n + q;
+                s += in[e];
+                t += gcur[e] * out[e];
+            }
+            for (int k = 0; k < n; ++k) {
+                const int e = (p % 2 == 0) ? q * n + k : k * n + q;
+                gnext[e] = (gcur[e] - t) / s;
+            }
+        }
+        for (int e = 0; e < nn; ++e) gcur[e] = gnext[e];
+    }
+    for (int e = 0; e < nn; ++e) dL[e] = gcur[e] * hist[e];
+}
+
+int hco_sinkhorn_backward(const float *L, const double *dA, double *dL, int64_t T, int n, int K) {
+    if (T < 0 || n < 1 || n > 16 || K < 0) return HCO_EINVAL;
+    int err = HCO_OK;
+#pragma omp parallel
+    {
+        double *hist = (double *)malloc(sizeof(double) * (size_t)(2 * K + 1) * (size_t)(n * n));
+        if (!hist) {
+#pragma omp atomic write
+            err = HCO_EINVAL;
+        } else {
+#pragma omp for schedule(static)
+            for (int64_t t = 0; t < T; ++t)
+                sinkhorn_backward_f64(L + t * n * n, dA + t * n * n, dL + t * n * n, n, K, hist);
+        }
+        free(hist);
+    }
+    return err;
+}
+
+int hco_write_then_read_backward(const void *H, const void *y, int dt, int64_t T, int n, int64_t d,
+                                 int mix_logits, const float *A, int64_t A_s, int K, const float *b,
+                                 int64_t b_s, int read_logits, const float *a, int64_t a_s,
+                                 const float *g, float eps, const double *dHout, const double *dx,
+                                 double *dH, double *dy, double *dA, double *db, double *da,
+                                 double *dg) {
+    if (check_common(dt, T, n, d) || !A || !b || !a || !dx || (mix_logits && K < 0) || n > 8)
+        return HCO_EINVAL;
+    int err = HCO_OK;
+    const int nt = omp_get_max_threads();
+    double *dg_part = dg ? (double *)calloc((size_t)nt * (size_t)d, sizeof(double)) : NULL;
+    if (dg && !dg_part) return HCO_EINVAL;
+#pragma omp parallel
+    {
+        const int tid = omp_get_thread_num();
+        float *Hs = (float *)malloc(sizeof(float) * (size_t)n * (size_t)d);
+        float *h = (float *)malloc(sizeof(float) * (size_t)d);
+        double *dh = (double *)malloc(sizeof(double) * (size_t)d);
+        double *hist = (double *)malloc(sizeof(double) * (size_t)(2 * (K > 0 ? K : 0) + 1) * 64);
+        if (!Hs || !h || !dh || !hist) {
+#pragma omp atomic write
+            err = HCO_EINVAL;
+        } else {
+#pragma omp for schedule(static)
+            for (int64_t t = 0; t < T; ++t) {
+                float Am[64], aw[8];
+                const float *At = tok_ptr(A, A_s, t), *bt = tok_ptr(b, b_s, t), *at = tok_ptr(a, a_s, t);
+                if (mix_logits) {
+                    sinkhorn_one_f32(At, Am, n, K);
+                    At = Am;
+                }
+                if (read_logits) {
+                    softmax_one_f32(at, aw, n);
+                    at = aw;
+                }
+                /* forward values as the forward stores / computes them */
+                for (int64_t k = 0; k < d; ++k) {
+                    const float yk = load_s(y, dt, t * d + k);
+                    float hk = -0.0f;
+                    for (int j = 0; j < n; ++j) {
+                        float acc = -0.0f;
+                        for (int i = 0; i < n; ++i)
+                            acc = fmaf(At[i * n + j], load_s(H, dt, (t * n + i) * d + k), acc);
+                        acc = fmaf(bt[j], yk, acc);
+                        Hs[j * d + k] = round_s(dt, acc);
+                        hk = fmaf(at[j], Hs[j * d + k], hk);
+                    }
+                    h[k] = hk;
+                }
+                double ss = 0.0;
+                for (int64_t k = 0; k < d; ++k) ss += (double)h[k] * (double)h[k];
+                const double r = (double)(float)(1.0 / sqrt(ss / (double)d + (double)eps));
+                /* RMSNorm backward */
+                double sg = 0.0;
+                for (int64_t k = 0; k < d; ++k) sg += (g ? (double)g[k] : 1.0) * dx[t * d + k] * (double)h[k];
+                for (int64_t k = 0; k < d; ++k) {
+                    const double gk = g ? (double)g[k] : 1.0;
+                    dh[k] = r * gk * dx[t * d + k] - r * r * r / (double)d * (double)h[k] * sg;
+                    if (dg_part) dg_part[(int64_t)tid * d + k] += dx[t * d + k] * (double)h[k] * r;
+                }
+                /* mixes */
+                double gA[64] = {0}, gb[8] = {0}, ga[8] = {0};
+                for (int64_t k = 0; k < d; ++k) {
+                    double G[8];
+                    const double yk = (double)load_s(y, dt, t * d + k);
+                    for (int j = 0; j < n; ++j) {
+                        G[j] = (dHout ? dHout[(t * n + j) * d + k] : 0.0) + (double)at[j] * dh[k];
+                        gb[j] += yk * G[j];
+                        ga[j] += dh[k] * (double)Hs[j * d + k];
+                    }
+                    double dyk = 0.0;
+                    for (int j = 0; j < n; ++j) dyk += (double)bt[j] * G[j];
+                    dy[t * d + k] = dyk;
+                    for (int i = 0; i < n; ++i) {
+                        const double hik = (double)load_s(H, dt, (t * n + i) * d + k);
+                        double acc = 0.0;
+                        for (int j = 0; j < n; ++j) {
+                            acc += (double)At[i * n + j] * G[j];
+                            gA[i * n + j] += hik * G[j];
+                        }
+                        dH[(t * n + i) * d + k] = acc;
+                    }
+                }
+                for (int j = 0; j < n; ++j) db[t * n + j] = gb[j];
+                if (read_logits) {
+                    double sa = 0.0;
+                    for (int j = 0; j < n; ++j) sa += (double)at[j] * ga[j];
+                    for (int j = 0; j < n; ++j) da[t * n + j] = (double)at[j] * (ga[j] - sa);
+                } else {
+                    for (int j = 0; j < n; ++j) da[t * n + j] = ga[j];
+                }
+                if (mix_logits)
+                    sinkhorn_backward_f64(tok_ptr(A, A_s, t), gA, dA + t * n * n, n, K, hist);
+                else
+                    for (int e = 0; e < n * n; ++e) dA[t * n * n + e] = gA[e];
+            }
+        }
+        free(Hs);
+        free(h);
+        free(dh);
+        free(hist);
+    }
+    if (dg) {
+        for (int64_t k = 0; k < d; ++k) {
+            double acc = 0.0;
+            for (int q = 0; q < nt; ++q) acc += dg_part[(int64_t)q * d + k];
+            dg[k] = acc;
+        }
+        free(dg_part);
+    }
+    return err;
+}
+
 /* Harness block stand-in: y = round_s(tanhf(x)). Not part of the HC step. */
 int hco_block_tanh(const void *x, void *y, int dt, int64_t count) {
     if (dt != HCO_F32 && dt != HCO_BF16) return HCO_EINVAL;

@@ -565,3 +565,129 @@ def test_linear_against_library_matmul_and_closed_forms():
     y1 = oracle.linear(X, gen.to_storage(W1, "bf16"), "bf16")
     assert np.array_equal(y1[:, 0], f32_of(X, "bf16")[:, 3])
     assert np.array_equal(y1[:, 1], -2.0 * f32_of(X, "bf16")[:, k - 1])
+
+
+# --------------------------------------------------------------------------
+# backward pass of the fused step, pinned against torch's automatic
+# differentiation (fp64) of the forward definition and against invariants
+# --------------------------------------------------------------------------
+
+def _torch_step(H, y, A, b, a, g, eps, K, mix_logits, read_logits):
+    """The fused step in torch fp64 (no storage rounding), differentiable."""
+    if mix_logits:
+        M = torch.exp(A)
+        for _ in range(K):
+            M = M / M.sum(dim=-1, keepdim=True)
+            M = M / M.sum(dim=-2, keepdim=True)
+        A = M
+    if read_logits:
+        a = torch.softmax(a, dim=-1)
+    Ab = A if A.dim() == 3 else A.expand(H.shape[0], *A.shape)
+    bb = b if b.dim() == 2 else b.expand(H.shape[0], *b.shape)
+    ab = a if a.dim() == 2 else a.expand(H.shape[0], *a.shape)
+    Hp = torch.einsum("tij,tik->tjk", Ab, H) + bb[:, :, None] * y[:, None, :]
+    h = torch.einsum("tj,tjk->tk", ab, Hp)
+    r = 1.0 / torch.sqrt((h * h).mean(dim=-1, keepdim=True) + eps)
+    return Hp, h * r * g
+
+
+@pytest.mark.parametrize("n,mix,read,per_token", [(4, True, True, True), (4, False, False, False),
+                                                  (2, True, False, True), (1, False, True, True),
+                                                  (8, True, True, True), (3, False, False, True)])
+def test_backward_against_autograd(n, mix, read, per_token):
+    T, d, K, eps = 5, 24, 7, 1e-3
+    H = gen.normal(1101 + n, (T, n, d))
+    y = gen.normal(1102, (T, d))
+    shapeA = (T, n, n) if per_token else (n, n)
+    shape_v = (T, n) if per_token else (n,)
+    A = gen.normal(1103, shapeA, std=0.7 if mix else 0.5)
+    b = gen.normal(1104, shape_v, mean=1.0, std=0.1)
+    a = gen.normal(1105, shape_v, std=0.7 if read else 0.5)
+    g = gen.uniform(1106, (d,), 0.5, 1.5)
+    dHo = gen.normal(1107, (T, n, d))
+    dx = gen.normal(1108, (T, d))
+    got = oracle.write_then_read_backward(H, y, A, b, a, g, eps, "f32", dHo, dx, K=K,
+                                          mix_logits=mix, read_logits=read)
+    tt = {k: torch.tensor(v.astype(np.float64), requires_grad=True)
+          for k, v in dict(H=H, y=y, A=A, b=b, a=a, g=g).items()}
+    Hp, x = _torch_step(tt["H"], tt["y"], tt["A"], tt["b"], tt["a"], tt["g"],
+                        float(np.float32(eps)), K, mix, read)
+    loss = (Hp * torch.from_numpy(dHo.astype(np.float64))).sum() + \
+        (x * torch.from_numpy(dx.astype(np.float64))).sum()
+    loss.backward()
+
+    def close(mine, ref, what, tol=2e-5):
+        ref = ref.detach().numpy()
+        scale = np.max(np.abs(ref)) + 1e-30
+        assert np.max(np.abs(mine - ref)) <= tol * scale, (what, np.max(np.abs(mine - ref)) / scale)
+
+    close(got["dH"], tt["H"].grad, "dH")
+    close(got["dy"], tt["y"].grad, "dy")
+    close(got["dg"], tt["g"].grad, "dg")
+    # per-token parameter gradients; a shared parameter's gradient is their sum
+    for key, name in (("dA", "A"), ("db", "b"), ("da", "a")):
+        mine = got[key] if per_token else got[key].sum(axis=0)
+        close(mine, tt[name].grad, key)
+
+
+def test_backward_invariants():
+    """A row shift of the Sinkhorn logits leaves the projection unchanged, so
+    each row of dL sums to 0; the softmax's shift invariance makes dl sum to 0;
+    with eps = 0, g = 1 and no gradient at H', dh is orthogonal to h."""
+    T, n, d, K = 6, 4, 32, 20
+    H = gen.normal(1111, (T, n, d))
+    y = gen.normal(1112, (T, d))
+    L = gen.normal(1113, (T, n, n))
+    b = gen.normal(1114, (T, n), mean=1.0, std=0.1)
+    l = gen.normal(1115, (T, n))
+    dx = gen.normal(1116, (T, d))
+    out = oracle.write_then_read_backward(H, y, L, b, l, None, 0.0, "f32", None, dx, K=K,
+                                          mix_logits=True, read_logits=True)
+    assert np.max(np.abs(out["dA"].sum(axis=-1))) < 1e-9 * (1 + np.max(np.abs(out["dA"])))
+    assert np.max(np.abs(out["da"].sum(axis=-1))) < 1e-9 * (1 + np.max(np.abs(out["da"])))
+    # standalone Sinkhorn backward equals the one inside the step
+    dA = gen.normal(1117, (T, n, n)).astype(np.float64)
+    dL = oracle.sinkhorn_backward(L, dA, K)
+    assert np.max(np.abs(dL.sum(axis=-1))) < 1e-12 * (1 + np.max(np.abs(dL)))
+    # dh orthogonal to h: through da (= sum_k dh_k H'_j,k) with a one-hot read,
+    # sum_j a_j da_j = sum_k dh_k h_k = 0
+    a1 = np.zeros(n, np.float32)
+    a1[2] = 1.0
+    o2 = oracle.write_then_read_backward(H, y, L, b, a1, None, 0.0, "f32", None, dx, K=K,
+                                         mix_logits=True, read_logits=False)
+    scale = np.max(np.abs(o2["da"]))
+    assert np.max(np.abs(o2["da"][:, 2])) < 1e-6 * scale
+
+
+def test_backward_finite_differences():
+    """Central differences of the oracle's own forward (fp32 storage) in a few
+    random directions agree with the analytic backward."""
+    T, n, d, K, eps = 3, 2, 16, 5, 1e-3
+    H = gen.normal(1121, (T, n, d))
+    y = gen.normal(1122, (T, d))
+    L = gen.normal(1123, (T, n, n))
+    b = gen.normal(1124, (T, n), mean=1.0, std=0.1)
+    l = gen.normal(1125, (T, n))
+    g = gen.uniform(1126, (d,), 0.5, 1.5)
+    dHo = gen.normal(1127, (T, n, d))
+    dx = gen.normal(1128, (T, d))
+    grads = oracle.write_then_read_backward(H, y, L, b, l, g, eps, "f32", dHo, dx, K=K,
+                                            mix_logits=True, read_logits=True)
+
+    def f(H_, y_, L_, l_):
+        Hp, x = oracle.write_then_read(H_.astype(np.float32), y_.astype(np.float32), L_, b,
+                                       l_, g, eps, "f32", K=K, mix_logits=True, read_logits=True)
+        return float(np.sum(Hp.astype(np.float64) * dHo) + np.sum(x.astype(np.float64) * dx))
+
+    rng = np.random.default_rng(3)
+    for name, base, grad in (("H", H, grads["dH"]), ("y", y, grads["dy"]), ("L", L, grads["dA"]),
+                             ("l", l, grads["da"])):
+        v = rng.standard_normal(base.shape)
+        hstep = 1e-2
+        args = dict(H_=H, y_=y, L_=L, l_=l)
+        key = {"H": "H_", "y": "y_", "L": "L_", "l": "l_"}[name]
+        plus = dict(args); plus[key] = (base + hstep * v).astype(np.float32)
+        minus = dict(args); minus[key] = (base - hstep * v).astype(np.float32)
+        fd = (f(**plus) - f(**minus)) / (2 * hstep)
+        an = float(np.sum(grad * v))
+        assert abs(fd - an) <= 2e-3 * (abs(an) + 1.0), (name, fd, an)
