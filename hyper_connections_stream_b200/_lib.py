@@ -40,6 +40,10 @@ SIGNATURES = {
     "hc_selftest_bounded_wait": ([_i32, _vp], _i32),
     "hc_mix_logits": ([_vp, _vp, _vp, _i32, _i64, _i32, _i64, _i32, _f32, _vp], _i32),
     "hc_expand": ([_vp, _vp, _i32, _i64, _i32, _i64, _vp], _i32),
+    "hc_write_then_read_backward": ([_vp, _vp, _i32, _i64, _i32, _i64, _i32, _vp, _i64, _i32, _vp,
+                                     _i64, _i32, _vp, _i64, _vp, _f32, _vp, _vp, _vp, _vp, _vp,
+                                     _vp, _vp, _vp, _vp, C.c_size_t, _vp], _i32),
+    "hc_write_then_read_backward_workspace_bytes": ([_i32, _i64, _i32, _i64], C.c_size_t),
     "hc_linear_then_write": ([_vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i64, _i64, _vp, _i64,
                               _vp, _i64, _vp], _i32),
     "hc_expand_then_read": ([_vp, _vp, _vp, _i32, _i64, _i32, _i64, _i32, _vp, _i64, _vp, _f32,
@@ -337,4 +341,46 @@ def linear_then_write(X, Wo, H, A, b, *, out=None, y_out=None):
         _need_out("y_out", y_out, (T, d), torch.bfloat16)
     _check(lib().hc_linear_then_write(_ptr(X), _ptr(Wo), _ptr(H), _ptr(out), _ptr(y_out), HC_BF16,
                                       T, n, d, k, _ptr(A), A_s, _ptr(b), b_s, _stream(H.device)))
+    return out
+
+
+def write_then_read_backward(H, y, A, b, a, g, dHout, dx, *, eps: float = 1e-6,
+                             mix: int = MIX_MATRIX, K: int = 0, read: int = READ_WEIGHTS,
+                             want_dg: bool = True, workspace=None):
+    """Backward of write_then_read. dHout [T, n, d] (or None) and dx [T, d] are
+    the gradients arriving at H' and x_next. Returns a dict with dH, dy (dtype
+    of H), dA [T, n, n], db [T, n], da [T, n] (fp32, per token; w.r.t. the
+    logits in the Sinkhorn / softmax modes) and dg [d] (summed over tokens, or
+    None). The gain gradient's workspace is allocated here unless given."""
+    _need_cuda("H", H)
+    T, n, d = _streams_shape(H)
+    _need_cuda("y", y, H.dtype)
+    _need_cuda("dx", dx, H.dtype)
+    if tuple(y.shape) != (T, d) or tuple(dx.shape) != (T, d):
+        raise ValueError("y and dx must be [T, d]")
+    if dHout is not None:
+        _need_out("dHout", dHout, (T, n, d), H.dtype)
+    A_s = _tok_param("A", A, T, (n, n))
+    b_s = _tok_param("b", b, T, (n,))
+    a_s = _tok_param("a", a, T, (n,))
+    _need_gain("g", g, d)
+    dev = H.device
+    out = dict(dH=torch.empty_like(H), dy=torch.empty_like(y),
+               dA=torch.empty((T, n, n), dtype=torch.float32, device=dev),
+               db=torch.empty((T, n), dtype=torch.float32, device=dev),
+               da=torch.empty((T, n), dtype=torch.float32, device=dev),
+               dg=torch.empty((d,), dtype=torch.float32, device=dev) if (g is not None and want_dg)
+               else None)
+    ws_bytes = 0
+    if out["dg"] is not None:
+        need = int(lib().hc_write_then_read_backward_workspace_bytes(_DT[H.dtype], T, n, d)) if T else 0
+        if workspace is None:
+            workspace = torch.empty((max(need, 16),), dtype=torch.uint8, device=dev)
+        _need_cuda("workspace", workspace, torch.uint8)
+        ws_bytes = workspace.numel()
+    _check(lib().hc_write_then_read_backward(
+        _ptr(H), _ptr(y), _DT[H.dtype], T, n, d, int(mix), _ptr(A), A_s, int(K), _ptr(b), b_s,
+        int(read), _ptr(a), a_s, _ptr(g), float(eps), _ptr(dHout), _ptr(dx), _ptr(out["dH"]),
+        _ptr(out["dy"]), _ptr(out["dA"]), _ptr(out["db"]), _ptr(out["da"]), _ptr(out["dg"]),
+        _ptr(workspace) if out["dg"] is not None else None, ws_bytes, _stream(dev)))
     return out

@@ -462,4 +462,83 @@ hc_status hc_linear_then_write(const void *X, const void *Wo, const void *H, voi
     return hc::launch_linear_write(la, ctx, static_cast<cudaStream_t>(stream));
 }
 
+size_t hc_write_then_read_backward_workspace_bytes(hc_dtype dt, int64_t T, int n, int64_t d) {
+    if ((dt != HC_F32 && dt != HC_BF16) || T < 1 || n < 1 || n > hc::kMaxStreams || d < 1) return 0;
+    hc::LaunchCtx ctx{};
+    if (launch_ctx(ctx) != HC_OK) return 0;
+    size_t bytes = 0;
+    if (hc::backward_workspace_bytes(n, dt, T, d, ctx, &bytes) != HC_OK) return 0;
+    return bytes;
+}
+
+hc_status hc_write_then_read_backward(const void *H, const void *y, hc_dtype dt, int64_t T, int n,
+                                      int64_t d, hc_mix_mode mm, const float *A, int64_t A_tok_stride,
+                                      int K, const float *b, int64_t b_tok_stride, hc_read_mode rm,
+                                      const float *a, int64_t a_tok_stride, const float *g, float eps,
+                                      const void *dHout, const void *dx, void *dH, void *dy,
+                                      float *dA, float *db, float *da, float *dg, void *workspace,
+                                      size_t workspace_bytes, hc_stream stream) {
+    static const char *fn = "hc_write_then_read_backward";
+    g_last_error[0] = '\0';
+    const Shape s{dt, T, n, d};
+    HC_TRY(check_shape(fn, s, true));
+    if (mm != HC_MIX_MATRIX && mm != HC_MIX_SINKHORN_LOGITS)
+        return fail(HC_ERR_INVALID_ARG, "%s: bad mix mode %d", fn, (int)mm);
+    if (rm != HC_READ_WEIGHTS && rm != HC_READ_SOFTMAX_LOGITS)
+        return fail(HC_ERR_INVALID_ARG, "%s: bad read mode %d", fn, (int)rm);
+    if (mm == HC_MIX_SINKHORN_LOGITS) HC_TRY(check_K(fn, K));
+    HC_TRY(check_stride(fn, "A_tok_stride", A_tok_stride));
+    HC_TRY(check_stride(fn, "b_tok_stride", b_tok_stride));
+    HC_TRY(check_stride(fn, "a_tok_stride", a_tok_stride));
+    HC_TRY(check_eps(fn, eps));
+    if (T == 0) return HC_OK;
+    HC_TRY(check_buf(fn, "H", H));
+    HC_TRY(check_buf(fn, "y", y));
+    HC_TRY(check_buf(fn, "dx", dx));
+    HC_TRY(check_buf(fn, "dH", dH));
+    HC_TRY(check_buf(fn, "dy", dy));
+    if (dHout && !aligned(dHout, 16)) return fail(HC_ERR_MISALIGNED, "%s: dHout is not 16-byte aligned", fn);
+    HC_TRY(check_param(fn, "A", A));
+    HC_TRY(check_param(fn, "b", b));
+    HC_TRY(check_param(fn, "a", a));
+    HC_TRY(check_param(fn, "dA", dA));
+    HC_TRY(check_param(fn, "db", db));
+    HC_TRY(check_param(fn, "da", da));
+    if (g && !aligned(g, 16)) return fail(HC_ERR_MISALIGNED, "%s: g is not 16-byte aligned", fn);
+    if (dg) {
+        if (!g) return fail(HC_ERR_INVALID_ARG, "%s: dg requested without a gain g", fn);
+        if (!aligned(dg, 4)) return fail(HC_ERR_MISALIGNED, "%s: dg is not 4-byte aligned", fn);
+        if (!workspace) return fail(HC_ERR_INVALID_ARG, "%s: dg needs a workspace", fn);
+        if (!aligned(workspace, 16)) return fail(HC_ERR_MISALIGNED, "%s: workspace is not 16-byte aligned", fn);
+    }
+    const int64_t es = elem_bytes(dt);
+    const int64_t hb = T * n * d * es, yb = T * d * es;
+    struct Span { const void *p; int64_t bytes; };
+    const Span ins[] = {{H, hb}, {y, yb}, {dx, yb}, {dHout, dHout ? hb : 0}, {A, 0}, {b, 0}, {a, 0}, {g, 0}};
+    const Span outs[] = {{dH, hb}, {dy, yb}, {dA, T * n * n * 4}, {db, T * n * 4}, {da, T * n * 4},
+                         {dg, dg ? d * 4 : 0}, {workspace, dg ? (int64_t)workspace_bytes : 0}};
+    for (const Span &o : outs) {
+        if (!o.p || o.bytes == 0) continue;
+        for (const Span &i : ins)
+            if (i.p && i.bytes && overlap(o.p, o.bytes, i.p, i.bytes))
+                return fail(HC_ERR_ALIAS, "%s: an output overlaps an input", fn);
+        for (const Span &o2 : outs)
+            if (&o2 != &o && o2.p && o2.bytes && overlap(o.p, o.bytes, o2.p, o2.bytes))
+                return fail(HC_ERR_ALIAS, "%s: two outputs overlap", fn);
+    }
+    hc::LaunchCtx ctx{};
+    HC_TRY(launch_ctx(ctx));
+    hc::BackwardArgs ba{};
+    ba.f.H = H; ba.f.y = y; ba.f.T = T; ba.f.d = d;
+    ba.f.A = A; ba.f.A_s = A_tok_stride; ba.f.b = b; ba.f.b_s = b_tok_stride;
+    ba.f.a = a; ba.f.a_s = a_tok_stride; ba.f.g = g; ba.f.eps = eps;
+    ba.f.K = K; ba.f.mix_logits = mm == HC_MIX_SINKHORN_LOGITS;
+    ba.f.read_logits = rm == HC_READ_SOFTMAX_LOGITS;
+    ba.n = n; ba.dt = dt;
+    ba.dHout = dHout; ba.dx = dx; ba.dH = dH; ba.dy = dy;
+    ba.dA = dA; ba.db = db; ba.da = da; ba.dg = dg;
+    ba.workspace = workspace; ba.workspace_bytes = workspace_bytes;
+    return hc::launch_backward(ba, ctx, static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

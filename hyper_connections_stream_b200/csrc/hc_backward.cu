@@ -1,0 +1,573 @@
+// hc_backward.cu -- backward pass of the fused HC step (training).
+//
+// Gradients of  H'_j = sum_i A[i][j] H_i + b_j y,  h = sum_j a_j H'_j,
+// x = h r g,  r = (sum h^2 / d + eps)^(-1/2)  (the forward of
+// hc_write_then_read; the glossary entry "Hyper-connections (mHC)": learned
+// mixing before and after each block, Sinkhorn-projected in mHC), straight
+// through the storage rounding:
+//   dh = r g dx - (r^3 / d) h sum(g dx h)       G_j = dH'_j + a_j dh
+//   dH_i = sum_j A[i][j] G_j    dy = sum_j b_j G_j    dg = sum_t dx h r
+//   dA[i][j] = sum_k H_i G_j    db_j = sum_k y G_j    da_j = sum_k dh H'_j
+// then per token through the read softmax and the Sinkhorn projection.
+//
+// Kernels:
+//   hc_step_bwd_kernel   one CTA per token at a time (grid-stride), threads own
+//                        column slices. Phase 1 recomputes H' (as stored) and
+//                        h and reduces sum h^2 and sum g dx h (fp64); phase 2
+//                        reloads the token (L2-resident by then), forms dh, G,
+//                        dH, dy and the per-token sums (fp32 per thread, fp64
+//                        across warps); the gain gradient accumulates per CTA
+//                        in shared memory and goes to the workspace at exit.
+//   hc_param_bwd_kernel  lane group per token: the softmax backward, and the
+//                        Sinkhorn backward with the 2K+1 iterates kept in
+//                        shared memory; in place on dA / da.
+//   hc_dg_reduce_kernel  sums the per-CTA gain partials in a fixed order.
+#include "hc_launch.h"
+
+namespace hc {
+
+namespace {
+
+constexpr int kBwTB = 32;       // parameter slots per batch
+constexpr int kBwThreads = 256;  // largest CTA of the step kernel (255 registers a thread)
+
+#define HC_BW_TRY(expr)                 \
+    do {                                \
+        hc_status _st = (expr);         \
+        if (_st != HC_OK) return _st;   \
+    } while (0)
+
+// VE fp32 gains (1 when g is null); k is a multiple of VE.
+template <int VE>
+__device__ __forceinline__ void bw_load_gain(const float *g, int64_t k, float (&gv)[VE]) {
+    if (g == nullptr) {
+#pragma unroll
+        for (int e = 0; e < VE; ++e) gv[e] = 1.0f;
+    } else if constexpr (VE == 2) {
+        const float2 q = __ldg(reinterpret_cast<const float2 *>(g + k));
+        gv[0] = q.x;
+        gv[1] = q.y;
+    } else {
+#pragma unroll
+        for (int e = 0; e < VE; e += 4) {
+            const float4 q = __ldg(reinterpret_cast<const float4 *>(g + k + e));
+            gv[e] = q.x; gv[e + 1] = q.y; gv[e + 2] = q.z; gv[e + 3] = q.w;
+        }
+    }
+}
+
+// VE-element vectors of the storage dtype (16 or 8 bytes), widened to fp32.
+template <typename S, int VE> struct BwVec;
+template <> struct BwVec<float, 4> {
+    static __device__ __forceinline__ void load(const float *p, float (&v)[4]) {
+        const float4 q = __ldcs(reinterpret_cast<const float4 *>(p));
+        v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+    }
+    static __device__ __forceinline__ void store(float *p, const float (&v)[4]) {
+        __stcs(reinterpret_cast<float4 *>(p), make_float4(v[0], v[1], v[2], v[3]));
+    }
+    static __device__ __forceinline__ void round(float (&)[4]) {}
+};
+template <> struct BwVec<float, 2> {
+    static __device__ __forceinline__ void load(const float *p, float (&v)[2]) {
+        const float2 q = __ldcs(reinterpret_cast<const float2 *>(p));
+        v[0] = q.x; v[1] = q.y;
+    }
+    static __device__ __forceinline__ void store(float *p, const float (&v)[2]) {
+        __stcs(reinterpret_cast<float2 *>(p), make_float2(v[0], v[1]));
+    }
+    static __device__ __forceinline__ void round(float (&)[2]) {}
+};
+template <> struct BwVec<__nv_bfloat16, 8> {
+    static __device__ __forceinline__ void load(const __nv_bfloat16 *p, float (&v)[8]) {
+        const uint4 q = __ldcs(reinterpret_cast<const uint4 *>(p));
+        widen_bf16x2(q.x, v[0], v[1]); widen_bf16x2(q.y, v[2], v[3]);
+        widen_bf16x2(q.z, v[4], v[5]); widen_bf16x2(q.w, v[6], v[7]);
+    }
+    static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float (&v)[8]) {
+        uint4 q;
+        q.x = pack_bf16x2_rn(v[0], v[1]); q.y = pack_bf16x2_rn(v[2], v[3]);
+        q.z = pack_bf16x2_rn(v[4], v[5]); q.w = pack_bf16x2_rn(v[6], v[7]);
+        __stcs(reinterpret_cast<uint4 *>(p), q);
+    }
+    static __device__ __forceinline__ void round(float (&v)[8]) {
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) widen_bf16x2(pack_bf16x2_rn(v[e], v[e + 1]), v[e], v[e + 1]);
+    }
+};
+template <> struct BwVec<__nv_bfloat16, 4> {
+    static __device__ __forceinline__ void load(const __nv_bfloat16 *p, float (&v)[4]) {
+        const uint2 q = __ldcs(reinterpret_cast<const uint2 *>(p));
+        widen_bf16x2(q.x, v[0], v[1]); widen_bf16x2(q.y, v[2], v[3]);
+    }
+    static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float (&v)[4]) {
+        uint2 q;
+        q.x = pack_bf16x2_rn(v[0], v[1]); q.y = pack_bf16x2_rn(v[2], v[3]);
+        __stcs(reinterpret_cast<uint2 *>(p), q);
+    }
+    static __device__ __forceinline__ void round(float (&v)[4]) {
+#pragma unroll
+        for (int e = 0; e < 4; e += 2) widen_bf16x2(pack_bf16x2_rn(v[e], v[e + 1]), v[e], v[e + 1]);
+    }
+};
+
+template <typename S> constexpr int bw_vec_elems(int n) {
+    return sizeof(S) == 2 ? (n <= 4 ? 8 : 4) : (n <= 4 ? 4 : 2);
+}
+
+struct BwKernelParams {
+    StepParams f;
+    const void *dHout;
+    const void *dx;
+    void *dH;
+    void *dy;
+    float *gA, *gb, *ga;  // per-token sums (gradients w.r.t. the matrix / weights)
+    float *dg_part;       // [gridDim.x][d] or null
+};
+
+// The forward of one VE-slice: H' as stored (hs) and h, exactly as the
+// forward kernels compute them (fp32 FMA chains in stream order, storage
+// rounding of H').
+template <int N, typename S, int VE>
+__device__ __forceinline__ void bw_forward_slice(const S *Ht, const S *Yt, int64_t d, int64_t k,
+                                                 const float *At, const float *bt, const float *at,
+                                                 float (&hv)[N][VE], float (&yv)[VE],
+                                                 float (&hs)[N][VE], float (&h)[VE]) {
+    using V = BwVec<S, VE>;
+#pragma unroll
+    for (int i = 0; i < N; ++i) V::load(Ht + i * d + k, hv[i]);
+    V::load(Yt + k, yv);
+#pragma unroll
+    for (int e = 0; e < VE; ++e) h[e] = -0.0f;
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+#pragma unroll
+        for (int e = 0; e < VE; ++e) hs[j][e] = -0.0f;
+#pragma unroll
+        for (int i = 0; i < N; ++i)
+#pragma unroll
+            for (int e = 0; e < VE; ++e) hs[j][e] = __fmaf_rn(At[i * N + j], hv[i][e], hs[j][e]);
+#pragma unroll
+        for (int e = 0; e < VE; ++e) hs[j][e] = __fmaf_rn(bt[j], yv[e], hs[j][e]);
+        V::round(hs[j]);
+#pragma unroll
+        for (int e = 0; e < VE; ++e) h[e] = __fmaf_rn(at[j], hs[j][e], h[e]);
+    }
+}
+
+template <int N, typename S, int VE>
+__global__ void __launch_bounds__(kBwThreads)
+hc_step_bwd_kernel(BwKernelParams bp) {
+    const StepParams &p = bp.f;
+    constexpr int NN = N * N;
+    constexpr int NR = NN + 2 * N;  // per-token sums: dA, db, da
+    using V = BwVec<S, VE>;
+    __shared__ float sA[kBwTB * NN], sb[kBwTB * N], sa[kBwTB * N];
+    __shared__ double sred[2][kBwThreads / 32];
+    __shared__ float pred[kBwThreads / 32][NR];
+    __shared__ float swork[kBwThreads / 32 * kGroupScratch];
+    extern __shared__ float sdg[];  // [d]: this CTA's gain-gradient partial
+
+    const int tid = threadIdx.x;
+    const int NT = blockDim.x;
+    const int nwarps = NT >> 5;
+    const int lane = tid & 31, warp = tid >> 5;
+    const int64_t d = p.d;
+    const int64_t nvec = d / VE;
+    const int64_t G = gridDim.x;
+    int TB = nwarps * Group<N>::TPW;
+    TB = TB < kBwTB ? TB : kBwTB;
+
+    const S *H = static_cast<const S *>(p.H);
+    const S *Y = static_cast<const S *>(p.y);
+    const S *DX = static_cast<const S *>(bp.dx);
+    const S *DHO = static_cast<const S *>(bp.dHout);
+    S *DH = static_cast<S *>(bp.dH);
+    S *DY = static_cast<S *>(bp.dy);
+    const bool want_dg = bp.dg_part != nullptr;
+    if (want_dg)
+        for (int64_t k = tid; k < d; k += NT) sdg[k] = 0.0f;
+
+    for (int64_t m0 = 0;; m0 += TB) {
+        const int64_t first = blockIdx.x + m0 * G;
+        if (first >= p.T) break;
+        __syncthreads();  // previous batch's parameters no longer read
+        prepare_params<N, true, true>(p, first, G, TB, sA, sb, sa, swork);
+        __syncthreads();
+        for (int tt = 0; tt < TB; ++tt) {
+            const int64_t t = first + (int64_t)tt * G;
+            if (t >= p.T) break;  // uniform over the CTA
+            const float *At = sA + tt * NN, *bt = sb + tt * N, *at = sa + tt * N;
+            const S *Ht = H + t * N * d, *Yt = Y + t * d, *DXt = DX + t * d;
+
+            // ---- phase 1: the token's statistics ----
+            double ss = 0.0, sg = 0.0;
+            for (int64_t c = tid; c < nvec; c += NT) {
+                const int64_t k = c * VE;
+                float hv[N][VE], yv[VE], hs[N][VE], h[VE], dxv[VE], gv[VE];
+                bw_forward_slice<N, S, VE>(Ht, Yt, d, k, At, bt, at, hv, yv, hs, h);
+                V::load(DXt + k, dxv);
+                bw_load_gain<VE>(p.g, k, gv);
+#pragma unroll
+                for (int e = 0; e < VE; ++e) {
+                    const double he = (double)h[e];
+                    ss = __fma_rn(he, he, ss);
+                    sg = __fma_rn((double)gv[e] * (double)dxv[e], he, sg);
+                }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                sg += __shfl_xor_sync(0xffffffffu, sg, off);
+            }
+            if (lane == 0) {
+                sred[0][warp] = ss;
+                sred[1][warp] = sg;
+            }
+            __syncthreads();
+            double tss = 0.0, tsg = 0.0;
+            for (int w = 0; w < nwarps; ++w) {
+                tss += sred[0][w];
+                tsg += sred[1][w];
+            }
+            const float r = __double2float_rn(1.0 / sqrt(tss / (double)d + (double)p.eps));
+            const double rd = (double)r;
+            const float coef = (float)(rd * rd * rd * tsg / (double)d);
+
+            // ---- phase 2: gradients (the token is re-read from L2) ----
+            float pA[NN], pb[N], pa[N];
+#pragma unroll
+            for (int v = 0; v < NN; ++v) pA[v] = 0.0f;
+#pragma unroll
+            for (int j = 0; j < N; ++j) {
+                pb[j] = 0.0f;
+                pa[j] = 0.0f;
+            }
+            for (int64_t c = tid; c < nvec; c += NT) {
+                const int64_t k = c * VE;
+                float hv[N][VE], yv[VE], hs[N][VE], h[VE], dxv[VE], gv[VE], dh[VE];
+                bw_forward_slice<N, S, VE>(Ht, Yt, d, k, At, bt, at, hv, yv, hs, h);
+                V::load(DXt + k, dxv);
+                bw_load_gain<VE>(p.g, k, gv);
+#pragma unroll
+                for (int e = 0; e < VE; ++e) dh[e] = __fmaf_rn(-coef, h[e], __fmul_rn(__fmul_rn(r, gv[e]), dxv[e]));
+                if (want_dg) {
+#pragma unroll
+                    for (int e = 0; e < VE; ++e) sdg[k + e] = __fmaf_rn(__fmul_rn(dxv[e], h[e]), r, sdg[k + e]);
+                }
+                float dHacc[N][VE], dyacc[VE];
+#pragma unroll
+                for (int e = 0; e < VE; ++e) dyacc[e] = 0.0f;
+#pragma unroll
+                for (int i = 0; i < N; ++i)
+#pragma unroll
+                    for (int e = 0; e < VE; ++e) dHacc[i][e] = 0.0f;
+#pragma unroll
+                for (int j = 0; j < N; ++j) {
+                    float Gj[VE];
+                    if (DHO) {
+                        V::load(DHO + (t * N + j) * d + k, Gj);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < VE; ++e) Gj[e] = 0.0f;
+                    }
+#pragma unroll
+                    for (int e = 0; e < VE; ++e) {
+                        Gj[e] = __fmaf_rn(at[j], dh[e], Gj[e]);
+                        pa[j] = __fmaf_rn(dh[e], hs[j][e], pa[j]);
+                        pb[j] = __fmaf_rn(yv[e], Gj[e], pb[j]);
+                        dyacc[e] = __fmaf_rn(bt[j], Gj[e], dyacc[e]);
+                    }
+#pragma unroll
+                    for (int i = 0; i < N; ++i) {
+                        const float aij = At[i * N + j];
+#pragma unroll
+                        for (int e = 0; e < VE; ++e) {
+                            pA[i * N + j] = __fmaf_rn(hv[i][e], Gj[e], pA[i * N + j]);
+                            dHacc[i][e] = __fmaf_rn(aij, Gj[e], dHacc[i][e]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < N; ++i) V::store(DH + (t * N + i) * d + k, dHacc[i]);
+                V::store(DY + t * d + k, dyacc);
+            }
+            // per-token sums: warp trees (fp32), then the warps in order (fp64)
+#pragma unroll
+            for (int v = 0; v < NR; ++v) {
+                float val = v < NN ? pA[v] : v < NN + N ? pb[v - NN] : pa[v - NN - N];
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) val += __shfl_xor_sync(0xffffffffu, val, off);
+                if (lane == 0) pred[warp][v] = val;
+            }
+            __syncthreads();
+            if (tid < NR) {
+                double acc = 0.0;
+                for (int w = 0; w < nwarps; ++w) acc += (double)pred[w][tid];
+                const float out = (float)acc;
+                if (tid < NN) bp.gA[t * NN + tid] = out;
+                else if (tid < NN + N) bp.gb[t * N + (tid - NN)] = out;
+                else bp.ga[t * N + (tid - NN - N)] = out;
+            }
+        }
+    }
+    if (want_dg) {
+        __syncthreads();
+        for (int64_t k = tid; k < d; k += NT) bp.dg_part[(int64_t)blockIdx.x * d + k] = sdg[k];
+    }
+}
+
+// Per token, in place: da <- softmax backward of da (read logits), dA <- the
+// Sinkhorn backward of dA (mixing logits). Lane groups as in the forward's
+// parameter preparation; the 2K+1 Sinkhorn iterates of every lane live in
+// dynamic shared memory.
+template <int N>
+__global__ void __launch_bounds__(128)
+hc_param_bwd_kernel(const float *L, int64_t L_s, const float *l, int64_t l_s, float *dA, float *da,
+                    int64_t T, int K, int mix, int read) {
+    constexpr int NN = N * N, GL = Group<N>::GL, EPL = Group<N>::EPL, TPW = Group<N>::TPW;
+    extern __shared__ float hist[];  // [(2K+1)][blockDim.x][EPL]
+    __shared__ float sw[4][2 * 64];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int q = lane & (GL - 1);
+    float *buf = sw[warp] + (lane / GL) * NN;       // values of the group's matrix
+    float *buf2 = sw[warp] + 64 + (lane / GL) * NN;  // second exchange buffer
+    const int64_t wg = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    int e[EPL], row[EPL], col[EPL];
+    bool own[EPL];
+#pragma unroll
+    for (int r = 0; r < EPL; ++r) {
+        e[r] = q + GL * r;
+        own[r] = e[r] < NN;
+        const int ec = own[r] ? e[r] : NN - 1;
+        row[r] = ec / N;
+        col[r] = ec - row[r] * N;
+    }
+    for (int64_t t0 = wg * TPW; t0 < T; t0 += nw * TPW) {
+        const int64_t t = t0 + lane / GL;
+        const bool live = t < T;
+        if (mix) {
+            float m[EPL], g[EPL];
+#pragma unroll
+            for (int r = 0; r < EPL; ++r) {
+                m[r] = expf((live && own[r]) ? L[t * L_s + e[r]] : 0.0f);
+                g[r] = (live && own[r]) ? dA[t * NN + e[r]] : 0.0f;
+                hist[((int64_t)0 * blockDim.x + threadIdx.x) * EPL + r] = m[r];
+            }
+            for (int pp = 0; pp < 2 * K; ++pp) {
+#pragma unroll
+                for (int r = 0; r < EPL; ++r)
+                    if (own[r]) buf[e[r]] = m[r];
+                __syncwarp();
+                float s[EPL];
+#pragma unroll
+                for (int r = 0; r < EPL; ++r) {
+                    float acc = 0.0f;
+#pragma unroll
+                    for (int k = 0; k < N; ++k)
+                        acc = __fadd_rn(acc, (pp & 1) == 0 ? buf[row[r] * N + k] : buf[k * N + col[r]]);
+                    s[r] = acc;
+                }
+                __syncwarp();
+#pragma unroll
+                for (int r = 0; r < EPL; ++r) {
+                    m[r] = __fdiv_rn(m[r], s[r]);
+                    hist[((int64_t)(pp + 1) * blockDim.x + threadIdx.x) * EPL + r] = m[r];
+                }
+            }
+            for (int pp = 2 * K - 1; pp >= 0; --pp) {
+                float in[EPL], out[EPL];
+#pragma unroll
+                for (int r = 0; r < EPL; ++r) {
+                    in[r] = hist[((int64_t)pp * blockDim.x + threadIdx.x) * EPL + r];
+                    out[r] = hist[((int64_t)(pp + 1) * blockDim.x + threadIdx.x) * EPL + r];
+                    if (own[r]) {
+                        buf[e[r]] = in[r];
+                        buf2[e[r]] = __fmul_rn(g[r], out[r]);
+                    }
+                }
+                __syncwarp();
+                float s[EPL], u[EPL];
+#pragma unroll
+                for (int r = 0; r < EPL; ++r) {
+                    float as = 0.0f, au = 0.0f;
+#pragma unroll
+                    for (int k = 0; k < N; ++k) {
+                        const int idx = (pp & 1) == 0 ? row[r] * N + k : k * N + col[r];
+                        as = __fadd_rn(as, buf[idx]);
+                        au = __fadd_rn(au, buf2[idx]);
+                    }
+                    s[r] = as;
+                    u[r] = au;
+                }
+                __syncwarp();
+#pragma unroll
+                for (int r = 0; r < EPL; ++r) g[r] = __fdiv_rn(__fsub_rn(g[r], u[r]), s[r]);
+            }
+#pragma unroll
+            for (int r = 0; r < EPL; ++r) {
+                const float m0 = hist[((int64_t)0 * blockDim.x + threadIdx.x) * EPL + r];
+                if (live && own[r]) dA[t * NN + e[r]] = __fmul_rn(g[r], m0);
+            }
+        }
+        if (read) {
+            // a = softmax(l) as the forward computes it, then dl = a (da - sum a da)
+            float lq = (live && q < N) ? l[t * l_s + q] : 0.0f;
+            float gq = (live && q < N) ? da[t * N + q] : 0.0f;
+            const float aq = group_softmax<N>(lq, sw[warp], lane);
+            float *ab = buf2;
+            if (q < N) ab[q] = __fmul_rn(aq, gq);
+            __syncwarp();
+            float tsum = 0.0f;
+#pragma unroll
+            for (int k = 0; k < N; ++k) tsum = __fadd_rn(tsum, ab[k]);
+            __syncwarp();
+            if (live && q < N) da[t * N + q] = __fmul_rn(aq, __fsub_rn(gq, tsum));
+        }
+    }
+}
+
+__global__ void hc_dg_reduce_kernel(const float *part, int rows, int64_t d, float *dg) {
+    for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < d;
+         k += (int64_t)gridDim.x * blockDim.x) {
+        double acc = 0.0;
+        for (int r = 0; r < rows; ++r) acc += (double)part[(int64_t)r * d + k];
+        dg[k] = (float)acc;
+    }
+}
+
+template <int N, typename S>
+struct StepBw {
+    static constexpr int VE = bw_vec_elems<S>(N);
+    static hc_status shape(int64_t d, int &NT) {
+        const int64_t nvec = d / VE;
+        int64_t nt = nvec < kBwThreads ? nvec : kBwThreads;
+        nt = (nt + 31) / 32 * 32;
+        if (nt < 32) nt = 32;
+        NT = (int)nt;
+        return HC_OK;
+    }
+    static hc_status plan(int64_t T, int64_t d, const LaunchCtx &ctx, int &NT, int64_t &grid) {
+        shape(d, NT);
+        auto kern = hc_step_bwd_kernel<N, S, VE>;
+        const size_t dyn = (size_t)d * 4;
+        if (dyn > (size_t)kSmemLimitLogits - 48 * 1024)
+            return set_error(HC_ERR_UNSUPPORTED, "d = %lld too large for the backward", (long long)d);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+        if (e != cudaSuccess) return set_error(HC_ERR_CUDA, "backward smem attribute: %s", cudaGetErrorString(e));
+        int per_sm = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NT, dyn);
+        if (e != cudaSuccess) return set_error(HC_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
+        if (per_sm < 1) per_sm = 1;
+        grid = (int64_t)ctx.sms * per_sm;
+        if (grid > T) grid = T;
+        if (grid < 1) grid = 1;
+        return HC_OK;
+    }
+    static hc_status launch(const BackwardArgs &a, const LaunchCtx &ctx, cudaStream_t st) {
+        // the Sinkhorn backward's iterates must fit shared memory: check before any launch
+        int pthreads = 128;
+        const int Kh = a.f.mix_logits ? a.f.K : 0;
+        size_t hist = (size_t)(2 * Kh + 1) * pthreads * Group<N>::EPL * 4;
+        if (hist > (size_t)kSmemLimitLogits - 4096) {
+            pthreads = 32;
+            hist = (size_t)(2 * Kh + 1) * pthreads * Group<N>::EPL * 4;
+        }
+        if (hist > (size_t)kSmemLimitLogits - 4096)
+            return set_error(HC_ERR_UNSUPPORTED, "K = %d too large for the Sinkhorn backward", a.f.K);
+        int NT = 0;
+        int64_t grid = 0;
+        HC_BW_TRY(plan(a.f.T, a.f.d, ctx, NT, grid));
+        BwKernelParams bp{};
+        bp.f = a.f;
+        bp.dHout = a.dHout;
+        bp.dx = a.dx;
+        bp.dH = a.dH;
+        bp.dy = a.dy;
+        bp.gA = a.dA;
+        bp.gb = a.db;
+        bp.ga = a.da;
+        bp.dg_part = a.dg ? static_cast<float *>(a.workspace) : nullptr;
+        const size_t dyn = a.dg ? (size_t)a.f.d * 4 : 0;
+        hc_step_bwd_kernel<N, S, VE><<<(unsigned)grid, NT, dyn, st>>>(bp);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return set_error(HC_ERR_CUDA, "hc_step_bwd_kernel launch: %s", cudaGetErrorString(e));
+        if (a.f.mix_logits || a.f.read_logits) {
+            auto pk = hc_param_bwd_kernel<N>;
+            e = cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist);
+            if (e != cudaSuccess) return set_error(HC_ERR_CUDA, "param backward smem: %s", cudaGetErrorString(e));
+            const int64_t tok_per_block = (pthreads / 32) * Group<N>::TPW;
+            int64_t pgrid = (a.f.T + tok_per_block - 1) / tok_per_block;
+            if (pgrid > (int64_t)ctx.sms * 16) pgrid = (int64_t)ctx.sms * 16;
+            pk<<<(unsigned)pgrid, pthreads, hist, st>>>(a.f.A, a.f.A_s, a.f.a, a.f.a_s, a.dA, a.da, a.f.T,
+                                                        a.f.K, a.f.mix_logits, a.f.read_logits);
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return set_error(HC_ERR_CUDA, "hc_param_bwd_kernel launch: %s", cudaGetErrorString(e));
+        }
+        if (a.dg) {
+            int64_t rgrid = (a.f.d + 255) / 256;
+            if (rgrid > 4096) rgrid = 4096;
+            hc_dg_reduce_kernel<<<(unsigned)rgrid, 256, 0, st>>>(static_cast<const float *>(a.workspace),
+                                                                (int)grid, a.f.d, a.dg);
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return set_error(HC_ERR_CUDA, "hc_dg_reduce_kernel launch: %s", cudaGetErrorString(e));
+        }
+        return HC_OK;
+    }
+};
+
+template <typename S>
+hc_status dispatch_bw_grid(int n, int64_t T, int64_t d, const LaunchCtx &ctx, int64_t &grid) {
+    int NT = 0;
+    switch (n) {
+        case 1: return StepBw<1, S>::plan(T, d, ctx, NT, grid);
+        case 2: return StepBw<2, S>::plan(T, d, ctx, NT, grid);
+        case 3: return StepBw<3, S>::plan(T, d, ctx, NT, grid);
+        case 4: return StepBw<4, S>::plan(T, d, ctx, NT, grid);
+        case 5: return StepBw<5, S>::plan(T, d, ctx, NT, grid);
+        case 6: return StepBw<6, S>::plan(T, d, ctx, NT, grid);
+        case 7: return StepBw<7, S>::plan(T, d, ctx, NT, grid);
+        default: return StepBw<8, S>::plan(T, d, ctx, NT, grid);
+    }
+}
+
+template <typename S>
+hc_status dispatch_bw(const BackwardArgs &a, const LaunchCtx &ctx, cudaStream_t st) {
+    switch (a.n) {
+        case 1: return StepBw<1, S>::launch(a, ctx, st);
+        case 2: return StepBw<2, S>::launch(a, ctx, st);
+        case 3: return StepBw<3, S>::launch(a, ctx, st);
+        case 4: return StepBw<4, S>::launch(a, ctx, st);
+        case 5: return StepBw<5, S>::launch(a, ctx, st);
+        case 6: return StepBw<6, S>::launch(a, ctx, st);
+        case 7: return StepBw<7, S>::launch(a, ctx, st);
+        default: return StepBw<8, S>::launch(a, ctx, st);
+    }
+}
+
+}  // namespace
+
+hc_status backward_workspace_bytes(int n, hc_dtype dt, int64_t T, int64_t d, const LaunchCtx &ctx,
+                                   size_t *bytes) {
+    int64_t grid = 0;
+    hc_status s = dt == HC_BF16 ? dispatch_bw_grid<__nv_bfloat16>(n, T, d, ctx, grid)
+                                : dispatch_bw_grid<float>(n, T, d, ctx, grid);
+    if (s != HC_OK) return s;
+    *bytes = (size_t)grid * (size_t)d * sizeof(float);
+    return HC_OK;
+}
+
+hc_status launch_backward(const BackwardArgs &a, const LaunchCtx &ctx, cudaStream_t st) {
+    if (a.dg) {
+        size_t need = 0;
+        hc_status s = backward_workspace_bytes(a.n, a.dt, a.f.T, a.f.d, ctx, &need);
+        if (s != HC_OK) return s;
+        if (a.workspace_bytes < need)
+            return set_error(HC_ERR_INVALID_ARG, "workspace of %zu bytes < %zu needed for dg",
+                             a.workspace_bytes, need);
+    }
+    return a.dt == HC_BF16 ? dispatch_bw<__nv_bfloat16>(a, ctx, st) : dispatch_bw<float>(a, ctx, st);
+}
+
+}  // namespace hc

@@ -49,6 +49,24 @@ struct LinearWriteArgs {
 };
 hc_status launch_linear_write(const LinearWriteArgs &a, const LaunchCtx &ctx, cudaStream_t st);
 
+// Backward pass of the fused step (see hc_write_then_read_backward).
+struct BackwardArgs {
+    StepParams f;  // forward inputs: H, y, A, b, a, g, eps, K, modes, T, d
+    int n;
+    hc_dtype dt;
+    const void *dHout;  // [T][n][d] or null
+    const void *dx;     // [T][d]
+    void *dH;           // [T][n][d]
+    void *dy;           // [T][d]
+    float *dA, *db, *da, *dg;
+    void *workspace;
+    size_t workspace_bytes;
+};
+// Workspace the backward needs for the gain gradient on the current device.
+hc_status backward_workspace_bytes(int n, hc_dtype dt, int64_t T, int64_t d, const LaunchCtx &ctx,
+                                   size_t *bytes);
+hc_status launch_backward(const BackwardArgs &a, const LaunchCtx &ctx, cudaStream_t st);
+
 hc_status launch_selftest_wait(int limit_us, const LaunchCtx &ctx, cudaStream_t st);
 
 hc_status launch_sinkhorn(const float *L, float *out, int64_t T, int n, int K,

@@ -162,6 +162,37 @@ HC_API hc_status hc_linear_then_write(const void *X, const void *Wo, const void 
                                       const float *b, int64_t b_tok_stride, hc_stream stream);
 
 /*
+ * Backward pass of hc_write_then_read (training; the forward is the
+ * glossary entry's mixing before and after a block with the mHC Sinkhorn
+ * projection, plus the block's pre-norm). Gradients pass straight through the
+ * storage rounding; every forward input is given again, unchanged.
+ *   dHout [T][n][d] (gradient arriving at H', or NULL for none) and
+ *   dx [T][d] (gradient arriving at x_next), dtype dt.
+ *   dH [T][n][d], dy [T][d] (dtype dt) receive the gradients of H and y.
+ *   dA [T][n][n], db [T][n], da [T][n] (fp32) receive per-token gradients:
+ *   w.r.t. the Sinkhorn logits when mm == HC_MIX_SINKHORN_LOGITS (else the
+ *   matrix) and w.r.t. the read logits when rm == HC_READ_SOFTMAX_LOGITS
+ *   (else the weights). For parameters shared by all tokens (stride 0) the
+ *   gradient is the sum of these over tokens.
+ *   dg [d] (fp32) receives the gain gradient summed over tokens, or pass NULL;
+ *   it needs g and a workspace of hc_write_then_read_backward_workspace_bytes()
+ *   bytes (16-byte aligned; the sum over tokens runs in a fixed order).
+ * Arithmetic: fp32 with fp64 per-token statistics and cross-warp sums. The
+ * Sinkhorn backward keeps the 2K+1 iterates of a token in shared memory
+ * (HC_ERR_UNSUPPORTED when K is too large for that). No output may overlap an
+ * input or another output. Asynchronous; T == 0 is a no-op.
+ */
+HC_API hc_status hc_write_then_read_backward(
+    const void *H, const void *y, hc_dtype dt, int64_t T, int n, int64_t d, hc_mix_mode mm,
+    const float *A, int64_t A_tok_stride, int K, const float *b, int64_t b_tok_stride,
+    hc_read_mode rm, const float *a, int64_t a_tok_stride, const float *g, float eps,
+    const void *dHout, const void *dx, void *dH, void *dy, float *dA, float *db, float *da,
+    float *dg, void *workspace, size_t workspace_bytes, hc_stream stream);
+/* Workspace bytes the backward's gain gradient needs on the current device
+ * (0 on invalid arguments). */
+HC_API size_t hc_write_then_read_backward_workspace_bytes(hc_dtype dt, int64_t T, int n, int64_t d);
+
+/*
  * Ends of a stack ("Tencent open-sources Hy4 Preview at 770B -- Identity
  * Hyper-Connections", learnaivisually: TL;DR and the residual-design table --
  * the n streams start as copies of one; the pages do not say how they are
