@@ -375,6 +375,73 @@ def run_linear_write(args):
     }
 
 
+def run_backward(args):
+    """Backward of the fused mHC step (hc_write_then_read_backward) on the
+    workload: T=16384, n=4, d=7168, bf16, per-token Sinkhorn (K=20) and softmax
+    logits, gradients arriving at both H' and x_next, gain gradient summed over
+    tokens. One step = the three launches (step kernel, parameter backward,
+    gain reduction); device-timed per step."""
+    import numpy as np
+    import torch
+    import hc_inputs as gen
+    from hyper_connections_stream_b200 import _lib as hc
+    ws, rank, local = _dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = dict(WORKLOAD)
+    if args.tokens:
+        w["T"] = args.tokens
+    T, n, d, K = w["T"], w["n"], w["d"], w["K"]
+    cfg = w["cfg"]
+    H = gen.device_normal(gen.SEED_H + cfg, (T, n, d), torch.bfloat16, device)
+    y = gen.device_normal(gen.SEED_Y + cfg, (T, d), torch.bfloat16, device)
+    L = gen.device_normal(gen.SEED_L + cfg, (T, n, n), torch.float32, device)
+    l = gen.device_normal(gen.SEED_L + 100 + cfg, (T, n), torch.float32, device)
+    b = torch.from_numpy(gen.normal(gen.SEED_P + cfg, (n,), mean=1.0, std=0.02)).to(device)
+    g = torch.from_numpy(gen.uniform(3500 + cfg, (d,), 0.5, 1.5)).to(device)
+    dHo = gen.device_normal(5000 + cfg, (T, n, d), torch.bfloat16, device)
+    dx = gen.device_normal(5100 + cfg, (T, d), torch.bfloat16, device)
+    need = int(hc.lib().hc_write_then_read_backward_workspace_bytes(hc.HC_BF16, T, n, d))
+    work = torch.empty((max(need, 16),), dtype=torch.uint8, device=device)
+
+    def step():
+        return hc.write_then_read_backward(H, y, L, b, l, g, dHo, dx, eps=w["eps"],
+                                           mix=hc.MIX_SINKHORN_LOGITS, K=K,
+                                           read=hc.READ_SOFTMAX_LOGITS, workspace=work)
+
+    stream = torch.cuda.current_stream(device)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    step_ms = statistics.mean(s_.elapsed_time(e) for s_, e in ev)
+    total_ms = ev[0][0].elapsed_time(ev[-1][1])
+    s = 2
+    alg_bytes = (T * d * s * (3 * n + 3) + T * 4 * (n * n + n) + T * 4 * (n * n + 2 * n)
+                 + d * 4 * 2)
+    peak, peak_kind = _peaks()
+    achieved = alg_bytes / (step_ms / 1e3) / 1e9
+    return {
+        "metric": "HC step backward tokens/sec at n=4, d=7168 (bf16, mHC K=20)",
+        "value": T * args.steps / (total_ms / 1e3), "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "backward", "T": T, "n": n, "d": d, "K": K,
+                   "l2": "inputs and outputs > L2; the binding allocates the gradient outputs"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "peak_source": peak_kind,
+                     "algorithmic_bytes_per_step": alg_bytes, "step_ms": step_ms},
+        "gpu_launches": 3 * args.steps, "device_fault": hc.device_fault(),
+    }
+
+
 def run_ours(args):
     import torch
     from hyper_connections_stream_b200 import _lib as hc
@@ -619,12 +686,13 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-only", action="store_true",
                     help="device-timed kernel only (no e2e, no CPU baseline): for profiling")
-    ap.add_argument("--op", choices=["step", "logits", "expand_read", "collapse", "linear_write"],
+    ap.add_argument("--op", choices=["step", "logits", "expand_read", "collapse", "linear_write",
+                                     "backward"],
                     default="step",
                     help="step: the fused HC step (the metric); logits: the tensor-core "
                          "mixing-logits kernel on the same streams; expand_read / collapse: "
                          "the stack ends on the same shape; linear_write: the block's output "
-                         "projection fused with the write")
+                         "projection fused with the write; backward: the step's backward pass")
     ap.add_argument("--path", choices=["auto", "pipelined", "register"], default="auto",
                     help="kernel family (auto = pipelined wherever it applies)")
     ap.add_argument("--tokens", type=int, default=0,
@@ -644,6 +712,8 @@ def main(argv=None):
         line = run_ends(args)
     elif args.op == "linear_write":
         line = run_linear_write(args)
+    elif args.op == "backward":
+        line = run_backward(args)
     else:
         line = run_ours(args)
     if line is not None:

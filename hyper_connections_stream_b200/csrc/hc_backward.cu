@@ -78,23 +78,6 @@ template <> struct BwVec<float, 2> {
     }
     static __device__ __forceinline__ void round(float (&)[2]) {}
 };
-template <> struct BwVec<__nv_bfloat16, 8> {
-    static __device__ __forceinline__ void load(const __nv_bfloat16 *p, float (&v)[8]) {
-        const uint4 q = __ldcs(reinterpret_cast<const uint4 *>(p));
-        widen_bf16x2(q.x, v[0], v[1]); widen_bf16x2(q.y, v[2], v[3]);
-        widen_bf16x2(q.z, v[4], v[5]); widen_bf16x2(q.w, v[6], v[7]);
-    }
-    static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float (&v)[8]) {
-        uint4 q;
-        q.x = pack_bf16x2_rn(v[0], v[1]); q.y = pack_bf16x2_rn(v[2], v[3]);
-        q.z = pack_bf16x2_rn(v[4], v[5]); q.w = pack_bf16x2_rn(v[6], v[7]);
-        __stcs(reinterpret_cast<uint4 *>(p), q);
-    }
-    static __device__ __forceinline__ void round(float (&v)[8]) {
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) widen_bf16x2(pack_bf16x2_rn(v[e], v[e + 1]), v[e], v[e + 1]);
-    }
-};
 template <> struct BwVec<__nv_bfloat16, 4> {
     static __device__ __forceinline__ void load(const __nv_bfloat16 *p, float (&v)[4]) {
         const uint2 q = __ldcs(reinterpret_cast<const uint2 *>(p));
@@ -111,8 +94,10 @@ template <> struct BwVec<__nv_bfloat16, 4> {
     }
 };
 
+// 8-byte vectors for bf16 (16 bytes would double the per-slice registers and
+// halve the CTAs per SM); 16-byte fp32 vectors up to n = 4.
 template <typename S> constexpr int bw_vec_elems(int n) {
-    return sizeof(S) == 2 ? (n <= 4 ? 8 : 4) : (n <= 4 ? 4 : 2);
+    return sizeof(S) == 2 ? 4 : (n <= 4 ? 4 : 2);
 }
 
 struct BwKernelParams {
@@ -155,8 +140,26 @@ __device__ __forceinline__ void bw_forward_slice(const S *Ht, const S *Yt, int64
     }
 }
 
+// Stream j of H' as the forward stores it, from the loaded H and y slices.
 template <int N, typename S, int VE>
-__global__ void __launch_bounds__(kBwThreads)
+__device__ __forceinline__ void bw_stream_out(const float (&hv)[N][VE], const float (&yv)[VE],
+                                              const float *At, const float *bt, int j,
+                                              float (&hs)[VE]) {
+#pragma unroll
+    for (int e = 0; e < VE; ++e) hs[e] = -0.0f;
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+#pragma unroll
+        for (int e = 0; e < VE; ++e) hs[e] = __fmaf_rn(At[i * N + j], hv[i][e], hs[e]);
+#pragma unroll
+    for (int e = 0; e < VE; ++e) hs[e] = __fmaf_rn(bt[j], yv[e], hs[e]);
+    BwVec<S, VE>::round(hs);
+}
+
+// Two CTAs per SM (128 registers a thread) up to n = 5; the n*n per-thread
+// sums of larger n need the full register file.
+template <int N, typename S, int VE>
+__global__ void __launch_bounds__(kBwThreads, (N <= 5 ? 2 : 1))
 hc_step_bwd_kernel(BwKernelParams bp) {
     const StepParams &p = bp.f;
     constexpr int NN = N * N;
@@ -245,15 +248,32 @@ hc_step_bwd_kernel(BwKernelParams bp) {
             }
             for (int64_t c = tid; c < nvec; c += NT) {
                 const int64_t k = c * VE;
-                float hv[N][VE], yv[VE], hs[N][VE], h[VE], dxv[VE], gv[VE], dh[VE];
-                bw_forward_slice<N, S, VE>(Ht, Yt, d, k, At, bt, at, hv, yv, hs, h);
-                V::load(DXt + k, dxv);
-                bw_load_gain<VE>(p.g, k, gv);
+                float hv[N][VE], yv[VE], h[VE], dh[VE];
 #pragma unroll
-                for (int e = 0; e < VE; ++e) dh[e] = __fmaf_rn(-coef, h[e], __fmul_rn(__fmul_rn(r, gv[e]), dxv[e]));
-                if (want_dg) {
+                for (int i = 0; i < N; ++i) V::load(Ht + i * d + k, hv[i]);
+                V::load(Yt + k, yv);
+                // h from the stored H' (each stream rebuilt on the fly)
 #pragma unroll
-                    for (int e = 0; e < VE; ++e) sdg[k + e] = __fmaf_rn(__fmul_rn(dxv[e], h[e]), r, sdg[k + e]);
+                for (int e = 0; e < VE; ++e) h[e] = -0.0f;
+#pragma unroll
+                for (int j = 0; j < N; ++j) {
+                    float hs[VE];
+                    bw_stream_out<N, S, VE>(hv, yv, At, bt, j, hs);
+#pragma unroll
+                    for (int e = 0; e < VE; ++e) h[e] = __fmaf_rn(at[j], hs[e], h[e]);
+                }
+                {
+                    float dxv[VE], gv[VE];
+                    V::load(DXt + k, dxv);
+                    bw_load_gain<VE>(p.g, k, gv);
+#pragma unroll
+                    for (int e = 0; e < VE; ++e)
+                        dh[e] = __fmaf_rn(-coef, h[e], __fmul_rn(__fmul_rn(r, gv[e]), dxv[e]));
+                    if (want_dg) {
+#pragma unroll
+                        for (int e = 0; e < VE; ++e)
+                            sdg[k + e] = __fmaf_rn(__fmul_rn(dxv[e], h[e]), r, sdg[k + e]);
+                    }
                 }
                 float dHacc[N][VE], dyacc[VE];
 #pragma unroll
@@ -264,7 +284,8 @@ hc_step_bwd_kernel(BwKernelParams bp) {
                     for (int e = 0; e < VE; ++e) dHacc[i][e] = 0.0f;
 #pragma unroll
                 for (int j = 0; j < N; ++j) {
-                    float Gj[VE];
+                    float hs[VE], Gj[VE];
+                    bw_stream_out<N, S, VE>(hv, yv, At, bt, j, hs);
                     if (DHO) {
                         V::load(DHO + (t * N + j) * d + k, Gj);
                     } else {
@@ -274,7 +295,7 @@ hc_step_bwd_kernel(BwKernelParams bp) {
 #pragma unroll
                     for (int e = 0; e < VE; ++e) {
                         Gj[e] = __fmaf_rn(at[j], dh[e], Gj[e]);
-                        pa[j] = __fmaf_rn(dh[e], hs[j][e], pa[j]);
+                        pa[j] = __fmaf_rn(dh[e], hs[e], pa[j]);
                         pb[j] = __fmaf_rn(yv[e], Gj[e], pb[j]);
                         dyacc[e] = __fmaf_rn(bt[j], Gj[e], dyacc[e]);
                     }
