@@ -44,6 +44,9 @@ SIGNATURES = {
                                      _i64, _i32, _vp, _i64, _vp, _f32, _vp, _vp, _vp, _vp, _vp,
                                      _vp, _vp, _vp, _vp, C.c_size_t, _vp], _i32),
     "hc_write_then_read_backward_workspace_bytes": ([_i32, _i64, _i32, _i64], C.c_size_t),
+    "hc_write_then_read_backward_noalloc": ([_vp, _vp, _i32, _i64, _i32, _i64, _i32, _vp, _i64, _i32,
+                                             _vp, _i64, _i32, _vp, _i64, _vp, _f32, _vp, _vp, _vp,
+                                             _vp, _vp, _vp, _vp, _vp, _vp], _i32),
     "hc_linear_then_write": ([_vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i64, _i64, _vp, _i64,
                               _vp, _i64, _vp], _i32),
     "hc_expand_then_read": ([_vp, _vp, _vp, _i32, _i64, _i32, _i64, _i32, _vp, _i64, _vp, _f32,
@@ -383,4 +386,45 @@ def write_then_read_backward(H, y, A, b, a, g, dHout, dx, *, eps: float = 1e-6,
         int(read), _ptr(a), a_s, _ptr(g), float(eps), _ptr(dHout), _ptr(dx), _ptr(out["dH"]),
         _ptr(out["dy"]), _ptr(out["dA"]), _ptr(out["db"]), _ptr(out["da"]), _ptr(out["dg"]),
         _ptr(workspace) if out["dg"] is not None else None, ws_bytes, _stream(dev)))
+    return out
+
+
+def write_then_read_backward_noalloc(H, y, A, b, a, g, dHout, dx, *, eps: float = 1e-6,
+                                     mix: int = MIX_MATRIX, K: int = 0, read: int = READ_WEIGHTS,
+                                     out=None):
+    """write_then_read_backward through hc_write_then_read_backward_noalloc
+    (the gain gradient's scratch is the library's static device array). out,
+    if given, is a dict of preallocated outputs as write_then_read_backward
+    returns them."""
+    _need_cuda("H", H)
+    T, n, d = _streams_shape(H)
+    _need_cuda("y", y, H.dtype)
+    _need_cuda("dx", dx, H.dtype)
+    if tuple(y.shape) != (T, d) or tuple(dx.shape) != (T, d):
+        raise ValueError("y and dx must be [T, d]")
+    if dHout is not None:
+        _need_out("dHout", dHout, (T, n, d), H.dtype)
+    A_s = _tok_param("A", A, T, (n, n))
+    b_s = _tok_param("b", b, T, (n,))
+    a_s = _tok_param("a", a, T, (n,))
+    _need_gain("g", g, d)
+    dev = H.device
+    if out is None:
+        out = dict(dH=torch.empty_like(H), dy=torch.empty_like(y),
+                   dA=torch.empty((T, n, n), dtype=torch.float32, device=dev),
+                   db=torch.empty((T, n), dtype=torch.float32, device=dev),
+                   da=torch.empty((T, n), dtype=torch.float32, device=dev),
+                   dg=torch.empty((d,), dtype=torch.float32, device=dev) if g is not None else None)
+    _need_out("dH", out["dH"], (T, n, d), H.dtype)
+    _need_out("dy", out["dy"], (T, d), H.dtype)
+    _need_out("dA", out["dA"], (T, n, n), torch.float32)
+    _need_out("db", out["db"], (T, n), torch.float32)
+    _need_out("da", out["da"], (T, n), torch.float32)
+    if out["dg"] is not None:
+        _need_out("dg", out["dg"], (d,), torch.float32)
+    _check(lib().hc_write_then_read_backward_noalloc(
+        _ptr(H), _ptr(y), _DT[H.dtype], T, n, d, int(mix), _ptr(A), A_s, int(K), _ptr(b), b_s,
+        int(read), _ptr(a), a_s, _ptr(g), float(eps), _ptr(dHout), _ptr(dx), _ptr(out["dH"]),
+        _ptr(out["dy"]), _ptr(out["dA"]), _ptr(out["db"]), _ptr(out["da"]), _ptr(out["dg"]),
+        _stream(dev)))
     return out

@@ -193,6 +193,30 @@ HC_API hc_status hc_write_then_read_backward(
 HC_API size_t hc_write_then_read_backward_workspace_bytes(hc_dtype dt, int64_t T, int n, int64_t d);
 
 /*
+ * hc_write_then_read_backward without a workspace argument: the pages have no
+ * counterpart to this; it is an interface convenience of this library. The
+ * gain gradient's per-CTA partials go to a 16 MiB scratch array that lives in
+ * the library's device image (one per device); the call allocates nothing.
+ * Arguments and results are those of hc_write_then_read_backward.
+ *   - Calls needing more than 16 MiB of partials (more SMs x d x 4 bytes)
+ *     return HC_ERR_UNSUPPORTED without launching anything.
+ *   - The scratch is shared by every call on a device: two calls whose
+ *     executions overlap (different streams without ordering between them)
+ *     race on it and corrupt dg. Order such calls, or use the workspace form.
+ *   - The first call on a device (with dg) looks the scratch address up on
+ *     the host (cudaGetSymbolAddress) and sets kernel attributes; make one
+ *     call before capturing work into a graph if that setup must not happen
+ *     during capture.
+ *   - No part of the scratch has to start at zero.
+ */
+HC_API hc_status hc_write_then_read_backward_noalloc(
+    const void *H, const void *y, hc_dtype dt, int64_t T, int n, int64_t d, hc_mix_mode mm,
+    const float *A, int64_t A_tok_stride, int K, const float *b, int64_t b_tok_stride,
+    hc_read_mode rm, const float *a, int64_t a_tok_stride, const float *g, float eps,
+    const void *dHout, const void *dx, void *dH, void *dy, float *dA, float *db, float *da,
+    float *dg, hc_stream stream);
+
+/*
  * Ends of a stack ("Tencent open-sources Hy4 Preview at 770B -- Identity
  * Hyper-Connections", learnaivisually: TL;DR and the residual-design table --
  * the n streams start as copies of one; the pages do not say how they are
