@@ -67,6 +67,13 @@ template <> struct BwVec<float, 4> {
         __stcs(reinterpret_cast<float4 *>(p), make_float4(v[0], v[1], v[2], v[3]));
     }
     static __device__ __forceinline__ void round(float (&)[4]) {}
+    static __device__ __forceinline__ void store_smem(float *p, const float (&v)[4]) {
+        *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    }
+    static __device__ __forceinline__ void load_smem(const float *p, float (&v)[4]) {
+        const float4 q = *reinterpret_cast<const float4 *>(p);
+        v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+    }
 };
 template <> struct BwVec<float, 2> {
     static __device__ __forceinline__ void load(const float *p, float (&v)[2]) {
@@ -77,6 +84,13 @@ template <> struct BwVec<float, 2> {
         __stcs(reinterpret_cast<float2 *>(p), make_float2(v[0], v[1]));
     }
     static __device__ __forceinline__ void round(float (&)[2]) {}
+    static __device__ __forceinline__ void store_smem(float *p, const float (&v)[2]) {
+        *reinterpret_cast<float2 *>(p) = make_float2(v[0], v[1]);
+    }
+    static __device__ __forceinline__ void load_smem(const float *p, float (&v)[2]) {
+        const float2 q = *reinterpret_cast<const float2 *>(p);
+        v[0] = q.x; v[1] = q.y;
+    }
 };
 template <> struct BwVec<__nv_bfloat16, 4> {
     static __device__ __forceinline__ void load(const __nv_bfloat16 *p, float (&v)[4]) {
@@ -91,6 +105,16 @@ template <> struct BwVec<__nv_bfloat16, 4> {
     static __device__ __forceinline__ void round(float (&v)[4]) {
 #pragma unroll
         for (int e = 0; e < 4; e += 2) widen_bf16x2(pack_bf16x2_rn(v[e], v[e + 1]), v[e], v[e + 1]);
+    }
+    // shared-memory copies of values already rounded to bf16 (exact)
+    static __device__ __forceinline__ void store_smem(__nv_bfloat16 *p, const float (&v)[4]) {
+        uint2 q;
+        q.x = pack_bf16x2_rn(v[0], v[1]); q.y = pack_bf16x2_rn(v[2], v[3]);
+        *reinterpret_cast<uint2 *>(p) = q;
+    }
+    static __device__ __forceinline__ void load_smem(const __nv_bfloat16 *p, float (&v)[4]) {
+        const uint2 q = *reinterpret_cast<const uint2 *>(p);
+        widen_bf16x2(q.x, v[0], v[1]); widen_bf16x2(q.y, v[2], v[3]);
     }
 };
 
@@ -122,21 +146,30 @@ __device__ __forceinline__ void bw_forward_slice(const S *Ht, const S *Yt, int64
 #pragma unroll
     for (int i = 0; i < N; ++i) V::load(Ht + i * d + k, hv[i]);
     V::load(Yt + k, yv);
+    // paired fp32 FMAs: each element's chain is the scalar one, bit for bit
 #pragma unroll
     for (int e = 0; e < VE; ++e) h[e] = -0.0f;
 #pragma unroll
     for (int j = 0; j < N; ++j) {
 #pragma unroll
-        for (int e = 0; e < VE; ++e) hs[j][e] = -0.0f;
+        for (int e = 0; e < VE; e += 2) {
+            float2 acc = make_float2(-0.0f, -0.0f);
 #pragma unroll
-        for (int i = 0; i < N; ++i)
-#pragma unroll
-            for (int e = 0; e < VE; ++e) hs[j][e] = __fmaf_rn(At[i * N + j], hv[i][e], hs[j][e]);
-#pragma unroll
-        for (int e = 0; e < VE; ++e) hs[j][e] = __fmaf_rn(bt[j], yv[e], hs[j][e]);
+            for (int i = 0; i < N; ++i)
+                acc = ffma2_rn(make_float2(At[i * N + j], At[i * N + j]),
+                               make_float2(hv[i][e], hv[i][e + 1]), acc);
+            acc = ffma2_rn(make_float2(bt[j], bt[j]), make_float2(yv[e], yv[e + 1]), acc);
+            hs[j][e] = acc.x;
+            hs[j][e + 1] = acc.y;
+        }
         V::round(hs[j]);
 #pragma unroll
-        for (int e = 0; e < VE; ++e) h[e] = __fmaf_rn(at[j], hs[j][e], h[e]);
+        for (int e = 0; e < VE; e += 2) {
+            const float2 hh = ffma2_rn(make_float2(at[j], at[j]), make_float2(hs[j][e], hs[j][e + 1]),
+                                       make_float2(h[e], h[e + 1]));
+            h[e] = hh.x;
+            h[e + 1] = hh.y;
+        }
     }
 }
 
@@ -158,7 +191,9 @@ __device__ __forceinline__ void bw_stream_out(const float (&hv)[N][VE], const fl
 
 // Two CTAs per SM (128 registers a thread) up to n = 5; the n*n per-thread
 // sums of larger n need the full register file.
-template <int N, typename S, int VE>
+// STAGE: phase 1 parks the token's H' (as stored, bf16) in shared memory and
+// phase 2 reads it back instead of rebuilding it (bf16 storage, when it fits).
+template <int N, typename S, int VE, bool STAGE>
 __global__ void __launch_bounds__(kBwThreads, (N <= 5 ? 2 : 1))
 hc_step_bwd_kernel(BwKernelParams bp) {
     const StepParams &p = bp.f;
@@ -169,7 +204,7 @@ hc_step_bwd_kernel(BwKernelParams bp) {
     __shared__ double sred[2][kBwThreads / 32];
     __shared__ float pred[kBwThreads / 32][NR];
     __shared__ float swork[kBwThreads / 32 * kGroupScratch];
-    extern __shared__ float sdg[];  // [d]: this CTA's gain-gradient partial
+    extern __shared__ __align__(16) unsigned char bw_dyn[];
 
     const int tid = threadIdx.x;
     const int NT = blockDim.x;
@@ -188,6 +223,8 @@ hc_step_bwd_kernel(BwKernelParams bp) {
     S *DH = static_cast<S *>(bp.dH);
     S *DY = static_cast<S *>(bp.dy);
     const bool want_dg = bp.dg_part != nullptr;
+    float *sdg = reinterpret_cast<float *>(bw_dyn);  // [d]: this CTA's gain-gradient partial
+    S *shs = reinterpret_cast<S *>(bw_dyn + (want_dg ? d * 4 : 0));  // [N][d] stored H' (STAGE)
     if (want_dg)
         for (int64_t k = tid; k < d; k += NT) sdg[k] = 0.0f;
 
@@ -209,6 +246,10 @@ hc_step_bwd_kernel(BwKernelParams bp) {
                 const int64_t k = c * VE;
                 float hv[N][VE], yv[VE], hs[N][VE], h[VE], dxv[VE], gv[VE];
                 bw_forward_slice<N, S, VE>(Ht, Yt, d, k, At, bt, at, hv, yv, hs, h);
+                if constexpr (STAGE) {
+#pragma unroll
+                    for (int j = 0; j < N; ++j) V::store_smem(shs + j * d + k, hs[j]);
+                }
                 V::load(DXt + k, dxv);
                 bw_load_gain<VE>(p.g, k, gv);
 #pragma unroll
@@ -238,13 +279,15 @@ hc_step_bwd_kernel(BwKernelParams bp) {
             const float coef = (float)(rd * rd * rd * tsg / (double)d);
 
             // ---- phase 2: gradients (the token is re-read from L2) ----
-            float pA[NN], pb[N], pa[N];
+            // per-thread partial sums, two lanes of a pair each (added at the end)
+            float pA[NN];
+            float2 pb2[N], pa2[N];
 #pragma unroll
             for (int v = 0; v < NN; ++v) pA[v] = 0.0f;
 #pragma unroll
             for (int j = 0; j < N; ++j) {
-                pb[j] = 0.0f;
-                pa[j] = 0.0f;
+                pb2[j] = make_float2(0.0f, 0.0f);
+                pa2[j] = make_float2(0.0f, 0.0f);
             }
             for (int64_t c = tid; c < nvec; c += NT) {
                 const int64_t k = c * VE;
@@ -252,13 +295,20 @@ hc_step_bwd_kernel(BwKernelParams bp) {
 #pragma unroll
                 for (int i = 0; i < N; ++i) V::load(Ht + i * d + k, hv[i]);
                 V::load(Yt + k, yv);
-                // h from the stored H' (each stream rebuilt on the fly)
+                // h from the stored H' (parked in phase 1, or each stream rebuilt)
+                float hsk[STAGE ? N : 1][VE];
 #pragma unroll
                 for (int e = 0; e < VE; ++e) h[e] = -0.0f;
 #pragma unroll
                 for (int j = 0; j < N; ++j) {
                     float hs[VE];
-                    bw_stream_out<N, S, VE>(hv, yv, At, bt, j, hs);
+                    if constexpr (STAGE) {
+                        V::load_smem(shs + j * d + k, hsk[j]);
+#pragma unroll
+                        for (int e = 0; e < VE; ++e) hs[e] = hsk[j][e];
+                    } else {
+                        bw_stream_out<N, S, VE>(hv, yv, At, bt, j, hs);
+                    }
 #pragma unroll
                     for (int e = 0; e < VE; ++e) h[e] = __fmaf_rn(at[j], hs[e], h[e]);
                 }
@@ -285,7 +335,12 @@ hc_step_bwd_kernel(BwKernelParams bp) {
 #pragma unroll
                 for (int j = 0; j < N; ++j) {
                     float hs[VE], Gj[VE];
-                    bw_stream_out<N, S, VE>(hv, yv, At, bt, j, hs);
+                    if constexpr (STAGE) {
+#pragma unroll
+                        for (int e = 0; e < VE; ++e) hs[e] = hsk[j][e];
+                    } else {
+                        bw_stream_out<N, S, VE>(hv, yv, At, bt, j, hs);
+                    }
                     if (DHO) {
                         V::load(DHO + (t * N + j) * d + k, Gj);
                     } else {
@@ -293,19 +348,27 @@ hc_step_bwd_kernel(BwKernelParams bp) {
                         for (int e = 0; e < VE; ++e) Gj[e] = 0.0f;
                     }
 #pragma unroll
-                    for (int e = 0; e < VE; ++e) {
-                        Gj[e] = __fmaf_rn(at[j], dh[e], Gj[e]);
-                        pa[j] = __fmaf_rn(dh[e], hs[e], pa[j]);
-                        pb[j] = __fmaf_rn(yv[e], Gj[e], pb[j]);
-                        dyacc[e] = __fmaf_rn(bt[j], Gj[e], dyacc[e]);
-                    }
+                    for (int e = 0; e < VE; e += 2) {
+                        const float2 dh2 = make_float2(dh[e], dh[e + 1]);
+                        const float2 G2 = ffma2_rn(make_float2(at[j], at[j]), dh2,
+                                                   make_float2(Gj[e], Gj[e + 1]));
+                        Gj[e] = G2.x;
+                        Gj[e + 1] = G2.y;
+                        pa2[j] = ffma2_rn(dh2, make_float2(hs[e], hs[e + 1]), pa2[j]);
+                        pb2[j] = ffma2_rn(make_float2(yv[e], yv[e + 1]), G2, pb2[j]);
+                        const float2 dy2 = ffma2_rn(make_float2(bt[j], bt[j]), G2,
+                                                    make_float2(dyacc[e], dyacc[e + 1]));
+                        dyacc[e] = dy2.x;
+                        dyacc[e + 1] = dy2.y;
 #pragma unroll
-                    for (int i = 0; i < N; ++i) {
-                        const float aij = At[i * N + j];
-#pragma unroll
-                        for (int e = 0; e < VE; ++e) {
-                            pA[i * N + j] = __fmaf_rn(hv[i][e], Gj[e], pA[i * N + j]);
-                            dHacc[i][e] = __fmaf_rn(aij, Gj[e], dHacc[i][e]);
+                        for (int i = 0; i < N; ++i) {
+                            const float aij = At[i * N + j];
+                            pA[i * N + j] = __fmaf_rn(hv[i][e + 1], G2.y,
+                                                      __fmaf_rn(hv[i][e], G2.x, pA[i * N + j]));
+                            const float2 dH2 = ffma2_rn(make_float2(aij, aij), G2,
+                                                        make_float2(dHacc[i][e], dHacc[i][e + 1]));
+                            dHacc[i][e] = dH2.x;
+                            dHacc[i][e + 1] = dH2.y;
                         }
                     }
                 }
@@ -316,7 +379,13 @@ hc_step_bwd_kernel(BwKernelParams bp) {
             // per-token sums: warp trees (fp32), then the warps in order (fp64)
 #pragma unroll
             for (int v = 0; v < NR; ++v) {
-                float val = v < NN ? pA[v] : v < NN + N ? pb[v - NN] : pa[v - NN - N];
+                float val;
+                if (v < NN) {
+                    val = pA[v];
+                } else {
+                    const float2 pv = v < NN + N ? pb2[v - NN] : pa2[v - NN - N];
+                    val = __fadd_rn(pv.x, pv.y);
+                }
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) val += __shfl_xor_sync(0xffffffffu, val, off);
                 if (lane == 0) pred[warp][v] = val;
@@ -461,6 +530,14 @@ __global__ void hc_dg_reduce_kernel(const float *part, int rows, int64_t d, floa
 template <int N, typename S>
 struct StepBw {
     static constexpr int VE = bw_vec_elems<S>(N);
+    // Shared-memory budget of the dynamic part: two CTAs per SM up to n = 5.
+    static constexpr size_t kDynBudget = N <= 5 ? 96 * 1024 : 176 * 1024;
+    static bool stage(int64_t d, bool want_dg) {
+        return sizeof(S) == 2 && (size_t)N * d * 2 + (want_dg ? (size_t)d * 4 : 0) <= kDynBudget;
+    }
+    static size_t dyn_bytes(int64_t d, bool want_dg) {
+        return (want_dg ? (size_t)d * 4 : 0) + (stage(d, want_dg) ? (size_t)N * d * 2 : 0);
+    }
     static hc_status shape(int64_t d, int &NT) {
         const int64_t nvec = d / VE;
         int64_t nt = nvec < kBwThreads ? nvec : kBwThreads;
@@ -469,17 +546,24 @@ struct StepBw {
         NT = (int)nt;
         return HC_OK;
     }
-    static hc_status plan(int64_t T, int64_t d, const LaunchCtx &ctx, int &NT, int64_t &grid) {
-        shape(d, NT);
-        auto kern = hc_step_bwd_kernel<N, S, VE>;
-        const size_t dyn = (size_t)d * 4;
-        if (dyn > (size_t)kSmemLimitLogits - 48 * 1024)
-            return set_error(HC_ERR_UNSUPPORTED, "d = %lld too large for the backward", (long long)d);
+    template <bool ST>
+    static hc_status occupancy(int NT, size_t dyn, int &per_sm) {
+        auto kern = hc_step_bwd_kernel<N, S, VE, ST>;
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
         if (e != cudaSuccess) return set_error(HC_ERR_CUDA, "backward smem attribute: %s", cudaGetErrorString(e));
-        int per_sm = 0;
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NT, dyn);
         if (e != cudaSuccess) return set_error(HC_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
+        return HC_OK;
+    }
+    // Launch shape; the grid is what the gain-gradient workspace is sized by.
+    static hc_status plan(int64_t T, int64_t d, bool want_dg, const LaunchCtx &ctx, int &NT,
+                          int64_t &grid) {
+        shape(d, NT);
+        const size_t dyn = dyn_bytes(d, want_dg);
+        if (dyn > (size_t)kSmemLimitLogits - 48 * 1024)
+            return set_error(HC_ERR_UNSUPPORTED, "d = %lld too large for the backward", (long long)d);
+        int per_sm = 0;
+        HC_BW_TRY(stage(d, want_dg) ? occupancy<true>(NT, dyn, per_sm) : occupancy<false>(NT, dyn, per_sm));
         if (per_sm < 1) per_sm = 1;
         grid = (int64_t)ctx.sms * per_sm;
         if (grid > T) grid = T;
@@ -497,9 +581,10 @@ struct StepBw {
         }
         if (hist > (size_t)kSmemLimitLogits - 4096)
             return set_error(HC_ERR_UNSUPPORTED, "K = %d too large for the Sinkhorn backward", a.f.K);
+        const bool want_dg = a.dg != nullptr;
         int NT = 0;
         int64_t grid = 0;
-        HC_BW_TRY(plan(a.f.T, a.f.d, ctx, NT, grid));
+        HC_BW_TRY(plan(a.f.T, a.f.d, want_dg, ctx, NT, grid));
         BwKernelParams bp{};
         bp.f = a.f;
         bp.dHout = a.dHout;
@@ -509,9 +594,12 @@ struct StepBw {
         bp.gA = a.dA;
         bp.gb = a.db;
         bp.ga = a.da;
-        bp.dg_part = a.dg ? static_cast<float *>(a.workspace) : nullptr;
-        const size_t dyn = a.dg ? (size_t)a.f.d * 4 : 0;
-        hc_step_bwd_kernel<N, S, VE><<<(unsigned)grid, NT, dyn, st>>>(bp);
+        bp.dg_part = want_dg ? static_cast<float *>(a.workspace) : nullptr;
+        const size_t dyn = dyn_bytes(a.f.d, want_dg);
+        if (stage(a.f.d, want_dg))
+            hc_step_bwd_kernel<N, S, VE, true><<<(unsigned)grid, NT, dyn, st>>>(bp);
+        else
+            hc_step_bwd_kernel<N, S, VE, false><<<(unsigned)grid, NT, dyn, st>>>(bp);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return set_error(HC_ERR_CUDA, "hc_step_bwd_kernel launch: %s", cudaGetErrorString(e));
         if (a.f.mix_logits || a.f.read_logits) {
@@ -542,14 +630,14 @@ template <typename S>
 hc_status dispatch_bw_grid(int n, int64_t T, int64_t d, const LaunchCtx &ctx, int64_t &grid) {
     int NT = 0;
     switch (n) {
-        case 1: return StepBw<1, S>::plan(T, d, ctx, NT, grid);
-        case 2: return StepBw<2, S>::plan(T, d, ctx, NT, grid);
-        case 3: return StepBw<3, S>::plan(T, d, ctx, NT, grid);
-        case 4: return StepBw<4, S>::plan(T, d, ctx, NT, grid);
-        case 5: return StepBw<5, S>::plan(T, d, ctx, NT, grid);
-        case 6: return StepBw<6, S>::plan(T, d, ctx, NT, grid);
-        case 7: return StepBw<7, S>::plan(T, d, ctx, NT, grid);
-        default: return StepBw<8, S>::plan(T, d, ctx, NT, grid);
+        case 1: return StepBw<1, S>::plan(T, d, true, ctx, NT, grid);
+        case 2: return StepBw<2, S>::plan(T, d, true, ctx, NT, grid);
+        case 3: return StepBw<3, S>::plan(T, d, true, ctx, NT, grid);
+        case 4: return StepBw<4, S>::plan(T, d, true, ctx, NT, grid);
+        case 5: return StepBw<5, S>::plan(T, d, true, ctx, NT, grid);
+        case 6: return StepBw<6, S>::plan(T, d, true, ctx, NT, grid);
+        case 7: return StepBw<7, S>::plan(T, d, true, ctx, NT, grid);
+        default: return StepBw<8, S>::plan(T, d, true, ctx, NT, grid);
     }
 }
 
