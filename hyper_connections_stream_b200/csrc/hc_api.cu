@@ -59,13 +59,15 @@ int vec_elems(hc_dtype dt) { return dt == HC_BF16 ? 8 : 4; }
 // Per-device launch context: SM count and the address of this device's fault
 // word (looked up once per device, with that device current).
 hc_status launch_ctx(hc::LaunchCtx &ctx) {
-    static int sms_cache[64] = {};
-    static int *fault_cache[64] = {};
+    // published with release/acquire: the SM count is stored last and read first
+    static std::atomic<int> sms_cache[64];
+    static std::atomic<int *> fault_cache[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return fail(HC_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
     if (dev < 0 || dev >= 64) return fail(HC_ERR_UNSUPPORTED, "device ordinal %d >= 64", dev);
-    if (sms_cache[dev] == 0) {
+    int sms_known = sms_cache[dev].load(std::memory_order_acquire);
+    if (sms_known == 0) {
         int sms = 0;
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess)
@@ -74,12 +76,13 @@ hc_status launch_ctx(hc::LaunchCtx &ctx) {
         e = cudaGetSymbolAddress(&addr, g_hc_device_fault);
         if (e != cudaSuccess)
             return fail(HC_ERR_CUDA, "cudaGetSymbolAddress(fault word): %s", cudaGetErrorString(e));
-        fault_cache[dev] = static_cast<int *>(addr);
-        sms_cache[dev] = sms;
+        fault_cache[dev].store(static_cast<int *>(addr), std::memory_order_relaxed);
+        sms_cache[dev].store(sms, std::memory_order_release);
+        sms_known = sms;
     }
     ctx.device = dev;
-    ctx.sms = sms_cache[dev];
-    ctx.fault = fault_cache[dev];
+    ctx.sms = sms_known;
+    ctx.fault = fault_cache[dev].load(std::memory_order_relaxed);
     ctx.path = hc::g_path.load(std::memory_order_relaxed);
     return HC_OK;
 }

@@ -10,6 +10,8 @@
 //     calls, and can be forced.
 #pragma once
 
+#include <atomic>
+
 #include "hc_launch.h"
 #include "hc_pipe_kernels.cuh"
 #include "hc_stream_kernels.cuh"
@@ -110,15 +112,15 @@ template <int N, typename S, int KIND>
 hc_status launch_pipe(const StepParams &p, const PipeShape &sh, int smem, const LaunchCtx &ctx,
                       cudaStream_t st) {
     auto kern = hc_pipe_kernel<N, S, KIND>;
-    static int configured[64] = {};  // largest dynamic smem opted in so far, per device
+    static std::atomic<int> configured[64];  // largest dynamic smem opted in so far, per device
     if (ctx.device < 0 || ctx.device >= 64)
         return set_error(HC_ERR_UNSUPPORTED, "device ordinal %d >= 64", ctx.device);
-    if (smem > configured[ctx.device]) {
+    if (smem > configured[ctx.device].load()) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess)
             return set_error(HC_ERR_CUDA, "cudaFuncSetAttribute(%d B smem): %s", smem,
                              cudaGetErrorString(e));
-        configured[ctx.device] = smem;
+        configured[ctx.device].store(smem);
     }
     int64_t grid = ctx.sms;
     if (grid > p.T) grid = p.T;

@@ -32,6 +32,8 @@
 // and MMAs and leaves through the closing cluster barrier.
 #include <cuda.h>
 
+#include <atomic>
+
 #include "hc_launch.h"
 #include "hc_tc.cuh"
 
@@ -354,15 +356,15 @@ template <int N>
 hc_status launch_n_lw(const CUtensorMap &mapX, const CUtensorMap &mapW, const LinearWriteParams &lp,
                       const LaunchCtx &ctx, cudaStream_t st) {
     auto kern = hc_linear_write_kernel<N>;
-    static bool configured[64] = {};
+    static std::atomic<bool> configured[64];
     if (ctx.device < 0 || ctx.device >= 64)
         return set_error(HC_ERR_UNSUPPORTED, "device ordinal %d >= 64", ctx.device);
-    if (!configured[ctx.device]) {
+    if (!configured[ctx.device].load()) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kLwSmem);
         if (e != cudaSuccess)
             return set_error(HC_ERR_CUDA, "cudaFuncSetAttribute(%d B smem): %s", kLwSmem,
                              cudaGetErrorString(e));
-        configured[ctx.device] = true;
+        configured[ctx.device].store(true);
     }
     // one CTA pair (a cluster of two) per two SMs, at most one pair per tile
     int64_t pairs = ctx.sms / 2;

@@ -20,6 +20,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
+
 #include "hc_launch.h"
 #include "hc_tc.cuh"
 
@@ -304,16 +306,16 @@ hc_status launch_mix_logits(const void *H, const void *W, float *z, int64_t T, i
     ms = make_tma_map_bf16(&mapW, W, (uint64_t)lp.K, (uint64_t)P, kLgKSub, (uint32_t)lp.Npad);
     if (ms != HC_OK) return ms;
 
-    static int configured[64] = {};
+    static std::atomic<int> configured[64];  // largest dynamic smem opted in so far, per device
     if (ctx.device < 0 || ctx.device >= 64)
         return set_error(HC_ERR_UNSUPPORTED, "device ordinal %d >= 64", ctx.device);
-    if (smem > configured[ctx.device]) {
+    if (smem > configured[ctx.device].load()) {
         cudaError_t e = cudaFuncSetAttribute(hc_logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              smem);
         if (e != cudaSuccess)
             return set_error(HC_ERR_CUDA, "cudaFuncSetAttribute(%d B smem): %s", smem,
                              cudaGetErrorString(e));
-        configured[ctx.device] = smem;
+        configured[ctx.device].store(smem);
     }
     const int64_t grid = (T + lp.rows - 1) / lp.rows;
     hc_logits_kernel<<<(unsigned)grid, kLgThreads, smem, st>>>(mapH, mapW, lp, ctx.fault);
