@@ -48,9 +48,28 @@ def _peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def _source_hash():
+# Kernel sources each profiled traffic record depends on (the record is
+# dropped as soon as one of them changes).
+KERNEL_SOURCES = {
+    "fused_mhc_n4_d7168_bf16_T16384": ["hc_pipe_kernels.cuh", "hc_device.cuh", "hc_sync.cuh",
+                                       "hc_kernels_impl.cuh", "hc_k_bf16_fused.cu"],
+    "mix_logits_n4_d7168_bf16_T16384": ["hc_logits.cu", "hc_tc.cuh", "hc_sync.cuh"],
+    "collapse_n4_d7168_bf16_T16384": ["hc_stream_kernels.cuh", "hc_device.cuh",
+                                      "hc_kernels_impl.cuh", "hc_k_bf16_ends.cu"],
+    "expand_read_n4_d7168_bf16_T16384": ["hc_stream_kernels.cuh", "hc_device.cuh",
+                                         "hc_kernels_impl.cuh", "hc_k_bf16_ends.cu"],
+    "linear_write_n4_d7168_k7168_bf16_T16384": ["hc_linear_write.cu", "hc_tc.cuh", "hc_sync.cuh"],
+    "backward_mhc_n4_d7168_bf16_T16384": ["hc_backward.cu", "hc_device.cuh", "hc_sync.cuh"],
+}
+
+
+def _source_hash(files=None):
+    """Hash of the named kernel sources (all of csrc/ when files is None)."""
+    csrc = os.path.join(ROOT, "hyper_connections_stream_b200", "csrc")
+    paths = (sorted(glob.glob(os.path.join(csrc, "*"))) if files is None
+             else [os.path.join(csrc, f) for f in sorted(files)])
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "hyper_connections_stream_b200", "csrc", "*"))):
+    for f in paths:
         with open(f, "rb") as fh:
             h.update(os.path.basename(f).encode())
             h.update(fh.read())
@@ -58,7 +77,7 @@ def _source_hash():
 
 
 def _profiled_traffic(kernel_key: str):
-    """ncu DRAM bytes per launch committed under profiles/, if the kernel
+    """ncu DRAM bytes per launch committed under profiles/, if the kernel's
     sources have not changed since the capture."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
@@ -66,7 +85,7 @@ def _profiled_traffic(kernel_key: str):
             entry = json.load(f)[kernel_key]
     except Exception:
         return None
-    if entry.get("source_sha") != _source_hash():
+    if entry.get("source_sha") != _source_hash(KERNEL_SOURCES.get(kernel_key)):
         return None
     return entry.get("dram_bytes_per_launch")
 
@@ -365,7 +384,10 @@ def run_linear_write(args):
         "config": {"workload": "linear_write", "T": T, "n": n, "d": d, "k": k,
                    "mix": "per-token Sinkhorn-projected A (K=20)", "l2": "inputs and outputs > L2"},
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
-                     "frac": tflops / peak, "traffic": None, "peak_source": peak_kind,
+                     "frac": tflops / peak,
+                     "traffic": _profiled_traffic("linear_write_n4_d7168_k7168_bf16_T16384")
+                     if T == 16384 else None,
+                     "peak_source": peak_kind,
                      "flops_per_launch": flops, "kernel_ms": kern_ms,
                      "hbm_bytes_min": hbm_bytes,
                      "hbm_gbs_at_min_bytes": hbm_bytes / (kern_ms / 1e3) / 1e9},
@@ -436,7 +458,10 @@ def run_backward(args):
         "config": {"workload": "backward", "T": T, "n": n, "d": d, "K": K,
                    "l2": "inputs and outputs > L2; the binding allocates the gradient outputs"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None, "peak_source": peak_kind,
+                     "frac": achieved / peak,
+                     "traffic": _profiled_traffic("backward_mhc_n4_d7168_bf16_T16384")
+                     if T == 16384 else None,
+                     "peak_source": peak_kind,
                      "algorithmic_bytes_per_step": alg_bytes, "step_ms": step_ms},
         "gpu_launches": 3 * args.steps, "device_fault": hc.device_fault(),
     }

@@ -518,12 +518,28 @@ hc_param_bwd_kernel(const float *L, int64_t L_s, const float *l, int64_t l_s, fl
     }
 }
 
-__global__ void hc_dg_reduce_kernel(const float *part, int rows, int64_t d, float *dg) {
-    for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < d;
-         k += (int64_t)gridDim.x * blockDim.x) {
+// Block of 256 threads = 32 columns x 8 row slices: slice q sums rows
+// q, q + 8, ... of its column in fp64, then the 8 partials are added in slice
+// order. The order is fixed by the launch shape, so dg is reproducible.
+constexpr int kDgCols = 32, kDgSlices = 8;
+__global__ void __launch_bounds__(kDgCols * kDgSlices)
+hc_dg_reduce_kernel(const float *part, int rows, int64_t d, float *dg) {
+    __shared__ double acc_s[kDgSlices][kDgCols];
+    const int col = threadIdx.x % kDgCols, q = threadIdx.x / kDgCols;
+    for (int64_t k0 = (int64_t)blockIdx.x * kDgCols; k0 < d; k0 += (int64_t)gridDim.x * kDgCols) {
+        const int64_t k = k0 + col;
         double acc = 0.0;
-        for (int r = 0; r < rows; ++r) acc += (double)part[(int64_t)r * d + k];
-        dg[k] = (float)acc;
+        if (k < d)
+            for (int r = q; r < rows; r += kDgSlices) acc += (double)part[(int64_t)r * d + k];
+        acc_s[q][col] = acc;
+        __syncthreads();
+        if (q == 0 && k < d) {
+            double tot = 0.0;
+#pragma unroll
+            for (int j = 0; j < kDgSlices; ++j) tot += acc_s[j][col];
+            dg[k] = (float)tot;
+        }
+        __syncthreads();
     }
 }
 
@@ -615,9 +631,9 @@ struct StepBw {
             if (e != cudaSuccess) return set_error(HC_ERR_CUDA, "hc_param_bwd_kernel launch: %s", cudaGetErrorString(e));
         }
         if (a.dg) {
-            int64_t rgrid = (a.f.d + 255) / 256;
+            int64_t rgrid = (a.f.d + kDgCols - 1) / kDgCols;
             if (rgrid > 4096) rgrid = 4096;
-            hc_dg_reduce_kernel<<<(unsigned)rgrid, 256, 0, st>>>(static_cast<const float *>(a.workspace),
+            hc_dg_reduce_kernel<<<(unsigned)rgrid, kDgCols * kDgSlices, 0, st>>>(static_cast<const float *>(a.workspace),
                                                                 (int)grid, a.f.d, a.dg);
             e = cudaGetLastError();
             if (e != cudaSuccess) return set_error(HC_ERR_CUDA, "hc_dg_reduce_kernel launch: %s", cudaGetErrorString(e));
