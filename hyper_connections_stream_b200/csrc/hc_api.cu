@@ -217,8 +217,9 @@ hc_status hc_mix_logits(const void *H, const void *W, float *logits, hc_dtype dt
     if (P < 1) return fail(HC_ERR_INVALID_ARG, "%s: P = %d < 1", fn, P);
     if (P > 256) return fail(HC_ERR_UNSUPPORTED, "%s: P = %d > 256", fn, P);
     HC_TRY(check_eps(fn, eps));
-    if (T > (int64_t)0x7fffffff || (int64_t)n * d > (int64_t)0x7fffffff)
-        return fail(HC_ERR_UNSUPPORTED, "%s: T or n*d beyond 2^31", fn);
+    // TMA coordinates are 32-bit and run up to one tile past the end
+    if (T > (int64_t)0x7fffff00 || (int64_t)n * d > (int64_t)0x7fffff00)
+        return fail(HC_ERR_UNSUPPORTED, "%s: T or n*d beyond 2^31 - 256", fn);
     if (T == 0) return HC_OK;
     HC_TRY(check_buf(fn, "H", H));
     HC_TRY(check_buf(fn, "W", W));
@@ -437,8 +438,10 @@ hc_status hc_linear_then_write(const void *X, const void *Wo, const void *H, voi
     if (k % 8 != 0)
         return fail(HC_ERR_UNSUPPORTED, "%s: k = %lld is not a multiple of 8 (16-byte rows)", fn,
                     (long long)k);
-    if (k > (int64_t(1) << 31) || d > (int64_t(1) << 31) || T > (int64_t(1) << 31))
-        return fail(HC_ERR_UNSUPPORTED, "%s: T, d and k must each be below 2^31", fn);
+    // TMA coordinates are 32-bit and run up to one tile past the end
+    const int64_t lim = (int64_t)0x7fffff00;
+    if (k > lim || d > lim || T > lim)
+        return fail(HC_ERR_UNSUPPORTED, "%s: T, d and k must each be below 2^31 - 256", fn);
     HC_TRY(check_stride(fn, "A_tok_stride", A_tok_stride));
     HC_TRY(check_stride(fn, "b_tok_stride", b_tok_stride));
     if (T == 0) return HC_OK;
