@@ -52,6 +52,7 @@
 #ifndef HC_API_H
 #define HC_API_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #if defined(__GNUC__)

@@ -181,3 +181,16 @@ def test_binding_refuses_cpu_tensors():
     H = torch.zeros((2, 4, 16), dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         _lib.read_rmsnorm(H, torch.ones(4))
+
+
+def test_public_header_compiles_standalone_as_c_and_cpp(tmp_path):
+    """include/hc_api.h is a C ABI: it must compile on its own (no CUDA headers)
+    as C99 and as C++."""
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "hc_api.h"\nint main(void) { return hc_version() < 0; }\n')
+    inc = os.path.join(ROOT, "include")
+    for cmd in (["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror"],
+                ["g++", "-std=c++17", "-Wall", "-Wextra", "-Werror", "-x", "c++"]):
+        out = subprocess.run([*cmd, "-I", inc, "-c", str(src), "-o", str(tmp_path / "o.o")],
+                             capture_output=True, text=True)
+        assert out.returncode == 0, (cmd[0], out.stderr)
