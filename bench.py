@@ -26,6 +26,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -106,8 +107,9 @@ class ClockSampler:
 
     def __enter__(self):
         try:
-            os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-            self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+            # the raw samples go to a temporary file; the JSON line carries the summary
+            fd, self.path = tempfile.mkstemp(prefix="hc_clocks_", suffix=".csv")
+            os.close(fd)
             cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                    "-lms", "100"]
             if self.uuid:
@@ -142,6 +144,10 @@ class ClockSampler:
                     rows.append((float(parts[0]), float(parts[1]), parts[4:8]))
                 except ValueError:
                     continue
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
         if not rows:
             return None
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
