@@ -491,6 +491,10 @@ def run_ours(args):
     w = dict(WORKLOAD)
     if args.tokens:
         w["T"] = args.tokens
+    if args.streams:
+        w["n"] = args.streams
+    if args.width:
+        w["d"] = args.width
     T, n, d, K = w["T"], w["n"], w["d"], w["K"]
     inp = make_inputs(w, rank, device)
     H0 = inp["H"]
@@ -543,7 +547,8 @@ def run_ours(args):
                                    per_token_read=True)
     peak, peak_kind = _peaks()
     achieved = alg_bytes / (kern_ms / 1e3) / 1e9
-    prof = _profiled_traffic("fused_mhc_n4_d7168_bf16_T16384")
+    prof = (_profiled_traffic("fused_mhc_n4_d7168_bf16_T16384")
+            if (T, n, d) == (WORKLOAD["T"], WORKLOAD["n"], WORKLOAD["d"]) else None)
 
     # end to end through the public API with host buffers
     e2e = None if args.kernel_only else run_e2e(args, inp, w, device, ws)
@@ -554,7 +559,9 @@ def run_ours(args):
     if rank != 0:
         return None
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "metric": METRIC if (n, d) == (WORKLOAD["n"], WORKLOAD["d"])
+        else f"HC step tokens/sec at n={n}, d={d} (bf16; sweep case)",
+        "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w["name"], "T": T, "n": n, "d": d, "K": K, "storage": "bf16",
@@ -728,6 +735,10 @@ def main(argv=None):
                     help="kernel family (auto = pipelined wherever it applies)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override T (smaller cases for ncu captures)")
+    ap.add_argument("--streams", type=int, default=0,
+                    help="override n for --op step (sweep cases; the metric's workload is n=4)")
+    ap.add_argument("--width", type=int, default=0,
+                    help="override d for --op step (sweep cases; the metric's workload is d=7168)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
