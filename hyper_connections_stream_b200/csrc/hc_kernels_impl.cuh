@@ -88,7 +88,7 @@ bool pipe_shape(const StepParams &p, PipeShape &sh, int &smem) {
     constexpr int V = pipe_vec_elems<N, S>();
     constexpr int ROWS = KIND != KIND_READ ? N + 1 : N;
     const int64_t d_h = KIND != KIND_WRITE ? p.d : 0;
-    sh.tile = kPipeGroupThreads * V;
+    sh.tile = pipe_group_warps(N) * 32 * V;
     const int64_t ntile = (p.d + sh.tile - 1) / sh.tile;
     if (ntile > (1 << 20)) return false;
     sh.ntile = (int)ntile;
@@ -124,7 +124,7 @@ hc_status launch_pipe(const StepParams &p, const PipeShape &sh, int smem, const 
     }
     int64_t grid = ctx.sms;
     if (grid > p.T) grid = p.T;
-    kern<<<(unsigned)grid, kPipeThreads, smem, st>>>(p, sh, ctx.fault);
+    kern<<<(unsigned)grid, pipe_threads(N), smem, st>>>(p, sh, ctx.fault);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(HC_ERR_CUDA, "hc_pipe_kernel launch: %s", cudaGetErrorString(e));
     return HC_OK;

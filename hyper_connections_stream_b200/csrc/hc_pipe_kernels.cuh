@@ -8,7 +8,7 @@
 //               completing on the stage's "full" mbarrier;
 //   warp 1      parameters: lane groups compute the per-token Sinkhorn
 //               projection / read softmax ahead of use into parameter slots;
-//   warps 2..   consumer groups (kPipeGroups x kPipeGroupWarps warps); group
+//   warps 2..   consumer groups (kPipeGroups x pipe_group_warps(n) warps); group
 //               r owns tokens r, r + kPipeGroups, ... of the CTA, reads the
 //               stages, writes H' with coalesced 128-bit stores, keeps h in an
 //               fp32 shared-memory row, reduces the fp64 sum of squares across
@@ -37,6 +37,9 @@ namespace hc {
 #ifndef HC_PIPE_GROUP_WARPS
 #define HC_PIPE_GROUP_WARPS 7
 #endif
+#ifndef HC_PIPE_GROUP_WARPS_WIDE
+#define HC_PIPE_GROUP_WARPS_WIDE 5
+#endif
 #ifndef HC_PIPE_L2_HINT
 #define HC_PIPE_L2_HINT 0
 #endif
@@ -54,9 +57,15 @@ namespace hc {
 #define HC_PIPE_SG_READ 16
 #endif
 constexpr int kPipeGroups = HC_PIPE_GROUPS;
-constexpr int kPipeGroupWarps = HC_PIPE_GROUP_WARPS;
-constexpr int kPipeGroupThreads = kPipeGroupWarps * 32;
-constexpr int kPipeThreads = 64 + kPipeGroups * kPipeGroupThreads;
+// Consumer warps per group: fewer for n > 4, so that each thread has the
+// registers to hold n widened 16-byte rows (launch bounds give 65536 /
+// threads registers a thread: 128 at 7 warps per group, 170 at 5).
+__host__ __device__ constexpr int pipe_group_warps(int n) {
+    return n > 4 ? HC_PIPE_GROUP_WARPS_WIDE : HC_PIPE_GROUP_WARPS;
+}
+__host__ __device__ constexpr int pipe_threads(int n) {
+    return 64 + kPipeGroups * pipe_group_warps(n) * 32;
+}
 // The parameter warp prepares kParamReplicas warps' worth of lane groups at a
 // time (4 tokens for n = 3, 4; 2 for n >= 5); each group's slot ring holds at
 // least 8 of its tokens, and two batches, so preparation runs ahead.
@@ -77,7 +86,7 @@ constexpr int kSmemLimit = 232448;  // 227 KB opt-in dynamic shared memory per C
 
 struct PipeShape {
     int stages;       // stages in all (kPipeGroups rings of stages / kPipeGroups)
-    int tile;         // elements of d per tile (= kPipeGroupThreads * pipe_vec_elems)
+    int tile;         // elements of d per tile (= group threads * pipe_vec_elems)
     int ntile;        // tiles per token
     int stage_bytes;  // bytes of one stage
 };
@@ -91,18 +100,17 @@ __host__ __device__ constexpr int64_t pipe_fixed_bytes(int n, int stages, int64_
            + kPipeGroups * pipe_param_slots_per_group(n) * 16  // param full + empty
            + (kPipeGroups + 1) / 2 * 16                // group reduction barriers
            + kPipeGroups * pipe_param_slots_per_group(n) * (n * n + 2 * n) * 4  // slots
-           + kPipeGroups * 2 * kPipeGroupWarps * 8     // reduction partials
+           + kPipeGroups * 2 * pipe_group_warps(n) * 8  // reduction partials
            + 16                                        // abort flag (padded)
            + kParamReplicas * kGroupScratch * 4        // parameter warp scratch
            + (int64_t)kPipeGroups * 2 * ((d_h * 4 + 15) / 16 * 16);  // h rows (2 per group)
 }
 
-// Elements of d one consumer thread handles per tile: a 16-byte vector, or
-// half of one (8 bytes) for bf16 with n > 4, which keeps the n widened input
-// rows within the register budget.
+// Elements of d one consumer thread handles per tile: one 16-byte vector
+// (n > 4 runs fewer, register-richer consumer threads to afford it).
 template <int N, typename S>
 __host__ __device__ constexpr int pipe_vec_elems() {
-    return (sizeof(S) == 2 && N > 4) ? 4 : StorageTraits<S>::V;
+    return StorageTraits<S>::V;
 }
 
 // Shared-memory loads and streaming global stores of VE storage elements,
@@ -182,7 +190,7 @@ template <> struct VecIO<__nv_bfloat16, 4> {
 };
 
 template <int N, typename S, int KIND>
-__global__ void __launch_bounds__(kPipeThreads, 1)
+__global__ void __launch_bounds__(pipe_threads(N), 1)
 hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
     constexpr int V = pipe_vec_elems<N, S>();
     constexpr int VB = V * (int)sizeof(S);  // bytes per thread per row of a tile
@@ -191,7 +199,7 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
     constexpr bool READ = KIND != KIND_WRITE;
     constexpr int ROWS = WRITE ? N + 1 : N;
     constexpr int PSTRIDE = NN + 2 * N;  // A transposed (column j at j*N) | b | a
-    constexpr int GW = kPipeGroupWarps;
+    constexpr int GW = pipe_group_warps(N);
     constexpr int NG = kPipeGroups;
     constexpr int PSG = pipe_param_slots_per_group(N);
     constexpr int kParamSlots = NG * PSG;
