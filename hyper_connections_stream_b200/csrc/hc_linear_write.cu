@@ -46,11 +46,15 @@ constexpr int kLwM = 128;                    // token rows per CTA (TMEM lanes)
 constexpr int kLwTileM = 2 * kLwM;           // token rows per pair tile (MMA M)
 constexpr int kLwN = 256;                    // channels per tile (MMA N)
 constexpr int kLwBRows = kLwN / 2;           // Wo rows staged per CTA
-constexpr int kLwK = 64;                     // k per stage: one 128-byte swizzle row
-constexpr int kLwABytes = kLwM * kLwK * 2;   // 16 KB
-constexpr int kLwBBytes = kLwBRows * kLwK * 2;  // 16 KB
+constexpr int kLwKSub = 64;                  // one 128-byte swizzle row
+constexpr int kLwSubs = 2;                   // adjacent sub-tiles per stage
+constexpr int kLwK = kLwKSub * kLwSubs;      // k per stage
+constexpr int kLwASub = kLwM * kLwKSub * 2;      // 16 KB
+constexpr int kLwBSub = kLwBRows * kLwKSub * 2;  // 16 KB
+constexpr int kLwABytes = kLwSubs * kLwASub;
+constexpr int kLwBBytes = kLwSubs * kLwBSub;
 constexpr int kLwStageBytes = kLwABytes + kLwBBytes;
-constexpr int kLwStages = 6;
+constexpr int kLwStages = 3;
 constexpr uint32_t kLwTmemCols = 2 * kLwN;
 constexpr int kLwYBufBytes = 32 * (kLwN / 2) * 2;  // one epilogue warp: 32 rows x 128 bf16
 constexpr int kLwSmem = 1024 /* alignment slack */ + kLwStages * kLwStageBytes + 4 * kLwYBufBytes +
@@ -163,10 +167,13 @@ hc_linear_write_kernel(const __grid_constant__ CUtensorMap mapX,
                     }
                     unsigned char *st = smem + s * kLwStageBytes;
                     if (leader) mbar_arrive_expect_tx(&full[s], (uint32_t)(2 * kLwStageBytes));
-                    tma_load_2d_pair(st, &mapX, ks * kLwK, m0 + (int32_t)rank * kLwM,
-                                     full_leader + 8u * (uint32_t)s);
-                    tma_load_2d_pair(st + kLwABytes, &mapW, ks * kLwK, n0 + (int32_t)rank * kLwBRows,
-                                     full_leader + 8u * (uint32_t)s);
+#pragma unroll
+                    for (int c = 0; c < kLwSubs; ++c) {
+                        tma_load_2d_pair(st + c * kLwASub, &mapX, ks * kLwK + c * kLwKSub,
+                                         m0 + (int32_t)rank * kLwM, full_leader + 8u * (uint32_t)s);
+                        tma_load_2d_pair(st + kLwABytes + c * kLwBSub, &mapW, ks * kLwK + c * kLwKSub,
+                                         n0 + (int32_t)rank * kLwBRows, full_leader + 8u * (uint32_t)s);
+                    }
                     if (++s == S) {
                         s = 0;
                         ph ^= 1u;
@@ -204,10 +211,14 @@ hc_linear_write_kernel(const __grid_constant__ CUtensorMap mapX,
                     const uint32_t a0 = smem_addr(smem + s * kLwStageBytes);
                     const uint32_t b0 = a0 + (uint32_t)kLwABytes;
 #pragma unroll
-                    for (int kk = 0; kk < kLwK / 16; ++kk) {
-                        // +32 bytes along K per 16-element step inside the swizzle atom
-                        umma_bf16_pair(dacc, umma_desc_sw128(a0 + kk * 32), umma_desc_sw128(b0 + kk * 32),
-                                       idesc, (ks | kk) != 0);
+                    for (int c = 0; c < kLwSubs; ++c) {
+#pragma unroll
+                        for (int kk = 0; kk < kLwKSub / 16; ++kk) {
+                            // +32 bytes along K per 16-element step inside the swizzle atom
+                            umma_bf16_pair(dacc, umma_desc_sw128(a0 + c * kLwASub + kk * 32),
+                                           umma_desc_sw128(b0 + c * kLwBSub + kk * 32), idesc,
+                                           (ks | c | kk) != 0);
+                        }
                     }
                     umma_commit_pair(&empty[s], 0x3);  // both CTAs' stages are free once read
                     if (++s == S) {
@@ -414,9 +425,9 @@ hc_status launch_linear_write(const LinearWriteArgs &a, const LaunchCtx &ctx, cu
     lp.nk = (int)nk;
 
     CUtensorMap mapX, mapW;
-    hc_status ms = make_tma_map_bf16(&mapX, a.X, (uint64_t)a.k, (uint64_t)a.T, kLwK, kLwM);
+    hc_status ms = make_tma_map_bf16(&mapX, a.X, (uint64_t)a.k, (uint64_t)a.T, kLwKSub, kLwM);
     if (ms != HC_OK) return ms;
-    ms = make_tma_map_bf16(&mapW, a.Wo, (uint64_t)a.k, (uint64_t)a.d, kLwK, kLwBRows);
+    ms = make_tma_map_bf16(&mapW, a.Wo, (uint64_t)a.k, (uint64_t)a.d, kLwKSub, kLwBRows);
     if (ms != HC_OK) return ms;
     switch (a.n) {
         case 1: return launch_n_lw<1>(mapX, mapW, lp, ctx, st);
