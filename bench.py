@@ -473,6 +473,64 @@ def run_backward(args):
     }
 
 
+def run_decode(args):
+    """Decode-sized calls of the fused mHC step (T = 1 by default, --tokens to
+    change), n=4, d=7168, bf16, K=20: 200 calls captured in one CUDA graph and
+    replayed, so the host's per-call overhead is out of the device time; the
+    line reports microseconds per call (lower is better)."""
+    import torch
+    from hyper_connections_stream_b200 import _lib as hc
+    ws, rank, local = _dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = dict(WORKLOAD)
+    w["T"] = args.tokens or 1
+    T, n, d, K = w["T"], w["n"], w["d"], w["K"]
+    inp = make_inputs(w, rank, device)
+    bufs = (inp["H"], torch.empty_like(inp["H"]))
+    x = torch.empty((T, d), dtype=torch.bfloat16, device=device)
+    calls = 200
+
+    def step(i):
+        hc.write_then_read(bufs[i % 2], inp["y"], inp["L"], inp["b"], inp["rl"], inp["g"],
+                           eps=w["eps"], mix=hc.MIX_SINKHORN_LOGITS, K=K,
+                           read=hc.READ_SOFTMAX_LOGITS, out=bufs[(i + 1) % 2], x_next=x)
+
+    side = torch.cuda.Stream(device)
+    side.wait_stream(torch.cuda.current_stream(device))
+    with torch.cuda.stream(side):
+        for i in range(max(args.warmup, 3)):
+            step(i)
+    torch.cuda.current_stream(device).wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(calls):
+            step(i)
+    graph.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(device)
+    times = []
+    for _ in range(args.steps):
+        s_, e_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s_.record(stream)
+        graph.replay()
+        e_.record(stream)
+        torch.cuda.synchronize()
+        times.append(s_.elapsed_time(e_) * 1e3 / calls)
+    del graph
+    us = statistics.median(times)
+    return {
+        "metric": f"fused mHC step latency per call at T={T}, n=4, d=7168 (bf16, CUDA graph replay)",
+        "value": us, "unit": "us/call", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": us / 1e3, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "decode", "T": T, "n": n, "d": d, "K": K,
+                   "calls_per_graph": calls, "kernel_family": "auto (register-streaming)"},
+        "gpu_launches": args.steps * calls, "device_fault": hc.device_fault(),
+    }
+
+
 def run_ours(args):
     import torch
     from hyper_connections_stream_b200 import _lib as hc
@@ -725,12 +783,13 @@ def main(argv=None):
     ap.add_argument("--kernel-only", action="store_true",
                     help="device-timed kernel only (no e2e, no CPU baseline): for profiling")
     ap.add_argument("--op", choices=["step", "logits", "expand_read", "collapse", "linear_write",
-                                     "backward"],
+                                     "backward", "decode"],
                     default="step",
                     help="step: the fused HC step (the metric); logits: the tensor-core "
                          "mixing-logits kernel on the same streams; expand_read / collapse: "
                          "the stack ends on the same shape; linear_write: the block's output "
-                         "projection fused with the write; backward: the step's backward pass")
+                         "projection fused with the write; backward: the step's backward pass; "
+                         "decode: per-call latency of small steps (CUDA graph)")
     ap.add_argument("--path", choices=["auto", "pipelined", "register"], default="auto",
                     help="kernel family (auto = pipelined wherever it applies)")
     ap.add_argument("--tokens", type=int, default=0,
@@ -756,6 +815,8 @@ def main(argv=None):
         line = run_linear_write(args)
     elif args.op == "backward":
         line = run_backward(args)
+    elif args.op == "decode":
+        line = run_decode(args)
     else:
         line = run_ours(args)
     if line is not None:
