@@ -72,8 +72,11 @@ __host__ __device__ constexpr int pipe_threads(int n) {
 // Independent token batches the parameter warp runs through each Sinkhorn
 // pass together (their latencies overlap).
 constexpr int kParamReplicas = 2;
+// n > 5 holds two matrix elements per lane and one token per warp, so its
+// parameter warp runs four batches per pass to keep pace.
+__host__ __device__ constexpr int pipe_param_replicas(int n) { return n > 5 ? 4 : kParamReplicas; }
 __host__ __device__ constexpr int pipe_param_batch(int n) {
-    return kParamReplicas *
+    return pipe_param_replicas(n) *
            (n * n <= 1 ? 32 : n * n <= 2 ? 16 : n * n <= 4 ? 8 : n * n <= 8 ? 4 : n * n <= 16 ? 2 : 1);
 }
 __host__ __device__ constexpr int pipe_param_slots_per_group(int n) {
@@ -102,7 +105,7 @@ __host__ __device__ constexpr int64_t pipe_fixed_bytes(int n, int stages, int64_
            + kPipeGroups * pipe_param_slots_per_group(n) * (n * n + 2 * n) * 4  // slots
            + kPipeGroups * 2 * pipe_group_warps(n) * 8  // reduction partials
            + 16                                        // abort flag (padded)
-           + kParamReplicas * kGroupScratch * 4        // parameter warp scratch
+           + pipe_param_replicas(n) * kGroupScratch * 4  // parameter warp scratch
            + (int64_t)kPipeGroups * 2 * ((d_h * 4 + 15) / 16 * 16);  // h rows (2 per group)
 }
 
@@ -217,7 +220,7 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
     int *abort_word = reinterpret_cast<int *>(sred + NG * 2 * GW);
     volatile int *abort_flag = abort_word;
     float *pscratch = reinterpret_cast<float *>(abort_word + 4);  // parameter warp scratch
-    float *hrow_base = pscratch + kParamReplicas * kGroupScratch;  // 16-byte aligned
+    float *hrow_base = pscratch + pipe_param_replicas(N) * kGroupScratch;  // 16-byte aligned
     const int64_t d = p.d;
     const int64_t hrow_stride = READ ? (d + 3) / 4 * 4 : 0;  // floats per group row
     const int SG = sh.stages / NG;  // stages per group ring
@@ -333,7 +336,7 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
         // m0 + rb * TPW + lane / GL. The next batch's inputs are loaded
         // before the current batch is projected, hiding their latency.
         constexpr int GL = Group<N>::GL, EPL = Group<N>::EPL, TPW = Group<N>::TPW;
-        constexpr int R = kParamReplicas;
+        constexpr int R = pipe_param_replicas(N);
         static_assert(R * TPW == PB, "a batch is R warps' worth of lane groups");
         const int q = lane & (GL - 1);
         float nmv[R][EPL], nlv[R], nbv[R];
