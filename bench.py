@@ -419,6 +419,8 @@ def run_backward(args):
     w = dict(WORKLOAD)
     if args.tokens:
         w["T"] = args.tokens
+    if args.streams:
+        w["n"] = args.streams
     T, n, d, K = w["T"], w["n"], w["d"], w["K"]
     cfg = w["cfg"]
     H = gen.device_normal(gen.SEED_H + cfg, (T, n, d), torch.bfloat16, device)
@@ -456,7 +458,7 @@ def run_backward(args):
     peak, peak_kind = _peaks()
     achieved = alg_bytes / (step_ms / 1e3) / 1e9
     return {
-        "metric": "HC step backward tokens/sec at n=4, d=7168 (bf16, mHC K=20)",
+        "metric": f"HC step backward tokens/sec at n={n}, d={d} (bf16, mHC K={K})",
         "value": T * args.steps / (total_ms / 1e3), "unit": UNIT, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -466,7 +468,7 @@ def run_backward(args):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak,
                      "traffic": _profiled_traffic("backward_mhc_n4_d7168_bf16_T16384")
-                     if T == 16384 else None,
+                     if (T, n) == (16384, 4) else None,
                      "peak_source": peak_kind,
                      "algorithmic_bytes_per_step": alg_bytes, "step_ms": step_ms},
         "gpu_launches": 3 * args.steps, "device_fault": hc.device_fault(),

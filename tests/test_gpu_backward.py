@@ -7,8 +7,15 @@ Sinkhorn backward in fp32) while the oracle runs it in fp64. Bars: dH and dy
 elementwise within 1e-4 (fp32 storage) or 2e-2 (bf16 storage, the outputs are
 rounded to bf16) relative with the per-token rms floor; the per-token
 parameter gradients and dg within 2e-4 of the tensor's largest magnitude
-(fp32 sums of thousands of products, and 40 fp32 Sinkhorn passes undone). A
-wrong index, transpose or sign errs by O(1) relative to those scales.
+(fp32 sums of thousands of products, and 40 fp32 Sinkhorn passes undone),
+except the read-logit gradient for bf16 storage with logit-mode parameters:
+within 1e-3 (DA_BF16_LOGITS). There the exp of the Sinkhorn and softmax
+definitions differs by ulps between the two sides, a small fraction of the
+recomputed H' rounds to the adjacent bf16 value, and the softmax backward
+(a difference of near-equal sums) turns that into up to 2.5e-4 of the largest
+magnitude; the oracle's own da moves that much when its logits move by 6e-8
+(tests/test_oracle_pins.py::test_backward_read_logit_gradient_conditioning).
+A wrong index, transpose or sign errs by O(1) relative to those scales.
 """
 from __future__ import annotations
 
@@ -22,6 +29,11 @@ from tests._parity import f32_dev, rel_err, to_dev, to_host, values
 
 pytestmark = pytest.mark.gpu
 EPS = 1e-6
+DA_BF16_LOGITS = 1e-3
+
+
+def _param_bar(key, dt, mix, read):
+    return DA_BF16_LOGITS if (key == "da" and dt == "bf16" and (mix or read)) else 2e-4
 
 
 @pytest.fixture(scope="module")
@@ -75,7 +87,7 @@ def _check(hc, T, n, d, dt, mix, read, per_token, seed, with_dHout=True, K=20):
         gv = got[key].cpu().numpy().astype(np.float64)
         o = ref[key]
         e = float(np.max(np.abs(gv - o)) / (np.max(np.abs(o)) + 1e-30))
-        assert e <= 2e-4, f"{key}: err / max {e:.3e}"
+        assert e <= _param_bar(key, dt, mix, read), f"{key}: err / max {e:.3e}"
 
 
 @pytest.mark.parametrize("T,n,d,dt,mix,read,per_token", [
@@ -87,9 +99,21 @@ def _check(hc, T, n, d, dt, mix, read, per_token, seed, with_dHout=True, K=20):
     (129, 3, 1000, "f32", True, False, True),
     (300, 4, 7168, "bf16", True, True, True),
     (17, 6, 264, "bf16", False, True, False),
+    # bf16 at every n <= 5: ragged T and d, one token, and enough tokens per
+    # CTA for several parameter batches
+    (1, 4, 520, "bf16", True, True, True),
+    (41, 1, 1032, "bf16", False, True, True),
+    (150, 2, 776, "bf16", True, False, True),
+    (97, 3, 1544, "bf16", True, True, False),
+    (61, 5, 2056, "bf16", True, True, True),
+    (2000, 4, 1024, "bf16", True, True, True),
 ])
 def test_backward_matches_oracle(hc, T, n, d, dt, mix, read, per_token):
     _check(hc, T, n, d, dt, mix, read, per_token, seed=1200 + T + n)
+
+
+def test_backward_bf16_without_dHout(hc):
+    _check(hc, 90, 4, 1024, "bf16", True, True, True, seed=1350, with_dHout=False, K=3)
 
 
 def test_backward_without_dHout_and_small_K(hc):
@@ -130,7 +154,7 @@ def test_backward_full_size_sampled(hc):
     for key in ("dA", "db", "da"):
         gv = got[key][it].cpu().numpy().astype(np.float64)
         e = float(np.max(np.abs(gv - ref[key])) / np.max(np.abs(ref[key])))
-        assert e <= 2e-4, (key, e)
+        assert e <= _param_bar(key, dt, True, True), (key, e)
     parts = []
     for c in range(8):
         sl = slice(c * T // 8, (c + 1) * T // 8)
