@@ -61,6 +61,8 @@ KERNEL_SOURCES = {
                                          "hc_kernels_impl.cuh", "hc_k_bf16_ends.cu"],
     "linear_write_n4_d7168_k7168_bf16_T16384": ["hc_linear_write.cu", "hc_tc.cuh", "hc_sync.cuh"],
     "backward_mhc_n4_d7168_bf16_T16384": ["hc_backward.cu", "hc_device.cuh", "hc_sync.cuh"],
+    "reduce_write_r8_mhc_n4_d7168_bf16_T16384": ["hc_reduce_write.cu", "hc_device.cuh",
+                                                 "hc_launch.h"],
 }
 
 
@@ -312,6 +314,88 @@ def run_ends(args):
                      "traffic": _profiled_traffic(f"{args.op}_n4_d7168_bf16_T16384") if T == 16384 else None,
                      "peak_source": peak_kind,
                      "algorithmic_bytes_per_launch": alg_bytes, "kernel_ms": kern_ms},
+        "gpu_launches": args.steps, "device_fault": hc.device_fault(),
+    }
+
+
+def run_reduce_write(args):
+    """The write fused with the tensor-parallel all-reduce of y
+    (hc_reduce_write_then_read) on the workload's streams: R partial block
+    outputs (default 8, one per rank of a tensor-parallel group, all in this
+    GPU's memory: the same kernel reads them over NVLink when they are peer
+    mappings), summed in rank order, then the fused mHC write + read. Device
+    timed, one launch per step. Also times the unfused pair on the same GPU
+    (torch sum of the partials storing y, then hc_write_then_read)."""
+    import torch
+    import hc_inputs as gen
+    from hyper_connections_stream_b200 import _lib as hc
+    ws, rank, local = _dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = dict(WORKLOAD)
+    if args.tokens:
+        w["T"] = args.tokens
+    T, n, d, K, R = w["T"], w["n"], w["d"], w["K"], args.ranks
+    cfg = w["cfg"]
+    s = 2
+    parts = [gen.device_normal(gen.SEED_Y + cfg + 10 * r, (T, d), torch.bfloat16, device)
+             for r in range(R)]
+    H = gen.device_normal(gen.SEED_H + cfg, (T, n, d), torch.bfloat16, device)
+    L = gen.device_normal(gen.SEED_L + cfg, (T, n, n), torch.float32, device)
+    l = gen.device_normal(gen.SEED_L + 100 + cfg, (T, n), torch.float32, device)
+    b = torch.from_numpy(gen.normal(gen.SEED_P + cfg, (n,), mean=1.0, std=0.02)).to(device)
+    g = torch.from_numpy(gen.uniform(3500 + cfg, (d,), 0.5, 1.5)).to(device)
+    Hout = torch.empty_like(H)
+    x = torch.empty((T, d), dtype=torch.bfloat16, device=device)
+    kw = dict(eps=w["eps"], mix=hc.MIX_SINKHORN_LOGITS, K=K, read=hc.READ_SOFTMAX_LOGITS)
+
+    def fused():
+        hc.reduce_write_then_read(parts, H, L, b, l, g, out=Hout, x_next=x, **kw)
+
+    y = torch.empty((T, d), dtype=torch.bfloat16, device=device)
+    stacked = torch.stack(parts)
+
+    def unfused():
+        y.copy_(torch.sum(stacked, 0, dtype=torch.float32))
+        hc.write_then_read(H, y, L, b, l, g, out=Hout, x_next=x, **kw)
+
+    stream = torch.cuda.current_stream(device)
+
+    def timed(fn, steps):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for i in range(steps):
+            ev[i][0].record(stream)
+            fn()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        return (statistics.mean(a.elapsed_time(e) for a, e in ev), ev[0][0].elapsed_time(ev[-1][1]))
+
+    kern_ms, total_ms = timed(fused, args.steps)
+    unfused_ms, _ = timed(unfused, max(3, args.steps // 4))
+    alg_bytes = T * (d * s * (R + 2 * n + 1) + 4 * (n * n + n)) + d * 4
+    peak, peak_kind = _peaks()
+    achieved = alg_bytes / (kern_ms / 1e3) / 1e9
+    return {
+        "metric": f"HC step on the all-reduced block output (R={R} partials) tokens/sec at n={n}, "
+                  f"d={d} (bf16, mHC K={K})",
+        "value": T * args.steps / (total_ms / 1e3), "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "reduce_write", "T": T, "n": n, "d": d, "K": K, "ranks": R,
+                   "partials": "all in this GPU's memory",
+                   "l2": "inputs > L2 (re-read from HBM every step)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak,
+                     "traffic": _profiled_traffic("reduce_write_r8_mhc_n4_d7168_bf16_T16384")
+                     if (T, n, R) == (16384, 4, 8) else None,
+                     "peak_source": peak_kind,
+                     "algorithmic_bytes_per_launch": alg_bytes, "kernel_ms": kern_ms},
+        "unfused_ms": unfused_ms,
         "gpu_launches": args.steps, "device_fault": hc.device_fault(),
     }
 
@@ -785,19 +869,22 @@ def main(argv=None):
     ap.add_argument("--kernel-only", action="store_true",
                     help="device-timed kernel only (no e2e, no CPU baseline): for profiling")
     ap.add_argument("--op", choices=["step", "logits", "expand_read", "collapse", "linear_write",
-                                     "backward", "decode"],
+                                     "reduce_write", "backward", "decode"],
                     default="step",
                     help="step: the fused HC step (the metric); logits: the tensor-core "
                          "mixing-logits kernel on the same streams; expand_read / collapse: "
                          "the stack ends on the same shape; linear_write: the block's output "
-                         "projection fused with the write; backward: the step's backward pass; "
-                         "decode: per-call latency of small steps (CUDA graph)")
+                         "projection fused with the write; reduce_write: the write fused with "
+                         "the tensor-parallel all-reduce of y (--ranks partials); backward: the "
+                         "step's backward pass; decode: per-call latency of small steps (CUDA graph)")
     ap.add_argument("--path", choices=["auto", "pipelined", "register"], default="auto",
                     help="kernel family (auto = pipelined wherever it applies)")
+    ap.add_argument("--ranks", type=int, default=8,
+                    help="partials summed by --op reduce_write (tensor-parallel group size)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="override T (smaller cases for ncu captures)")
     ap.add_argument("--streams", type=int, default=0,
-                    help="override n for --op step (sweep cases; the metric's workload is n=4)")
+                    help="override n for --op step / backward (sweep cases; the metric's workload is n=4)")
     ap.add_argument("--width", type=int, default=0,
                     help="override d for --op step (sweep cases; the metric's workload is d=7168)")
     args = ap.parse_args(argv)
@@ -815,6 +902,8 @@ def main(argv=None):
         line = run_ends(args)
     elif args.op == "linear_write":
         line = run_linear_write(args)
+    elif args.op == "reduce_write":
+        line = run_reduce_write(args)
     elif args.op == "backward":
         line = run_backward(args)
     elif args.op == "decode":

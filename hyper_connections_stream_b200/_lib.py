@@ -52,6 +52,11 @@ SIGNATURES = {
     "hc_expand_then_read": ([_vp, _vp, _vp, _i32, _i64, _i32, _i64, _i32, _vp, _i64, _vp, _f32,
                              _vp], _i32),
     "hc_collapse": ([_vp, _vp, _i32, _i64, _i32, _i64, _i32, _vp, _i64, _vp], _i32),
+    "hc_reduce_write_then_read": ([_vp, _i32, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i64, _i32, _vp,
+                                   _i64, _i32, _vp, _i64, _i32, _vp, _i64, _vp, _f32, _vp], _i32),
+    "hc_ipc_export": ([_vp, _vp, C.POINTER(C.c_uint64)], _i32),
+    "hc_ipc_open": ([_vp, C.POINTER(_vp)], _i32),
+    "hc_ipc_close": ([_vp], _i32),
     "hc_status_string": ([_i32], C.c_char_p),
     "hc_last_error": ([], C.c_char_p),
     "hc_version": ([], _i32),
@@ -275,6 +280,73 @@ def write_then_read(H, y, A, b, a_next, g_next=None, *, eps: float = 1e-6,
                                     int(read), _ptr(a_next), a_s, _ptr(g_next), float(eps),
                                     _stream(H.device)))
     return out, x_next
+
+
+def reduce_write_then_read(parts, H, A, b, a_next, g_next=None, *, eps: float = 1e-6,
+                           mix: int = MIX_MATRIX, K: int = 0, read: int = READ_WEIGHTS,
+                           out=None, x_next=None, y_out=None):
+    """The fused step on the tensor-parallel all-reduce of the block output:
+    y = rnd(sum of the R partials in rank order, fp32), then
+    (H', x_next) = write_then_read(H, y, ...). `parts` lists the R partials in
+    rank order, each a [T, d] CUDA tensor of H's dtype or an int device
+    address (a peer mapping from dist.PeerPartials). y is stored only into
+    y_out when given. Returns (H', x_next). The call does not order the
+    partials' writes or overwrites against other ranks; dist.reduce_step
+    does."""
+    _need_cuda("H", H)
+    T, n, d = _streams_shape(H)
+    R = len(parts)
+    if not 1 <= R <= 8:
+        raise ValueError("1 <= len(parts) <= 8")
+    addrs = []
+    for r, q in enumerate(parts):
+        if isinstance(q, int):
+            addrs.append(q)
+        else:
+            _need_cuda(f"parts[{r}]", q, H.dtype)
+            if tuple(q.shape) != (T, d):
+                raise ValueError(f"parts[{r}] must be [T, d]")
+            addrs.append(q.data_ptr())
+    A_s = _tok_param("A", A, T, (n, n))
+    b_s = _tok_param("b", b, T, (n,))
+    a_s = _tok_param("a_next", a_next, T, (n,))
+    if g_next is not None:
+        _need_cuda("g_next", g_next, torch.float32)
+        if tuple(g_next.shape) != (d,):
+            raise ValueError("g_next must be [d]")
+    out = torch.empty_like(H) if out is None else out
+    x_next = torch.empty((T, d), dtype=H.dtype, device=H.device) if x_next is None else x_next
+    _need_out("out", out, (T, n, d), H.dtype)
+    _need_out("x_next", x_next, (T, d), H.dtype)
+    if y_out is not None:
+        _need_out("y_out", y_out, (T, d), H.dtype)
+    arr = (C.c_void_p * R)(*addrs)
+    _check(lib().hc_reduce_write_then_read(C.cast(arr, C.c_void_p), R, _ptr(H), _ptr(out),
+                                           _ptr(x_next), _ptr(y_out), _DT[H.dtype], T, n, d,
+                                           int(mix), _ptr(A), A_s, int(K), _ptr(b), b_s,
+                                           int(read), _ptr(a_next), a_s, _ptr(g_next),
+                                           float(eps), _stream(H.device)))
+    return out, x_next
+
+
+def ipc_export(t: torch.Tensor):
+    """(64-byte handle, byte offset) of the CUDA allocation holding t."""
+    handle = C.create_string_buffer(64)
+    off = C.c_uint64(0)
+    _check(lib().hc_ipc_export(C.c_void_p(t.data_ptr()), handle, C.byref(off)))
+    return handle.raw, int(off.value)
+
+
+def ipc_open(handle: bytes) -> int:
+    """Base address of another process's allocation, mapped into this one."""
+    buf = C.create_string_buffer(bytes(handle), 64)
+    base = C.c_void_p(0)
+    _check(lib().hc_ipc_open(buf, C.byref(base)))
+    return int(base.value)
+
+
+def ipc_close(base: int) -> None:
+    _check(lib().hc_ipc_close(C.c_void_p(base)))
 
 
 def expand(x, n: int, *, out=None):

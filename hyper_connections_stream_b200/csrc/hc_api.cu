@@ -6,6 +6,7 @@
 // the caller's stream.
 
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <climits>
 #include <cmath>
@@ -423,6 +424,115 @@ hc_status hc_collapse(const void *H, void *out, hc_dtype dt, int64_t T, int n, i
     p.a = w; p.a_s = w_tok_stride;
     p.read_logits = rm == HC_READ_SOFTMAX_LOGITS;
     return dispatch<hc::KIND_COLLAPSE>(dt, n, p, static_cast<cudaStream_t>(stream));
+}
+
+hc_status hc_reduce_write_then_read(const void *const *y_parts, int R, const void *H, void *Hout,
+                                    void *x_next, void *y_out, hc_dtype dt, int64_t T, int n,
+                                    int64_t d, hc_mix_mode mm, const float *A, int64_t A_tok_stride,
+                                    int K, const float *b, int64_t b_tok_stride, hc_read_mode rm,
+                                    const float *a_next, int64_t a_tok_stride, const float *g_next,
+                                    float eps, hc_stream stream) {
+    static const char *fn = "hc_reduce_write_then_read";
+    g_last_error[0] = '\0';
+    const Shape s{dt, T, n, d};
+    HC_TRY(check_shape(fn, s, true));
+    if (R < 1) return fail(HC_ERR_INVALID_ARG, "%s: R = %d < 1", fn, R);
+    if (R > hc::kMaxRanks) return fail(HC_ERR_UNSUPPORTED, "%s: R = %d > %d", fn, R, hc::kMaxRanks);
+    if (!y_parts) return fail(HC_ERR_INVALID_ARG, "%s: y_parts is NULL", fn);
+    if (mm != HC_MIX_MATRIX && mm != HC_MIX_SINKHORN_LOGITS)
+        return fail(HC_ERR_INVALID_ARG, "%s: bad mix mode %d", fn, (int)mm);
+    if (rm != HC_READ_WEIGHTS && rm != HC_READ_SOFTMAX_LOGITS)
+        return fail(HC_ERR_INVALID_ARG, "%s: bad read mode %d", fn, (int)rm);
+    if (mm == HC_MIX_SINKHORN_LOGITS) HC_TRY(check_K(fn, K));
+    HC_TRY(check_stride(fn, "A_tok_stride", A_tok_stride));
+    HC_TRY(check_stride(fn, "b_tok_stride", b_tok_stride));
+    HC_TRY(check_stride(fn, "a_tok_stride", a_tok_stride));
+    HC_TRY(check_eps(fn, eps));
+    if (T == 0) return HC_OK;
+    HC_TRY(check_buf(fn, "H", H));
+    HC_TRY(check_buf(fn, "Hout", Hout));
+    HC_TRY(check_buf(fn, "x_next", x_next));
+    for (int r = 0; r < R; ++r) {
+        char name[24];
+        snprintf(name, sizeof name, "y_parts[%d]", r);
+        HC_TRY(check_buf(fn, name, y_parts[r]));
+    }
+    if (y_out && !aligned(y_out, 16)) return fail(HC_ERR_MISALIGNED, "%s: y_out is not 16-byte aligned", fn);
+    HC_TRY(check_param(fn, "A", A));
+    HC_TRY(check_param(fn, "b", b));
+    HC_TRY(check_param(fn, "a_next", a_next));
+    if (g_next && !aligned(g_next, 16))
+        return fail(HC_ERR_MISALIGNED, "%s: g_next is not 16-byte aligned", fn);
+    const int64_t es = elem_bytes(dt);
+    const int64_t hb = T * n * d * es, yb = T * d * es;
+    if (Hout != H && overlap(Hout, hb, H, hb)) return fail(HC_ERR_ALIAS, "%s: Hout partially overlaps H", fn);
+    if (overlap(x_next, yb, H, hb) || overlap(x_next, yb, Hout, hb))
+        return fail(HC_ERR_ALIAS, "%s: x_next overlaps H or Hout", fn);
+    if (y_out && (overlap(y_out, yb, H, hb) || overlap(y_out, yb, Hout, hb) || overlap(y_out, yb, x_next, yb)))
+        return fail(HC_ERR_ALIAS, "%s: y_out overlaps H, Hout or x_next", fn);
+    for (int r = 0; r < R; ++r) {
+        const void *q = y_parts[r];
+        if (overlap(Hout, hb, q, yb) || overlap(x_next, yb, q, yb) || (y_out && overlap(y_out, yb, q, yb)))
+            return fail(HC_ERR_ALIAS, "%s: an output overlaps y_parts[%d]", fn, r);
+    }
+    hc::LaunchCtx ctx{};
+    HC_TRY(launch_ctx(ctx));
+    hc::ReduceWriteArgs ra{};
+    ra.f.H = H; ra.f.Hout = Hout; ra.f.x = x_next; ra.f.T = T; ra.f.d = d;
+    ra.f.A = A; ra.f.A_s = A_tok_stride; ra.f.b = b; ra.f.b_s = b_tok_stride;
+    ra.f.a = a_next; ra.f.a_s = a_tok_stride; ra.f.g = g_next; ra.f.eps = eps;
+    ra.f.K = K; ra.f.mix_logits = mm == HC_MIX_SINKHORN_LOGITS;
+    ra.f.read_logits = rm == HC_READ_SOFTMAX_LOGITS;
+    for (int r = 0; r < R; ++r) ra.parts[r] = y_parts[r];
+    ra.R = R;
+    ra.n = n;
+    ra.y_out = y_out;
+    return hc::launch_reduce_write(ra, dt, ctx, static_cast<cudaStream_t>(stream));
+}
+
+hc_status hc_ipc_export(const void *dev_ptr, void *handle, uint64_t *offset) {
+    static const char *fn = "hc_ipc_export";
+    g_last_error[0] = '\0';
+    if (!dev_ptr || !handle || !offset) return fail(HC_ERR_INVALID_ARG, "%s: NULL argument", fn);
+    static PFN_cuMemGetAddressRange_v3020 range_fn = nullptr;
+    if (!range_fn) {
+        void *fp = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &fp, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fp)
+            return fail(HC_ERR_CUDA, "%s: cuMemGetAddressRange is not available", fn);
+        range_fn = reinterpret_cast<PFN_cuMemGetAddressRange_v3020>(fp);
+    }
+    CUdeviceptr base = 0;
+    size_t bytes = 0;
+    const CUresult cr = range_fn(&base, &bytes, reinterpret_cast<CUdeviceptr>(dev_ptr));
+    if (cr != CUDA_SUCCESS) return fail(HC_ERR_CUDA, "%s: cuMemGetAddressRange failed (%d)", fn, (int)cr);
+    cudaIpcMemHandle_t h;
+    const cudaError_t e = cudaIpcGetMemHandle(&h, reinterpret_cast<void *>(base));
+    if (e != cudaSuccess) return fail(HC_ERR_CUDA, "%s: cudaIpcGetMemHandle: %s", fn, cudaGetErrorString(e));
+    memcpy(handle, &h, sizeof h);
+    *offset = (uint64_t)(reinterpret_cast<CUdeviceptr>(dev_ptr) - base);
+    return HC_OK;
+}
+
+hc_status hc_ipc_open(const void *handle, void **base) {
+    static const char *fn = "hc_ipc_open";
+    g_last_error[0] = '\0';
+    if (!handle || !base) return fail(HC_ERR_INVALID_ARG, "%s: NULL argument", fn);
+    cudaIpcMemHandle_t h;
+    memcpy(&h, handle, sizeof h);
+    const cudaError_t e = cudaIpcOpenMemHandle(base, h, cudaIpcMemLazyEnablePeerAccess);
+    if (e != cudaSuccess) return fail(HC_ERR_CUDA, "%s: cudaIpcOpenMemHandle: %s", fn, cudaGetErrorString(e));
+    return HC_OK;
+}
+
+hc_status hc_ipc_close(void *base) {
+    static const char *fn = "hc_ipc_close";
+    g_last_error[0] = '\0';
+    if (!base) return fail(HC_ERR_INVALID_ARG, "%s: base is NULL", fn);
+    const cudaError_t e = cudaIpcCloseMemHandle(base);
+    if (e != cudaSuccess) return fail(HC_ERR_CUDA, "%s: cudaIpcCloseMemHandle: %s", fn, cudaGetErrorString(e));
+    return HC_OK;
 }
 
 hc_status hc_linear_then_write(const void *X, const void *Wo, const void *H, void *Hout, void *y_out,

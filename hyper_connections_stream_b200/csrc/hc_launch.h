@@ -67,6 +67,19 @@ hc_status backward_workspace_bytes(int n, hc_dtype dt, int64_t T, int64_t d, con
                                    size_t *bytes);
 hc_status launch_backward(const BackwardArgs &a, const LaunchCtx &ctx, cudaStream_t st);
 
+// The write mix fused with the tensor-parallel all-reduce of y, then the
+// next layer's read (see hc_reduce_write_then_read).
+constexpr int kMaxRanks = 8;
+struct ReduceWriteArgs {
+    StepParams f;                  // H, Hout, x, params, T, d (f.y unused)
+    const void *parts[kMaxRanks];  // the ranks' partial y, in rank order
+    int R;
+    int n;
+    void *y_out;  // reduced y, or null
+};
+hc_status launch_reduce_write(const ReduceWriteArgs &ra, hc_dtype dt, const LaunchCtx &ctx,
+                              cudaStream_t st);
+
 hc_status launch_selftest_wait(int limit_us, const LaunchCtx &ctx, cudaStream_t st);
 
 hc_status launch_sinkhorn(const float *L, float *out, int64_t T, int n, int K,

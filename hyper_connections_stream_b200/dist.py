@@ -47,3 +47,74 @@ def max_over_ranks(value: float, world: int, device=None) -> float:
                      device=device if device is not None else "cpu")
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+# ---- tensor-parallel all-reduce of y fused with the write ---------------------
+#
+# Under tensor parallelism every rank of a group ends a block with a partial y
+# and holds a replica of the streams H. hc_reduce_write_then_read reads all
+# ranks' partials over peer memory and sums them in rank order inside the
+# fused write + read, so y never goes through a separate all-reduce. The
+# kernel waits on no other rank; the host orders the partials' writes before
+# the call and their next overwrite after every rank's call (reduce_step).
+
+class PeerPartials:
+    """Every rank's partial-y buffer, mapped into this process.
+
+    `local` is this rank's [T, d] partial buffer (kept and rewritten in place
+    every layer). The ranks exchange CUDA IPC handles over `group` (any
+    torch.distributed backend) and open each other's; `pointers` lists the R
+    device addresses in rank order, this rank's own buffer at its index.
+    export / open_ / close default to the library's hc_ipc_* calls and are
+    parameters so the exchange can be exercised without GPUs."""
+
+    def __init__(self, local, group=None, *, export=None, open_=None, close=None):
+        import torch.distributed as dist
+        if export is None or open_ is None or close is None:
+            from . import _lib as hc
+            export = export or hc.ipc_export
+            open_ = open_ or hc.ipc_open
+            close = close or hc.ipc_close
+        self._close = close
+        self.rank = dist.get_rank(group)
+        self.world = dist.get_world_size(group)
+        handle, offset = export(local)
+        gathered = [None] * self.world
+        dist.all_gather_object(gathered, (self.rank, bytes(handle), int(offset)), group=group)
+        self._bases = []
+        self.pointers = []
+        for r, (who, h, off) in enumerate(gathered):
+            if who != r:
+                raise RuntimeError(f"rank {r} reported itself as rank {who}")
+            if r == self.rank:
+                self.pointers.append(int(local.data_ptr()))
+            else:
+                base = int(open_(h))
+                self._bases.append(base)
+                self.pointers.append(base + off)
+
+    def close(self):
+        while self._bases:
+            self._close(self._bases.pop())
+
+
+def reduce_step(peers: PeerPartials, H, A, b, a_next, g_next=None, group=None, *,
+                call=None, sync=None, **kw):
+    """One fused step on the all-reduced y: waits until every rank's partial
+    is written (stream sync + barrier), runs hc_reduce_write_then_read on the
+    peers' pointers, then waits until every rank has read them (stream sync +
+    barrier) so each may overwrite its partial for the next layer. Returns
+    (H', x_next). `call` and `sync` default to the library call and
+    torch.cuda.current_stream().synchronize."""
+    import torch.distributed as dist
+    if call is None:
+        from . import _lib as hc
+        call = hc.reduce_write_then_read
+    if sync is None:
+        sync = lambda: torch.cuda.current_stream().synchronize()  # noqa: E731
+    sync()
+    dist.barrier(group)
+    out = call(peers.pointers, H, A, b, a_next, g_next, **kw)
+    sync()
+    dist.barrier(group)
+    return out

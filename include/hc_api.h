@@ -163,6 +163,57 @@ HC_API hc_status hc_linear_then_write(const void *X, const void *Wo, const void 
                                       const float *b, int64_t b_tok_stride, hc_stream stream);
 
 /*
+ * The write mix fused with the tensor-parallel all-reduce of the block output,
+ * then the next layer's read (Hy4-preview model techniques map,
+ * models.inteligile.com, "inference kernel": kernel fusion used, the model
+ * served with its layers split over eight GPUs; glossary entry
+ * "Hyper-connections (mHC)": streams mixed after each block). Under tensor
+ * parallelism each of R ranks ends the block with a partial output y_r and
+ * holds a replica of H; every rank makes this call and reads all R partials:
+ *   y        = rnd( ((y_0 + y_1) + y_2) + ... + y_{R-1} )   fp32 adds in rank
+ *              order, one rounding to dt (the same on every rank, so the
+ *              replicas of H' and x_next stay bit-identical);
+ *   then exactly hc_write_then_read(H, y, ...) with that y.
+ *   y_parts: host array of R device pointers (1 <= R <= 8), the partials
+ *     [T][d] of dtype dt in rank order. Each may be this device's memory or a
+ *     peer's memory mapped into this process (hc_ipc_open, or an allocation
+ *     on a peer-accessible device); the kernel reads them with plain loads.
+ *     16-byte aligned; the library only reads them.
+ *   y_out: if not NULL, y is also stored there ([T][d], dt), else never.
+ *   Other arguments, layouts and checks as hc_write_then_read; no output may
+ *   overlap a partial. Asynchronous on `stream`; T == 0 is a no-op.
+ * The kernel never waits on another rank. The caller orders every rank's
+ * writes of its partial before this call's work starts on `stream`, and any
+ * later overwrite of a partial after every rank's call has finished reading
+ * it (the Python layer uses a barrier on each side).
+ */
+HC_API hc_status hc_reduce_write_then_read(
+    const void *const *y_parts, int R, const void *H, void *Hout, void *x_next, void *y_out,
+    hc_dtype dt, int64_t T, int n, int64_t d, hc_mix_mode mm, const float *A, int64_t A_tok_stride,
+    int K, const float *b, int64_t b_tok_stride, hc_read_mode rm, const float *a_next,
+    int64_t a_tok_stride, const float *g_next, float eps, hc_stream stream);
+
+/*
+ * Peer mappings for the partials of hc_reduce_write_then_read (CUDA IPC;
+ * one process per GPU). The pages have no counterpart to these; they are
+ * plumbing of this library.
+ *   hc_ipc_export: for a device pointer of this process, the 64-byte handle
+ *     (HC_IPC_HANDLE_BYTES) of the allocation that holds it and the pointer's
+ *     byte offset from that allocation's start (caching allocators hand out
+ *     pointers inside larger allocations).
+ *   hc_ipc_open: maps another process's allocation into this one (peer
+ *     access enabled lazily) and returns its base; add the exporter's offset.
+ *     A process cannot open its own handles (HC_ERR_CUDA).
+ *   hc_ipc_close: unmaps a base returned by hc_ipc_open.
+ * HC_ERR_INVALID_ARG on NULL arguments, HC_ERR_CUDA when the runtime refuses
+ * (its message in hc_last_error). Synchronous host calls.
+ */
+#define HC_IPC_HANDLE_BYTES 64
+HC_API hc_status hc_ipc_export(const void *dev_ptr, void *handle, uint64_t *offset);
+HC_API hc_status hc_ipc_open(const void *handle, void **base);
+HC_API hc_status hc_ipc_close(void *base);
+
+/*
  * Backward pass of hc_write_then_read (training; the forward is the
  * glossary entry's mixing before and after a block with the mHC Sinkhorn
  * projection, plus the block's pre-norm). Gradients pass straight through the

@@ -166,6 +166,29 @@ def write_then_read(H, y, A, b, a, g, eps: float, dt: str, K: int = 0,
     return Hout, x
 
 
+def reduce_partials(parts, dt: str):
+    """The block output as the tensor-parallel all-reduce of R partials
+    defines it for the fused write (a reading: the pages say the model is
+    served split over eight GPUs and name no summation order): the partials,
+    widened to fp32, are added left to right in rank order with an fp32
+    rounding after every add (numpy float32 addition is IEEE round to nearest
+    even), and the sum is rounded once to the storage dtype."""
+    acc = np.array(to_f32(parts[0], dt), dtype=np.float32, copy=True)
+    for p in parts[1:]:
+        acc = np.add(acc, to_f32(p, dt), dtype=np.float32)
+    return round_to(acc, dt)
+
+
+def reduce_write_then_read(parts, H, A, b, a, g, eps: float, dt: str, K: int = 0,
+                           mix_logits: bool = False, read_logits: bool = False):
+    """The fused step on the all-reduced block output: (H', x_next, y) with
+    y = reduce_partials(parts) and (H', x_next) = write_then_read(H, y, ...)."""
+    y = reduce_partials(parts, dt)
+    Hp, x = write_then_read(H, y, A, b, a, g, eps, dt, K=K, mix_logits=mix_logits,
+                            read_logits=read_logits)
+    return Hp, x, y
+
+
 def mix_logits(H, W, eps: float, dt: str):
     """fp64 logits z[t, j] = r_t * sum_k u_t[k] W[j, k], u_t = H[t] flattened,
     r_t = 1 / sqrt(mean(u_t^2) + eps). H [T, n, d]; W [P, n*d]."""

@@ -129,6 +129,30 @@ _CHILD = textwrap.dedent(r"""
     call("lw_null_A", "hc_linear_then_write", Xl, Wl, H, Ho, None, bf, T, n, d, 64, None, 0, b, 0, None)
     call("lw_alias_y", "hc_linear_then_write", Xl, Wl, H, Ho, Ho + 64, bf, T, n, d, 64, A, 0, b, 0, None)
     call("lw_alias_X", "hc_linear_then_write", Xl, Wl, H, Xl + 32, None, bf, T, n, d, 64, A, 0, b, 0, None)
+    P0, P1, P2 = buf(60), buf(61), buf(62)
+    def parts(*ps):
+        arr = (C.c_void_p * len(ps))(*ps)
+        parts.keep.append(arr)  # the host array must outlive the call
+        return C.cast(arr, C.c_void_p)
+    parts.keep = []
+    ok3 = parts(P0, P1, P2)
+    def rw(tag, pp, R, Hh=H, Hout=Ho, xx=x, yo=None, d_=d, T_=T, dt=bf):
+        call(tag, "hc_reduce_write_then_read", pp, R, Hh, Hout, xx, yo, dt, T_, n, d_, 0, A, 0, 0,
+             b, 0, 0, a, 0, None, 1e-6, None)
+    rw("rw_T0", ok3, 3, Hh=None, Hout=None, xx=None, T_=0)
+    rw("rw_R0", ok3, 0)
+    rw("rw_R9", parts(*([P0] * 9)), 9)
+    rw("rw_parts_null", None, 3)
+    rw("rw_part_null", parts(P0, None, P2), 3)
+    rw("rw_part_mis", parts(P0, P1 + 8, P2), 3)
+    rw("rw_alias_x_part", ok3, 3, xx=P1 + 32)
+    rw("rw_alias_Hout_part", ok3, 3, Hout=P2 - hb + 64)
+    rw("rw_alias_yout_H", ok3, 3, yo=H + 64)
+    rw("rw_mis_yout", ok3, 3, yo=buf(70) + 8)
+    rw("rw_d_too_big", ok3, 3, d_=32768 + 8)
+    call("ipc_export_null", "hc_ipc_export", None, None, None)
+    call("ipc_open_null", "hc_ipc_open", None, None)
+    call("ipc_close_null", "hc_ipc_close", None)
     print(json.dumps(res))
 """)
 
@@ -156,6 +180,10 @@ def test_argument_validation_statuses():
         "co_alias": ALI, "co_mis_w": MIS,
         "lw_f32": UNS, "lw_k_ragged": UNS, "lw_k0": INV, "lw_T0": OK, "lw_mis_X": MIS,
         "lw_null_A": INV, "lw_alias_y": ALI, "lw_alias_X": ALI,
+        "rw_T0": OK, "rw_R0": INV, "rw_R9": UNS, "rw_parts_null": INV, "rw_part_null": INV,
+        "rw_part_mis": MIS, "rw_alias_x_part": ALI, "rw_alias_Hout_part": ALI,
+        "rw_alias_yout_H": ALI, "rw_mis_yout": MIS, "rw_d_too_big": UNS,
+        "ipc_export_null": INV, "ipc_open_null": INV, "ipc_close_null": INV,
     }
     for tag, code in want.items():
         got, msg = res[tag]

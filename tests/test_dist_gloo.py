@@ -93,3 +93,97 @@ def test_token_shard_partitions_exactly():
                 assert start == pos
                 pos += count
             assert max(c for _, c in spans) - min(c for _, c in spans) <= 1
+
+
+class _FakeLocal:
+    """Stands in for a rank's partial-y tensor: only its address is used."""
+
+    def __init__(self, addr):
+        self.addr = addr
+
+    def data_ptr(self):
+        return self.addr
+
+
+def _peer_worker(rank, world, port, T, n, d, out_dir):
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    import hc_inputs as gen
+    import oracle
+    from hyper_connections_stream_b200 import dist as hd
+    oracle.set_threads(1)
+    opened, closed, events = [], [], []
+    # fake IPC: a handle names its exporter; an exporter's allocation starts
+    # 16 * rank bytes before its partial; a peer's allocation maps at 1e6 * (r + 1)
+    local = _FakeLocal(1000 * (rank + 1))
+
+    def export(t):
+        return f"rank{rank}".encode().ljust(64, b"\0"), 16 * rank
+
+    def open_(h):
+        r = int(h.rstrip(b"\0").decode()[4:])
+        opened.append(r)
+        return 10 ** 6 * (r + 1)
+
+    peers = hd.PeerPartials(local, export=export, open_=open_, close=closed.append)
+    want = [1000 * (rank + 1) if r == rank else 10 ** 6 * (r + 1) + 16 * r for r in range(world)]
+    assert peers.pointers == want, (peers.pointers, want)
+    assert sorted(opened) == [r for r in range(world) if r != rank]
+
+    # every rank's partial, reachable "through its address" (the data moves
+    # with gloo here, standing in for the peer loads of the GPU kernel)
+    part = gen.to_storage(gen.normal(2600 + rank, (T, d)), "bf16")
+    parts = [None] * world
+    dist.all_gather_object(parts, part)
+    by_addr = {want_r: parts[r] for r, want_r in enumerate(peers.pointers)}
+    H = gen.to_storage(gen.normal(2700, (T, n, d)), "bf16")   # replicated stream state
+    L = gen.normal(2701, (T, n, n))
+    b = gen.normal(2702, (n,), mean=1.0, std=0.02)
+    l = gen.normal(2703, (T, n))
+
+    def call(ptrs, H_, A_, b_, a_, g_, **kw):
+        events.append("call")
+        Hp, x, _ = oracle.reduce_write_then_read([by_addr[p] for p in ptrs], H_, A_, b_, a_, g_,
+                                                 1e-6, "bf16", K=20, mix_logits=True,
+                                                 read_logits=True)
+        return Hp, x
+
+    Hp, x = hd.reduce_step(peers, H, L, b, l, None, call=call, sync=lambda: events.append("sync"))
+    assert events == ["sync", "call", "sync"], events
+    peers.close()
+    assert sorted(closed) == sorted(10 ** 6 * (r + 1) for r in range(world) if r != rank)
+    outs = [None] * world
+    dist.all_gather_object(outs, (Hp, x))
+    if rank == 0:
+        np.save(os.path.join(out_dir, "Hp.npy"), np.stack([o[0] for o in outs]))
+        np.save(os.path.join(out_dir, "x.npy"), np.stack([o[1] for o in outs]))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_peer_partials_and_reduce_step_on_gloo_ranks(tmp_path):
+    """Three gloo ranks exchange (fake) IPC handles: each gets every rank's
+    partial address in rank order (its own unopened, the others opened and
+    offset), runs the step between two synchronisations, and closes what it
+    opened. Every rank's H' and x_next equal the single-process oracle on all
+    partials, so the replicas stay identical."""
+    import hc_inputs as gen
+    import oracle
+    world, T, n, d = 3, 5, 4, 64
+    mp.spawn(_peer_worker, args=(world, _free_port(), T, n, d, str(tmp_path)), nprocs=world,
+             join=True)
+    parts = [gen.to_storage(gen.normal(2600 + r, (T, d)), "bf16") for r in range(world)]
+    H = gen.to_storage(gen.normal(2700, (T, n, d)), "bf16")
+    L = gen.normal(2701, (T, n, n))
+    b = gen.normal(2702, (n,), mean=1.0, std=0.02)
+    l = gen.normal(2703, (T, n))
+    Hp, x, _ = oracle.reduce_write_then_read(parts, H, L, b, l, None, 1e-6, "bf16", K=20,
+                                             mix_logits=True, read_logits=True)
+    got_H = np.load(tmp_path / "Hp.npy")
+    got_x = np.load(tmp_path / "x.npy")
+    for r in range(world):
+        assert np.array_equal(got_H[r], Hp) and np.array_equal(got_x[r], x)

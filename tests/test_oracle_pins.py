@@ -724,3 +724,31 @@ def test_backward_read_logit_gradient_conditioning():
               for k in ("dA", "db", "da")}
     assert spread["dA"] < 2e-5 and spread["db"] < 1e-4, spread
     assert 1e-5 < spread["da"] < 1e-3, spread
+
+
+# ---- all-reduce of the block output (the fused reduce + write) ----
+
+def test_reduce_partials_is_the_rank_order_sum_rounded_once():
+    """Pins reduce_partials to what the reading fixes: a sum (exact on small
+    integers), taken left to right in fp32 (2^24 + 1 + 1 keeps 2^24 in that
+    order, gives 2^24 + 2 in the other), rounded to bf16 once at the end
+    (1 + 2^-8 + 2^-8 is 1 + 2^-7 exactly in fp32; rounding after each add would
+    give 1), and one partial passes through unchanged."""
+    rng = np.random.default_rng(2024)
+    ints = rng.integers(-30, 31, size=(8, 5, 16))
+    parts = [oracle.round_to(v.astype(np.float32), "bf16") for v in ints]
+    got = oracle.to_f32(oracle.reduce_partials(parts, "bf16"), "bf16")
+    assert np.array_equal(got, ints.sum(axis=0).astype(np.float32))
+
+    big = np.float32(2.0 ** 24)
+    f = [np.array([big], np.float32), np.array([1.0], np.float32), np.array([1.0], np.float32)]
+    assert oracle.reduce_partials(f, "f32")[0] == big
+    assert oracle.reduce_partials(f[::-1], "f32")[0] == big + 2
+
+    one, tiny = np.array([1.0], np.float32), np.array([2.0 ** -8], np.float32)
+    b3 = [oracle.round_to(v, "bf16") for v in (one, tiny, tiny)]
+    assert oracle.to_f32(oracle.reduce_partials(b3, "bf16"), "bf16")[0] == np.float32(1 + 2.0 ** -7)
+    assert oracle.to_f32(oracle.reduce_partials(b3[:2], "bf16"), "bf16")[0] == np.float32(1.0)
+
+    y = oracle.round_to(rng.standard_normal((3, 40)).astype(np.float32), "bf16")
+    assert np.array_equal(oracle.reduce_partials([y], "bf16"), y)
