@@ -165,7 +165,7 @@ hc_status dispatch(hc_dtype dt, int n, const hc::StepParams &p, cudaStream_t st)
 
 extern "C" {
 
-int hc_version(void) { return 200; }
+int hc_version(void) { return 300; }
 
 const char *hc_status_string(hc_status st) {
     switch (st) {
