@@ -494,15 +494,16 @@ hc_status hc_ipc_export(const void *dev_ptr, void *handle, uint64_t *offset) {
     static const char *fn = "hc_ipc_export";
     g_last_error[0] = '\0';
     if (!dev_ptr || !handle || !offset) return fail(HC_ERR_INVALID_ARG, "%s: NULL argument", fn);
-    static PFN_cuMemGetAddressRange_v3020 range_fn = nullptr;
-    if (!range_fn) {
+    // looked up once (thread-safe static initialisation); null if unavailable
+    static const PFN_cuMemGetAddressRange_v3020 range_fn = [] {
         void *fp = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &fp, cudaEnableDefault, &q) != cudaSuccess ||
-            q != cudaDriverEntryPointSuccess || !fp)
-            return fail(HC_ERR_CUDA, "%s: cuMemGetAddressRange is not available", fn);
-        range_fn = reinterpret_cast<PFN_cuMemGetAddressRange_v3020>(fp);
-    }
+            q != cudaDriverEntryPointSuccess)
+            fp = nullptr;
+        return reinterpret_cast<PFN_cuMemGetAddressRange_v3020>(fp);
+    }();
+    if (!range_fn) return fail(HC_ERR_CUDA, "%s: cuMemGetAddressRange is not available", fn);
     CUdeviceptr base = 0;
     size_t bytes = 0;
     const CUresult cr = range_fn(&base, &bytes, reinterpret_cast<CUdeviceptr>(dev_ptr));

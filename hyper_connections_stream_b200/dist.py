@@ -83,15 +83,19 @@ class PeerPartials:
         dist.all_gather_object(gathered, (self.rank, bytes(handle), int(offset)), group=group)
         self._bases = []
         self.pointers = []
-        for r, (who, h, off) in enumerate(gathered):
-            if who != r:
-                raise RuntimeError(f"rank {r} reported itself as rank {who}")
-            if r == self.rank:
-                self.pointers.append(int(local.data_ptr()))
-            else:
-                base = int(open_(h))
-                self._bases.append(base)
-                self.pointers.append(base + off)
+        try:
+            for r, (who, h, off) in enumerate(gathered):
+                if who != r:
+                    raise RuntimeError(f"rank {r} reported itself as rank {who}")
+                if r == self.rank:
+                    self.pointers.append(int(local.data_ptr()))
+                else:
+                    base = int(open_(h))
+                    self._bases.append(base)
+                    self.pointers.append(base + off)
+        except BaseException:
+            self.close()  # unmap what was opened before the failure
+            raise
 
     def close(self):
         while self._bases:

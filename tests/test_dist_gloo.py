@@ -187,3 +187,40 @@ def test_peer_partials_and_reduce_step_on_gloo_ranks(tmp_path):
     got_x = np.load(tmp_path / "x.npy")
     for r in range(world):
         assert np.array_equal(got_H[r], Hp) and np.array_equal(got_x[r], x)
+
+
+def _peer_fail_worker(rank, world, port):
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    from hyper_connections_stream_b200 import dist as hd
+    closed = []
+
+    def open_(h):
+        r = int(h.rstrip(b"\0").decode()[4:])
+        if r == world - 1 and rank == 0:
+            raise OSError("peer mapping refused")
+        return 10 ** 6 * (r + 1)
+
+    export = lambda t: (f"rank{rank}".encode().ljust(64, b"\0"), 0)  # noqa: E731
+    if rank == 0:
+        try:
+            hd.PeerPartials(_FakeLocal(64), export=export, open_=open_, close=closed.append)
+        except OSError:
+            pass
+        else:
+            raise AssertionError("the refused mapping did not propagate")
+        # the peer opened before the failure (rank 1) is unmapped again
+        assert closed == [10 ** 6 * 2], closed
+    else:
+        peers = hd.PeerPartials(_FakeLocal(64), export=export, open_=open_, close=closed.append)
+        peers.close()
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_peer_partials_unmaps_on_a_failed_open():
+    mp.spawn(_peer_fail_worker, args=(3, _free_port()), nprocs=3, join=True)
