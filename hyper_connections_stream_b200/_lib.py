@@ -54,6 +54,9 @@ SIGNATURES = {
     "hc_collapse": ([_vp, _vp, _i32, _i64, _i32, _i64, _i32, _vp, _i64, _vp], _i32),
     "hc_reduce_write_then_read": ([_vp, _i32, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i64, _i32, _vp,
                                    _i64, _i32, _vp, _i64, _i32, _vp, _i64, _vp, _f32, _vp], _i32),
+    "hc_reduce_scatter_write_then_read": ([_vp, _i32, _i32, _i64, _vp, _vp, _vp, _vp, _i32, _i32,
+                                           _i64, _i32, _vp, _i64, _i32, _vp, _i64, _i32, _vp, _i64,
+                                           _vp, _f32, _vp], _i32),
     "hc_ipc_export": ([_vp, _vp, C.POINTER(C.c_uint64)], _i32),
     "hc_ipc_open": ([_vp, C.POINTER(_vp)], _i32),
     "hc_ipc_close": ([_vp], _i32),
@@ -132,13 +135,12 @@ def _need_gain(name, g, d):
             raise ValueError(f"{name} must be [d]")
 
 
-def _tok_param(name, p, T, per_shape):
-    """Shared ([*per_shape], contiguous) or per-token ([T, *per_shape]) fp32
-    parameter -> token stride in floats. A per-token parameter may be a view
-    whose tokens are `stride(0)` floats apart as long as each token's set is
-    contiguous (e.g. a slice of the [T, P] output of mix_logits)."""
-    if not isinstance(p, torch.Tensor) or not p.is_cuda or p.dtype != torch.float32:
-        raise ValueError(f"{name} must be a float32 CUDA tensor")
+def _tok_layout(name, p, T, per_shape):
+    """Token stride in floats of a shared ([*per_shape], contiguous) or
+    per-token ([T, *per_shape]) parameter: 0 when shared. A per-token
+    parameter may be a view whose tokens are `stride(0)` floats apart as long
+    as each token's set is contiguous (e.g. a slice of the [T, P] output of
+    mix_logits); with T == 0 nothing of it is read."""
     per = 1
     for s in per_shape:
         per *= s
@@ -147,12 +149,18 @@ def _tok_param(name, p, T, per_shape):
             raise ValueError(f"{name} must be contiguous")
         return 0
     if tuple(p.shape) == (T, *per_shape):
-        inner = p[0] if T > 0 else p.reshape(per_shape)
-        if T > 0 and not inner.is_contiguous():
+        if T > 0 and not p[0].is_contiguous():
             raise ValueError(f"{name}: each token's values must be contiguous")
         return p.stride(0) if T > 1 else per
     raise ValueError(f"{name} must have shape {tuple(per_shape)} or {(T, *per_shape)}, "
                      f"got {tuple(p.shape)}")
+
+
+def _tok_param(name, p, T, per_shape):
+    """A float32 CUDA parameter, shared or per token -> its token stride."""
+    if not isinstance(p, torch.Tensor) or not p.is_cuda or p.dtype != torch.float32:
+        raise ValueError(f"{name} must be a float32 CUDA tensor")
+    return _tok_layout(name, p, T, per_shape)
 
 
 def _streams_shape(H):
@@ -327,6 +335,66 @@ def reduce_write_then_read(parts, H, A, b, a_next, g_next=None, *, eps: float = 
                                            int(read), _ptr(a_next), a_s, _ptr(g_next),
                                            float(eps), _stream(H.device)))
     return out, x_next
+
+
+def _addrs(name, bufs, shape, dtype):
+    out = []
+    for r, q in enumerate(bufs):
+        if isinstance(q, int):
+            out.append(q)
+        else:
+            _need_cuda(f"{name}[{r}]", q, dtype)
+            if tuple(q.shape) != shape:
+                raise ValueError(f"{name}[{r}] must be {list(shape)}")
+            out.append(q.data_ptr())
+    return out
+
+
+def reduce_scatter_write_then_read(parts, x_all, rank: int, H, A, b, a_next, g_next=None, *,
+                                   eps: float = 1e-6, mix: int = MIX_MATRIX, K: int = 0,
+                                   read: int = READ_WEIGHTS, out=None, y_out=None):
+    """The reduce-scatter form: H is this rank's token shard [T_r, n, d] of
+    the group's streams; parts and x_all list the R ranks' full [T, d] partials
+    and x_next buffers (tensors or int device addresses). Reduces the rank's
+    rows of the partials, writes its shard of H' (returned) and stores x_next
+    for its rows into every x_all buffer. T is inferred from the buffers."""
+    _need_cuda("H", H)
+    Tr, n, d = _streams_shape(H)
+    R = len(parts)
+    if not 1 <= R <= 8 or len(x_all) != R:
+        raise ValueError("1 <= len(parts) == len(x_all) <= 8")
+    T = None
+    for q in list(parts) + list(x_all):
+        if not isinstance(q, int):
+            T = q.shape[0]
+            break
+    if T is None:
+        raise ValueError("pass at least one partial or x buffer as a tensor (to give T)")
+    if not 0 <= rank < R:
+        raise ValueError("0 <= rank < len(parts)")
+    base, extra = divmod(T, R)
+    if Tr != base + (1 if rank < extra else 0):
+        raise ValueError(f"H holds {Tr} tokens; rank {rank} of {R} owns {base + (rank < extra)} of {T}")
+    pa = _addrs("parts", parts, (T, d), H.dtype)
+    xa = _addrs("x_all", x_all, (T, d), H.dtype)
+    A_s = _tok_param("A", A, Tr, (n, n))
+    b_s = _tok_param("b", b, Tr, (n,))
+    a_s = _tok_param("a_next", a_next, Tr, (n,))
+    if g_next is not None:
+        _need_cuda("g_next", g_next, torch.float32)
+        if tuple(g_next.shape) != (d,):
+            raise ValueError("g_next must be [d]")
+    out = torch.empty_like(H) if out is None else out
+    _need_out("out", out, (Tr, n, d), H.dtype)
+    if y_out is not None:
+        _need_out("y_out", y_out, (Tr, d), H.dtype)
+    parr = (C.c_void_p * R)(*pa)
+    xarr = (C.c_void_p * R)(*xa)
+    _check(lib().hc_reduce_scatter_write_then_read(
+        C.cast(parr, C.c_void_p), R, int(rank), T, _ptr(H), _ptr(out), C.cast(xarr, C.c_void_p),
+        _ptr(y_out), _DT[H.dtype], n, d, int(mix), _ptr(A), A_s, int(K), _ptr(b), b_s, int(read),
+        _ptr(a_next), a_s, _ptr(g_next), float(eps), _stream(H.device)))
+    return out
 
 
 def ipc_export(t: torch.Tensor):

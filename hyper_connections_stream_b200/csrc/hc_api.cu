@@ -478,7 +478,7 @@ hc_status hc_reduce_write_then_read(const void *const *y_parts, int R, const voi
     hc::LaunchCtx ctx{};
     HC_TRY(launch_ctx(ctx));
     hc::ReduceWriteArgs ra{};
-    ra.f.H = H; ra.f.Hout = Hout; ra.f.x = x_next; ra.f.T = T; ra.f.d = d;
+    ra.f.H = H; ra.f.Hout = Hout; ra.f.T = T; ra.f.d = d;
     ra.f.A = A; ra.f.A_s = A_tok_stride; ra.f.b = b; ra.f.b_s = b_tok_stride;
     ra.f.a = a_next; ra.f.a_s = a_tok_stride; ra.f.g = g_next; ra.f.eps = eps;
     ra.f.K = K; ra.f.mix_logits = mm == HC_MIX_SINKHORN_LOGITS;
@@ -487,6 +487,92 @@ hc_status hc_reduce_write_then_read(const void *const *y_parts, int R, const voi
     ra.R = R;
     ra.n = n;
     ra.y_out = y_out;
+    ra.t0 = 0;
+    ra.xs[0] = x_next;
+    ra.nx = 1;
+    return hc::launch_reduce_write(ra, dt, ctx, static_cast<cudaStream_t>(stream));
+}
+
+hc_status hc_reduce_scatter_write_then_read(const void *const *y_parts, int R, int rank,
+                                            int64_t T_total, const void *H, void *Hout,
+                                            void *const *x_all, void *y_out, hc_dtype dt, int n,
+                                            int64_t d, hc_mix_mode mm, const float *A,
+                                            int64_t A_tok_stride, int K, const float *b,
+                                            int64_t b_tok_stride, hc_read_mode rm,
+                                            const float *a_next, int64_t a_tok_stride,
+                                            const float *g_next, float eps, hc_stream stream) {
+    static const char *fn = "hc_reduce_scatter_write_then_read";
+    g_last_error[0] = '\0';
+    if (R < 1) return fail(HC_ERR_INVALID_ARG, "%s: R = %d < 1", fn, R);
+    if (R > hc::kMaxRanks) return fail(HC_ERR_UNSUPPORTED, "%s: R = %d > %d", fn, R, hc::kMaxRanks);
+    if (rank < 0 || rank >= R) return fail(HC_ERR_INVALID_ARG, "%s: rank %d outside 0..%d", fn, rank, R - 1);
+    HC_TRY(check_shape(fn, Shape{dt, T_total, n, d}, true));
+    // this rank's tokens: contiguous shards, the first T_total % R one longer
+    const int64_t base = T_total / R, extra = T_total % R;
+    const int64_t t0 = rank * base + (rank < extra ? rank : extra);
+    const int64_t T = base + (rank < extra ? 1 : 0);
+    if (!y_parts) return fail(HC_ERR_INVALID_ARG, "%s: y_parts is NULL", fn);
+    if (!x_all) return fail(HC_ERR_INVALID_ARG, "%s: x_all is NULL", fn);
+    if (mm != HC_MIX_MATRIX && mm != HC_MIX_SINKHORN_LOGITS)
+        return fail(HC_ERR_INVALID_ARG, "%s: bad mix mode %d", fn, (int)mm);
+    if (rm != HC_READ_WEIGHTS && rm != HC_READ_SOFTMAX_LOGITS)
+        return fail(HC_ERR_INVALID_ARG, "%s: bad read mode %d", fn, (int)rm);
+    if (mm == HC_MIX_SINKHORN_LOGITS) HC_TRY(check_K(fn, K));
+    HC_TRY(check_stride(fn, "A_tok_stride", A_tok_stride));
+    HC_TRY(check_stride(fn, "b_tok_stride", b_tok_stride));
+    HC_TRY(check_stride(fn, "a_tok_stride", a_tok_stride));
+    HC_TRY(check_eps(fn, eps));
+    if (T == 0) return HC_OK;
+    HC_TRY(check_buf(fn, "H", H));
+    HC_TRY(check_buf(fn, "Hout", Hout));
+    for (int r = 0; r < R; ++r) {
+        char name[24];
+        snprintf(name, sizeof name, "y_parts[%d]", r);
+        HC_TRY(check_buf(fn, name, y_parts[r]));
+        snprintf(name, sizeof name, "x_all[%d]", r);
+        HC_TRY(check_buf(fn, name, x_all[r]));
+    }
+    if (y_out && !aligned(y_out, 16)) return fail(HC_ERR_MISALIGNED, "%s: y_out is not 16-byte aligned", fn);
+    HC_TRY(check_param(fn, "A", A));
+    HC_TRY(check_param(fn, "b", b));
+    HC_TRY(check_param(fn, "a_next", a_next));
+    if (g_next && !aligned(g_next, 16))
+        return fail(HC_ERR_MISALIGNED, "%s: g_next is not 16-byte aligned", fn);
+    const int64_t es = elem_bytes(dt);
+    const int64_t hb = T * n * d * es, yb = T * d * es, fb = T_total * d * es;
+    if (Hout != H && overlap(Hout, hb, H, hb)) return fail(HC_ERR_ALIAS, "%s: Hout partially overlaps H", fn);
+    if (y_out && (overlap(y_out, yb, H, hb) || overlap(y_out, yb, Hout, hb)))
+        return fail(HC_ERR_ALIAS, "%s: y_out overlaps H or Hout", fn);
+    for (int q = 0; q < R; ++q) {
+        const void *xq = x_all[q], *pq = y_parts[q];
+        if (overlap(xq, fb, H, hb) || overlap(xq, fb, Hout, hb) || (y_out && overlap(xq, fb, y_out, yb)))
+            return fail(HC_ERR_ALIAS, "%s: x_all[%d] overlaps H, Hout or y_out", fn, q);
+        if (overlap(Hout, hb, pq, fb) || (y_out && overlap(y_out, yb, pq, fb)))
+            return fail(HC_ERR_ALIAS, "%s: an output overlaps y_parts[%d]", fn, q);
+        for (int r = 0; r < R; ++r) {
+            if (overlap(xq, fb, y_parts[r], fb))
+                return fail(HC_ERR_ALIAS, "%s: x_all[%d] overlaps y_parts[%d]", fn, q, r);
+            if (r > q && overlap(xq, fb, x_all[r], fb))
+                return fail(HC_ERR_ALIAS, "%s: x_all[%d] overlaps x_all[%d]", fn, q, r);
+        }
+    }
+    hc::LaunchCtx ctx{};
+    HC_TRY(launch_ctx(ctx));
+    hc::ReduceWriteArgs ra{};
+    ra.f.H = H; ra.f.Hout = Hout; ra.f.T = T; ra.f.d = d;
+    ra.f.A = A; ra.f.A_s = A_tok_stride; ra.f.b = b; ra.f.b_s = b_tok_stride;
+    ra.f.a = a_next; ra.f.a_s = a_tok_stride; ra.f.g = g_next; ra.f.eps = eps;
+    ra.f.K = K; ra.f.mix_logits = mm == HC_MIX_SINKHORN_LOGITS;
+    ra.f.read_logits = rm == HC_READ_SOFTMAX_LOGITS;
+    for (int r = 0; r < R; ++r) {
+        ra.parts[r] = y_parts[r];
+        ra.xs[r] = x_all[r];
+    }
+    ra.R = R;
+    ra.nx = R;
+    ra.n = n;
+    ra.y_out = y_out;
+    ra.t0 = t0;
     return hc::launch_reduce_write(ra, dt, ctx, static_cast<cudaStream_t>(stream));
 }
 

@@ -71,11 +71,14 @@ hc_status launch_backward(const BackwardArgs &a, const LaunchCtx &ctx, cudaStrea
 // next layer's read (see hc_reduce_write_then_read).
 constexpr int kMaxRanks = 8;
 struct ReduceWriteArgs {
-    StepParams f;                  // H, Hout, x, params, T, d (f.y unused)
+    StepParams f;                  // H, Hout, params, T (tokens of this call), d (f.y, f.x unused)
     const void *parts[kMaxRanks];  // the ranks' partial y, in rank order
     int R;
     int n;
-    void *y_out;  // reduced y, or null
+    void *y_out;                   // reduced y [T][d] (this call's tokens), or null
+    int64_t t0;                    // row of the partials and of x for this call's token 0
+    void *xs[kMaxRanks];           // x_next destinations (rows t0 .. t0 + T - 1 of each)
+    int nx;
 };
 hc_status launch_reduce_write(const ReduceWriteArgs &ra, hc_dtype dt, const LaunchCtx &ctx,
                               cudaStream_t st);

@@ -14,11 +14,19 @@
 // rank, so the replicas of H stay equal without another exchange. y never
 // makes a round trip through HBM unless the caller asks for it.
 //
-// The kernel only reads peer memory (plain loads, no TMA, no multicast) and
-// never waits on another rank: the caller orders each partial's writes before
-// the call and its next overwrite after every rank's call (the host layer
-// does this with two barriers). With R buffers of one GPU it is the same
-// computation over all ranks' data in one launch.
+// Two forms share the kernel. One-shot (hc_reduce_write_then_read): every
+// rank reduces every token and writes its own replica of H' and x. Reduce-
+// scatter (hc_reduce_scatter_write_then_read): the streams are sharded by
+// token over the ranks; a rank reduces the partials' rows of its own tokens
+// only, writes its shard of H', and stores that shard's x_next into every
+// rank's x buffer (the all-gather, as plain stores to peer memory).
+//
+// The kernel reads and writes peer memory with plain loads and stores (no
+// TMA, no multicast) and never waits on another rank: the caller orders each
+// partial's writes before the call, and every later read of x or overwrite
+// of a partial after every rank's call (the host layer does this with two
+// barriers). With buffers of one GPU it is the same computation over all
+// ranks' data, one launch per rank.
 //
 // One CTA per token at a time (grid-stride), threads own 16-byte column
 // slices; h stays in registers until the CTA's fp64 sum of squares is known.
@@ -62,7 +70,6 @@ hc_reduce_step_kernel(ReduceWriteArgs ra) {
 
     const S *H = static_cast<const S *>(p.H);
     S *Ho = static_cast<S *>(p.Hout);
-    S *X = static_cast<S *>(p.x);
     S *Yo = static_cast<S *>(ra.y_out);
 
     int parity = 0;
@@ -77,6 +84,7 @@ hc_reduce_step_kernel(ReduceWriteArgs ra) {
             if (t >= p.T) break;  // uniform over the CTA
             const S *Ht = H + t * N * p.d;
             S *Hot = Ho + t * N * p.d;
+            const int64_t tg = ra.t0 + t;  // row of the partials and of x
             float hs[CPT][V];
             double ss = 0.0;
 #pragma unroll
@@ -88,12 +96,12 @@ hc_reduce_step_kernel(ReduceWriteArgs ra) {
 #pragma unroll
                     for (int i = 0; i < N; ++i) load_vec_cs(Ht + i * p.d + k, h[i]);
                     // the all-reduce: partials added in rank order, one rounding
-                    load_vec_cs(static_cast<const S *>(ra.parts[0]) + t * p.d + k, yv);
+                    load_vec_cs(static_cast<const S *>(ra.parts[0]) + tg * p.d + k, yv);
 #pragma unroll
                     for (int r = 1; r < kMaxRanks; ++r) {
                         if (r < R) {
                             float pv[V];
-                            load_vec_cs(static_cast<const S *>(ra.parts[r]) + t * p.d + k, pv);
+                            load_vec_cs(static_cast<const S *>(ra.parts[r]) + tg * p.d + k, pv);
 #pragma unroll
                             for (int e = 0; e < V; ++e) yv[e] = __fadd_rn(yv[e], pv[e]);
                         }
@@ -144,7 +152,6 @@ hc_reduce_step_kernel(ReduceWriteArgs ra) {
             for (int w = 0; w < nwarps; ++w) tot += sred[parity][w];
             parity ^= 1;
             const float r = __double2float_rn(1.0 / sqrt(tot / (double)p.d + (double)p.eps));
-            S *Xt = X + t * p.d;
 #pragma unroll
             for (int u = 0; u < CPT; ++u) {
                 const int64_t c = tid + (int64_t)u * NT;
@@ -154,7 +161,12 @@ hc_reduce_step_kernel(ReduceWriteArgs ra) {
                     load_gain<V>(p.g, k, gv);
 #pragma unroll
                     for (int e = 0; e < V; ++e) xv[e] = __fmul_rn(__fmul_rn(hs[u][e], r), gv[e]);
-                    store_vec_cs(Xt + k, xv);
+                    // x_next to every destination (the all-gather of the
+                    // reduce-scatter form: peers' buffers take plain stores)
+                    store_vec_cs(static_cast<S *>(ra.xs[0]) + tg * p.d + k, xv);
+#pragma unroll
+                    for (int q = 1; q < kMaxRanks; ++q)
+                        if (q < ra.nx) store_vec_cs(static_cast<S *>(ra.xs[q]) + tg * p.d + k, xv);
                 }
             }
         }

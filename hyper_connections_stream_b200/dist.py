@@ -122,3 +122,27 @@ def reduce_step(peers: PeerPartials, H, A, b, a_next, g_next=None, group=None, *
     sync()
     dist.barrier(group)
     return out
+
+
+def reduce_scatter_step(peers_y: PeerPartials, peers_x: PeerPartials, H_shard, A, b, a_next,
+                        g_next=None, group=None, *, call=None, sync=None, **kw):
+    """The reduce-scatter form of reduce_step: the streams are sharded by
+    token over the group (this rank holds H_shard, token_shard(T, rank, R)),
+    peers_y maps the ranks' partials and peers_x the ranks' x_next buffers.
+    The call reduces this rank's rows, writes its shard of H' and stores its
+    rows of x_next into every rank's x buffer; the second barrier makes all of
+    x_next complete on every rank before anyone reads it. Returns H'_shard."""
+    import torch.distributed as dist
+    if peers_y.rank != peers_x.rank or peers_y.world != peers_x.world:
+        raise ValueError("peers_y and peers_x must come from the same group")
+    if call is None:
+        from . import _lib as hc
+        call = hc.reduce_scatter_write_then_read
+    if sync is None:
+        sync = lambda: torch.cuda.current_stream().synchronize()  # noqa: E731
+    sync()
+    dist.barrier(group)
+    out = call(peers_y.pointers, peers_x.pointers, peers_y.rank, H_shard, A, b, a_next, g_next, **kw)
+    sync()
+    dist.barrier(group)
+    return out

@@ -194,7 +194,39 @@ HC_API hc_status hc_reduce_write_then_read(
     int64_t a_tok_stride, const float *g_next, float eps, hc_stream stream);
 
 /*
- * Peer mappings for the partials of hc_reduce_write_then_read (CUDA IPC;
+ * The reduce-scatter form of hc_reduce_write_then_read, for streams sharded
+ * by token over the R ranks of a tensor-parallel group (same pages; same
+ * arithmetic per token). Rank `rank` owns the contiguous tokens
+ *   t0 = rank * (T_total / R) + min(rank, T_total % R),
+ *   T  = T_total / R + (rank < T_total % R ? 1 : 0)
+ * and, for each of them, sums the rows t0..t0+T-1 of the R partials in rank
+ * order (fp32, one rounding), writes its shard of H', and stores x_next into
+ * rows t0..t0+T-1 of EVERY rank's x buffer (the all-gather of x). Each rank
+ * thus moves about as many bytes over NVLink as a ring all-reduce of y, and
+ * does 1/R of the HBM work of the one-shot form.
+ *   y_parts: R device pointers, the ranks' full partials [T_total][d].
+ *   x_all:   R device pointers, the ranks' full x_next buffers [T_total][d]
+ *            (x_all[rank] this rank's own); peers' may be hc_ipc_open
+ *            mappings. Written only in this rank's rows.
+ *   H, Hout: this rank's shard [T][n][d]; y_out: [T][d] or NULL. A, b,
+ *            a_next per token index the shard's tokens (pass pointers to the
+ *            shard's rows), or stride 0 for one set.
+ *   1 <= R <= 8, 0 <= rank < R. Other arguments and checks as
+ *   hc_reduce_write_then_read; no x_all buffer may overlap another, a
+ *   partial, or this rank's inputs and outputs. T == 0 is a no-op.
+ * The kernel never waits on another rank: the caller orders every partial's
+ * writes before the call, and every read of x_next (or overwrite of a
+ * partial) after every rank's call has finished.
+ */
+HC_API hc_status hc_reduce_scatter_write_then_read(
+    const void *const *y_parts, int R, int rank, int64_t T_total, const void *H, void *Hout,
+    void *const *x_all, void *y_out, hc_dtype dt, int n, int64_t d, hc_mix_mode mm,
+    const float *A, int64_t A_tok_stride, int K, const float *b, int64_t b_tok_stride,
+    hc_read_mode rm, const float *a_next, int64_t a_tok_stride, const float *g_next, float eps,
+    hc_stream stream);
+
+/*
+ * Peer mappings for the partials and x buffers of the reduce calls (CUDA IPC;
  * one process per GPU). The pages have no counterpart to these; they are
  * plumbing of this library.
  *   hc_ipc_export: for a device pointer of this process, the 64-byte handle

@@ -150,6 +150,23 @@ _CHILD = textwrap.dedent(r"""
     rw("rw_alias_yout_H", ok3, 3, yo=H + 64)
     rw("rw_mis_yout", ok3, 3, yo=buf(70) + 8)
     rw("rw_d_too_big", ok3, 3, d_=32768 + 8)
+    X0, X1 = buf(80), buf(81)
+    okx = parts(X0, X1)
+    ok2 = parts(P0, P1)
+    def rs(tag, pp, xx, R, rank, T_=T, Hh=H, Hout=Ho):
+        call(tag, "hc_reduce_scatter_write_then_read", pp, R, rank, T_, Hh, Hout, xx, None, bf, n,
+             d, 0, A, 0, 0, b, 0, 0, a, 0, None, 1e-6, None)
+    rs("rs_T0", ok2, okx, 2, 1, T_=0, Hh=None, Hout=None)
+    rs("rs_empty_shard", ok2, okx, 2, 1, T_=1, Hh=None, Hout=None)
+    rs("rs_rank_neg", ok2, okx, 2, -1)
+    rs("rs_rank_big", ok2, okx, 2, 2)
+    rs("rs_R9", parts(*([P0] * 9)), parts(*([X0] * 9)), 9, 0)
+    rs("rs_x_null", ok2, None, 2, 0)
+    rs("rs_x_entry_null", ok2, parts(X0, None), 2, 0)
+    rs("rs_x_mis", ok2, parts(X0, X1 + 8), 2, 0)
+    rs("rs_x_dup", ok2, parts(X0, X0), 2, 0)
+    rs("rs_x_is_part", ok2, parts(X0, P1), 2, 0)
+    rs("rs_x_over_H", ok2, parts(X0, H + 64), 2, 0)
     call("ipc_export_null", "hc_ipc_export", None, None, None)
     call("ipc_open_null", "hc_ipc_open", None, None)
     call("ipc_close_null", "hc_ipc_close", None)
@@ -184,6 +201,9 @@ def test_argument_validation_statuses():
         "rw_part_mis": MIS, "rw_alias_x_part": ALI, "rw_alias_Hout_part": ALI,
         "rw_alias_yout_H": ALI, "rw_mis_yout": MIS, "rw_d_too_big": UNS,
         "ipc_export_null": INV, "ipc_open_null": INV, "ipc_close_null": INV,
+        "rs_T0": OK, "rs_empty_shard": OK, "rs_rank_neg": INV, "rs_rank_big": INV, "rs_R9": UNS,
+        "rs_x_null": INV, "rs_x_entry_null": INV, "rs_x_mis": MIS, "rs_x_dup": ALI,
+        "rs_x_is_part": ALI, "rs_x_over_H": ALI,
     }
     for tag, code in want.items():
         got, msg = res[tag]
@@ -222,3 +242,26 @@ def test_public_header_compiles_standalone_as_c_and_cpp(tmp_path):
         out = subprocess.run([*cmd, "-I", inc, "-c", str(src), "-o", str(tmp_path / "o.o")],
                              capture_output=True, text=True)
         assert out.returncode == 0, (cmd[0], out.stderr)
+
+
+def test_parameter_layouts():
+    """Token strides the binding passes for shared and per-token parameters,
+    including no tokens at all (a rank of the reduce-scatter form may own
+    none) and a strided view of a wider per-token array."""
+    import pytest
+    import torch
+    from hyper_connections_stream_b200._lib import _tok_layout
+    n = 4
+    assert _tok_layout("A", torch.zeros(n, n), 7, (n, n)) == 0
+    assert _tok_layout("A", torch.zeros(0, n, n), 0, (n, n)) == n * n
+    assert _tok_layout("a", torch.zeros(0, n), 0, (n,)) == n
+    assert _tok_layout("A", torch.zeros(1, n, n), 1, (n, n)) == n * n
+    assert _tok_layout("A", torch.zeros(5, n, n), 5, (n, n)) == n * n
+    z = torch.zeros(5, 24)
+    assert _tok_layout("a", z[:, 16:20], 5, (n,)) == 24
+    with pytest.raises(ValueError):
+        _tok_layout("A", torch.zeros(n, n).t(), 3, (n, n))       # shared but transposed
+    with pytest.raises(ValueError):
+        _tok_layout("A", torch.zeros(5, n, n).transpose(1, 2), 5, (n, n))
+    with pytest.raises(ValueError):
+        _tok_layout("A", torch.zeros(4, n, n), 5, (n, n))

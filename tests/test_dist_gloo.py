@@ -154,8 +154,25 @@ def _peer_worker(rank, world, port, T, n, d, out_dir):
 
     Hp, x = hd.reduce_step(peers, H, L, b, l, None, call=call, sync=lambda: events.append("sync"))
     assert events == ["sync", "call", "sync"], events
+
+    # the reduce-scatter form: x buffers mapped like the partials; the call
+    # gets both pointer lists and this rank's shard
+    xpeers = hd.PeerPartials(_FakeLocal(5000 + rank), export=export, open_=open_,
+                             close=closed.append)
+    t0, Tr = hd.token_shard(T, rank, world)
+    seen = []
+
+    def rs_call(yp, xp, r, H_, A_, b_, a_, g_, **kw):
+        seen.append((list(yp), list(xp), r, H_.shape[0]))
+        return H_
+
+    hd.reduce_scatter_step(peers, xpeers, H[t0:t0 + Tr], L[t0:t0 + Tr], b, l[t0:t0 + Tr], None,
+                           call=rs_call, sync=lambda: events.append("sync"))
+    assert seen == [(peers.pointers, xpeers.pointers, rank, Tr)], seen
+    assert xpeers.pointers[rank] == 5000 + rank
+    xpeers.close()
     peers.close()
-    assert sorted(closed) == sorted(10 ** 6 * (r + 1) for r in range(world) if r != rank)
+    assert sorted(closed) == sorted(2 * [10 ** 6 * (r + 1) for r in range(world) if r != rank])
     outs = [None] * world
     dist.all_gather_object(outs, (Hp, x))
     if rank == 0:

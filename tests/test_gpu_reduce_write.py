@@ -174,3 +174,67 @@ def test_rejections(hc):
     assert e.value.status == hc.HC_ERR_ALIAS
     Hp, x = hc.reduce_write_then_read([y[:0]], H[:0], A, b, a)
     assert Hp.shape == (0, n, d) and x.shape == (0, d)
+
+
+def _shard(T, r, R):
+    base, extra = divmod(T, R)
+    return r * base + min(r, extra), base + (1 if r < extra else 0)
+
+
+@pytest.mark.parametrize("T,n,d,R,dt,logits", [
+    (37, 4, 1024, 4, "bf16", False),   # ragged shards: 37 = 4 x 9 + 1
+    (300, 4, 7168, 8, "bf16", True),
+    (5, 2, 520, 8, "bf16", False),     # fewer tokens than ranks: three ranks own none
+    (64, 3, 1032, 3, "f32", False),
+    (41, 8, 512, 2, "bf16", True),
+])
+def test_reduce_scatter_form(hc, T, n, d, R, dt, logits):
+    """R ranks emulated on one GPU, one launch per rank: each reduces its
+    token shard of the partials, writes its shard of H', and stores its rows
+    of x_next into all R x buffers (which start as NaN, so every row must be
+    written by exactly one rank). Shards concatenated equal the oracle's step
+    over all tokens; every x buffer equals the oracle's x_next."""
+    parts, H, A, b, a, g = _case(T, n, d, R, dt, logits, True, seed=3500 + T + R)
+    Hr, xr, yr = oracle.reduce_write_then_read(parts, H, A, b, a, g, EPS, dt, K=20,
+                                               mix_logits=logits, read_logits=logits)
+    sdt = TORCH_DT[dt]
+    dparts = [to_dev(p, dt) for p in parts]
+    xs = [torch.full((T, d), float("nan"), dtype=sdt, device="cuda") for _ in range(R)]
+    Hs, ys = [], []
+    for r in range(R):
+        t0, Tr = _shard(T, r, R)
+        sl = slice(t0, t0 + Tr)
+        y_out = torch.empty((Tr, d), dtype=sdt, device="cuda")
+        Hs.append(hc.reduce_scatter_write_then_read(
+            dparts, xs, r, to_dev(H[sl], dt), f32_dev(A[sl]), f32_dev(b[sl]), f32_dev(a[sl]),
+            f32_dev(g), eps=EPS, mix=hc.MIX_SINKHORN_LOGITS if logits else hc.MIX_MATRIX, K=20,
+            read=hc.READ_SOFTMAX_LOGITS if logits else hc.READ_WEIGHTS, y_out=y_out))
+        ys.append(y_out)
+    torch.cuda.synchronize()
+    Hp = np.concatenate([to_host(h, dt) for h in Hs])
+    assert np.array_equal(np.concatenate([to_host(y, dt) for y in ys]), yr)
+    x0 = to_host(xs[0], dt)
+    for q in range(1, R):
+        assert np.array_equal(to_host(xs[q], dt), x0)
+    if logits:
+        assert_close(Hp, Hr, dt, "H'", token_axes=2)
+        assert_close(x0, xr, dt, "x_next")
+    else:
+        assert np.array_equal(Hp, Hr) and np.array_equal(x0, xr)
+
+
+def test_reduce_scatter_rejections(hc):
+    dev = torch.device("cuda")
+    T, n, d, R = 8, 4, 64, 2
+    parts = [torch.zeros((T, d), dtype=torch.bfloat16, device=dev) for _ in range(R)]
+    xs = [torch.zeros((T, d), dtype=torch.bfloat16, device=dev) for _ in range(R)]
+    H = torch.zeros((T // R, n, d), dtype=torch.bfloat16, device=dev)
+    A, b, a = torch.eye(n, device=dev), torch.ones(n, device=dev), torch.ones(n, device=dev) / n
+    with pytest.raises(ValueError):      # H is not this rank's shard
+        hc.reduce_scatter_write_then_read(parts, xs, 0, H[:1], A, b, a)
+    with pytest.raises(hc.HCError) as e:  # two ranks' x buffers are one
+        hc.reduce_scatter_write_then_read(parts, [xs[0], xs[0]], 0, H, A, b, a)
+    assert e.value.status == hc.HC_ERR_ALIAS
+    with pytest.raises(hc.HCError) as e:  # an x buffer is a partial
+        hc.reduce_scatter_write_then_read(parts, [xs[0], parts[1]], 1, H, A, b, a)
+    assert e.value.status == hc.HC_ERR_ALIAS
