@@ -844,7 +844,7 @@ def run_reference(args):
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": w["name"], "T": w["T"], "n": w["n"], "d": w["d"], "K": w["K"],
                    "storage": "bf16", "accumulate": "fp32",
