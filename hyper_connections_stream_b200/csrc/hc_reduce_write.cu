@@ -1,8 +1,8 @@
 // hc_reduce_write.cu -- the write mix fused with the tensor-parallel
 // all-reduce of the block output, then the next layer's read, in one pass.
 //
-// Under tensor parallelism (Hy4-preview model techniques map, "inference
-// kernel": kernel fusion used; the model is served with its layers split over
+// Under tensor parallelism (Hy4-preview model techniques map, the "inference
+// kernel" row: Hy4's kernels are fused and the model is served split over
 // eight GPUs) each of R ranks ends a block with a partial y_r of the block's
 // output and holds a replica of the streams H. Here every rank reads all R
 // partials -- its own from HBM, the others' from peer memory over NVLink --

@@ -143,8 +143,9 @@ HC_API hc_status hc_write_then_read(const void *H, const void *y, void *Hout, vo
 /*
  * The block's output projection fused with the write mix, so the block output
  * y never makes a round trip through HBM (Hy4-preview model techniques map,
- * models.inteligile.com, "inference kernel": kernel fusion used; glossary entry
- * "Hyper-connections (mHC)": the streams are mixed after each block):
+ * models.inteligile.com, the "inference kernel" row, which records that Hy4's
+ * kernels are fused; glossary entry "Hyper-connections (mHC)": the streams are
+ * mixed after each block):
  *   y[t][c]  = bf16( sum_k X[t][k] * Wo[c][k] )   fp32 accumulation on the tensor
  *              cores, rounded to bf16 as a stored y would be;
  *   H'[t][j] = sum_i A[i][j] H[t][i] + b_j y[t]   as hc_write_mix with a given
@@ -165,8 +166,8 @@ HC_API hc_status hc_linear_then_write(const void *X, const void *Wo, const void 
 /*
  * The write mix fused with the tensor-parallel all-reduce of the block output,
  * then the next layer's read (Hy4-preview model techniques map,
- * models.inteligile.com, "inference kernel": kernel fusion used, the model
- * served with its layers split over eight GPUs; glossary entry
+ * models.inteligile.com, the "inference kernel" row: Hy4's kernels are fused
+ * and the model is served split over eight GPUs; glossary entry
  * "Hyper-connections (mHC)": streams mixed after each block). Under tensor
  * parallelism each of R ranks ends the block with a partial output y_r and
  * holds a replica of H; every rank makes this call and reads all R partials:
