@@ -679,7 +679,10 @@ def run_ours(args):
         return total_ms, per_launch, clk.summary()
 
     total_ms, per_launch, clocks = timed()
-    if clocks and BAD_REASONS & set(clocks["reasons"]):
+    # rank 0 alone samples the clocks; every rank takes its decision through one
+    # collective, so all ranks re-measure together (same collectives, same order)
+    bad = 1.0 if clocks and BAD_REASONS & set(clocks["reasons"]) else 0.0
+    if _max_over_ranks(bad, ws, device) > 0:
         total_ms, per_launch, clocks = timed()  # re-measured once
     total_ms = _max_over_ranks(total_ms, ws, device)
     ms_per_step = total_ms / args.steps
