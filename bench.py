@@ -61,8 +61,12 @@ KERNEL_SOURCES = {
                                          "hc_kernels_impl.cuh", "hc_k_bf16_ends.cu"],
     "linear_write_n4_d7168_k7168_bf16_T16384": ["hc_linear_write.cu", "hc_tc.cuh", "hc_sync.cuh"],
     "backward_mhc_n4_d7168_bf16_T16384": ["hc_backward.cu", "hc_device.cuh", "hc_sync.cuh"],
-    "reduce_write_r8_mhc_n4_d7168_bf16_T16384": ["hc_reduce_write.cu", "hc_device.cuh",
-                                                 "hc_launch.h"],
+    "reduce_write_r8_mhc_n4_d7168_bf16_T16384": ["hc_pipe_kernels.cuh", "hc_device.cuh",
+                                                 "hc_sync.cuh", "hc_kernels_impl.cuh",
+                                                 "hc_k_bf16_reduce.cu", "hc_reduce_write.cu"],
+    "reduce_scatter_r8_mhc_n4_d7168_bf16_T16384": ["hc_pipe_kernels.cuh", "hc_device.cuh",
+                                                   "hc_sync.cuh", "hc_kernels_impl.cuh",
+                                                   "hc_k_bf16_reduce.cu", "hc_reduce_write.cu"],
 }
 
 
@@ -180,6 +184,20 @@ def _max_over_ranks(value: float, ws: int, device) -> float:
 def _barrier(ws):
     from hyper_connections_stream_b200 import dist as hd
     hd.barrier(ws)
+
+
+def _gpu_uuid(device):
+    import torch
+    try:
+        return "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+    except Exception:
+        return None
+
+
+def _set_path(args):
+    from hyper_connections_stream_b200 import _lib as hc
+    hc.set_path({"auto": hc.PATH_AUTO, "pipelined": hc.PATH_PIPELINED,
+                 "register": hc.PATH_REGISTER}[args.path])
 
 
 def make_inputs(w, rank, device):
@@ -318,23 +336,36 @@ def run_ends(args):
     }
 
 
-def run_reduce_write(args):
-    """The write fused with the tensor-parallel all-reduce of y
-    (hc_reduce_write_then_read) on the workload's streams: R partial block
-    outputs (default 8, one per rank of a tensor-parallel group, all in this
-    GPU's memory: the same kernel reads them over NVLink when they are peer
-    mappings), summed in rank order, then the fused mHC write + read. Device
-    timed, one launch per step. Also times the unfused pair on the same GPU
-    (torch sum of the partials storing y, then hc_write_then_read)."""
+def run_reduce_write(args, scatter=False):
+    """The write fused with the tensor-parallel all-reduce of y on the
+    workload's streams: R partial block outputs (default 8, one per rank of a
+    tensor-parallel group, all in this GPU's memory: the same kernels read
+    them over NVLink when they are peer mappings), summed in rank order, then
+    the fused mHC write + read. Device timed.
+
+    One-shot form (--op reduce_write, hc_reduce_write_then_read): one launch
+    per step over all T tokens. Unfused pair timed beside it: torch sum of the
+    partials storing y, then hc_write_then_read.
+
+    Reduce-scatter form (--op reduce_scatter, hc_reduce_scatter_write_then_read):
+    the R ranks emulated on this GPU, one launch per rank per step, each over
+    its token shard, storing its rows of x_next into all R ranks' x buffers.
+    A step is all R launches (the whole group's work on one GPU). Unfused
+    group work timed beside it: torch sum of the partials storing y, the
+    fused step over all T tokens, and R - 1 copies of x_next (the
+    all-gather)."""
     import torch
     import hc_inputs as gen
     from hyper_connections_stream_b200 import _lib as hc
     ws, rank, local = _dist_env()
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
+    _set_path(args)
     w = dict(WORKLOAD)
     if args.tokens:
         w["T"] = args.tokens
+    if args.streams:
+        w["n"] = args.streams
     T, n, d, K, R = w["T"], w["n"], w["d"], w["K"], args.ranks
     cfg = w["cfg"]
     s = 2
@@ -348,16 +379,40 @@ def run_reduce_write(args):
     Hout = torch.empty_like(H)
     x = torch.empty((T, d), dtype=torch.bfloat16, device=device)
     kw = dict(eps=w["eps"], mix=hc.MIX_SINKHORN_LOGITS, K=K, read=hc.READ_SOFTMAX_LOGITS)
-
-    def fused():
-        hc.reduce_write_then_read(parts, H, L, b, l, g, out=Hout, x_next=x, **kw)
-
     y = torch.empty((T, d), dtype=torch.bfloat16, device=device)
     stacked = torch.stack(parts)
 
-    def unfused():
-        y.copy_(torch.sum(stacked, 0, dtype=torch.float32))
-        hc.write_then_read(H, y, L, b, l, g, out=Hout, x_next=x, **kw)
+    if scatter:
+        xs = [x] + [torch.empty((T, d), dtype=torch.bfloat16, device=device) for _ in range(R - 1)]
+        shards = []
+        for r in range(R):
+            base, extra = divmod(T, R)
+            t0 = r * base + min(r, extra)
+            sl = slice(t0, t0 + base + (1 if r < extra else 0))
+            shards.append((H[sl], L[sl], l[sl], Hout[sl]))
+
+        def fused():
+            for r, (Hr, Lr, lr, Ho) in enumerate(shards):
+                hc.reduce_scatter_write_then_read(parts, xs, r, Hr, Lr, b, lr, g, out=Ho, **kw)
+
+        def unfused():
+            y.copy_(torch.sum(stacked, 0, dtype=torch.float32))
+            hc.write_then_read(H, y, L, b, l, g, out=Hout, x_next=x, **kw)
+            for q in range(1, R):
+                xs[q].copy_(x)
+        launches = R
+        # per token: R partial rows and n stream rows read, n stream rows and
+        # R x rows (one per rank) written; per launch the gain
+        alg_bytes = T * (d * s * (2 * R + 2 * n) + 4 * (n * n + n)) + R * d * 4
+    else:
+        def fused():
+            hc.reduce_write_then_read(parts, H, L, b, l, g, out=Hout, x_next=x, **kw)
+
+        def unfused():
+            y.copy_(torch.sum(stacked, 0, dtype=torch.float32))
+            hc.write_then_read(H, y, L, b, l, g, out=Hout, x_next=x, **kw)
+        launches = 1
+        alg_bytes = T * (d * s * (R + 2 * n + 1) + 4 * (n * n + n)) + d * 4
 
     stream = torch.cuda.current_stream(device)
 
@@ -374,29 +429,32 @@ def run_reduce_write(args):
         torch.cuda.synchronize()
         return (statistics.mean(a.elapsed_time(e) for a, e in ev), ev[0][0].elapsed_time(ev[-1][1]))
 
-    kern_ms, total_ms = timed(fused, args.steps)
+    with ClockSampler(_gpu_uuid(device)) as clk:
+        kern_ms, total_ms = timed(fused, args.steps)
     unfused_ms, _ = timed(unfused, max(3, args.steps // 4))
-    alg_bytes = T * (d * s * (R + 2 * n + 1) + 4 * (n * n + n)) + d * 4
     peak, peak_kind = _peaks()
     achieved = alg_bytes / (kern_ms / 1e3) / 1e9
+    key = ("reduce_scatter" if scatter else "reduce_write") + "_r8_mhc_n4_d7168_bf16_T16384"
+    form = "reduce-scatter form, R ranks emulated on one GPU" if scatter else "one-shot form"
     return {
-        "metric": f"HC step on the all-reduced block output (R={R} partials) tokens/sec at n={n}, "
-                  f"d={d} (bf16, mHC K={K})",
+        "metric": f"HC step on the all-reduced block output (R={R} partials, {form}) tokens/sec at "
+                  f"n={n}, d={d} (bf16, mHC K={K})",
         "value": T * args.steps / (total_ms / 1e3), "unit": UNIT, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": "reduce_write", "T": T, "n": n, "d": d, "K": K, "ranks": R,
+        "config": {"workload": "reduce_scatter" if scatter else "reduce_write", "T": T, "n": n,
+                   "d": d, "K": K, "ranks": R, "launches_per_step": launches,
                    "partials": "all in this GPU's memory",
                    "l2": "inputs > L2 (re-read from HBM every step)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak,
-                     "traffic": _profiled_traffic("reduce_write_r8_mhc_n4_d7168_bf16_T16384")
-                     if (T, n, R) == (16384, 4, 8) else None,
+                     "traffic": _profiled_traffic(key) if (T, n, R) == (16384, 4, 8) else None,
                      "peak_source": peak_kind,
-                     "algorithmic_bytes_per_launch": alg_bytes, "kernel_ms": kern_ms},
+                     "algorithmic_bytes_per_step": alg_bytes, "kernel_ms": kern_ms},
         "unfused_ms": unfused_ms,
-        "gpu_launches": args.steps, "device_fault": hc.device_fault(),
+        "clocks": clk.summary(),
+        "gpu_launches": args.steps * launches, "device_fault": hc.device_fault(),
     }
 
 
@@ -617,6 +675,240 @@ def run_decode(args):
     }
 
 
+SWEEP_T = (1, 64, 1024, 16384, 65536)
+SWEEP_N = (2, 4, 8)
+SWEEP_D = (4096, 7168)
+L2_BYTES = 126 * 2 ** 20
+
+
+def _slots(bytes_per_call):
+    """Distinct buffer sets cycled through by consecutive calls, so that the
+    calls between two uses of one set touch well over twice the L2."""
+    return int(min(1024, max(1, -(-(3 * L2_BYTES) // max(1, bytes_per_call)))))
+
+
+def _per_call_ms(fn, ncalls, device, warmup=3, graph=False, reps=5):
+    """Mean device time per call of fn(i), i = 0 .. ncalls - 1, with CUDA
+    events on the launching stream around the whole sequence (graph=True:
+    captured once in a CUDA graph and replayed, the median of reps replays,
+    so no host overhead lands between calls)."""
+    import torch
+    stream = torch.cuda.current_stream(device)
+    side = torch.cuda.Stream(device)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for i in range(warmup):
+            fn(i)
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(ncalls):
+                fn(i)
+        g.replay()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b) / ncalls)
+        del g
+        return statistics.median(times)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(ncalls):
+        fn(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / ncalls
+
+
+def _oracle_point_rate(T, n, d, K, eps, seconds=0.25):
+    """Oracle tokens/s (all host cores) on a sample of up to 32 tokens of
+    the point's shape and distributions."""
+    import numpy as np
+    import hc_inputs as gen
+    import oracle
+    S = min(T, 32)
+    H = gen.streams(5, S, n, d, "bf16")
+    y = gen.block_out(5, S, d, "bf16")
+    L = gen.mix_logits(5, S, n)
+    rl = gen.read_logits(5, S, n)
+    _, _, b = gen.static_params(5, n)
+    g = np.ones(d, np.float32)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.write_then_read(H, y, L, b, rl, g, eps, "bf16", K=K, mix_logits=True, read_logits=True)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= seconds:
+            return S * reps / dt, S
+
+
+def run_sweep(args):
+    """Per-point throughput of the fused mHC step (per-token Sinkhorn K=20 and
+    read softmax, bf16) over T x n x d, then the static layer at T=4096, n=4,
+    d=4096 (read, write, the unfused pair and the fused call) and the 78-layer
+    depth stack at T=8192, n=4, d=7168. One JSON line per point / op, device
+    timed; consecutive calls cycle through distinct buffers so the working
+    set between two uses of a buffer exceeds the L2 several times over; calls
+    of T <= 4096 are replayed from a CUDA graph (no host time between them).
+    Each sweep point also carries the oracle's tokens/s on a small sample."""
+    import numpy as np
+    import torch
+    import hc_inputs as gen
+    from hyper_connections_stream_b200 import _lib as hc
+    from hyper_connections_stream_b200 import traffic
+    ws, rank, local = _dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    _set_path(args)
+    peak, peak_kind = _peaks()
+    K, eps = WORKLOAD["K"], WORKLOAD["eps"]
+    bf = torch.bfloat16
+    lines = []
+
+    def point_line(kind, T, n, d, ms, alg, extra):
+        ach = alg / (ms / 1e3) / 1e9
+        line = {"op": kind, "T": T, "n": n, "d": d, "us_per_call": ms * 1e3,
+                "tokens_per_s": T / (ms / 1e3), "algorithmic_bytes_per_call": alg,
+                "achieved_GBs": ach, "frac": ach / peak, "frac_of_8TBs": ach / 8000.0,
+                "peak": peak, "peak_source": peak_kind}
+        line.update(extra)
+        print(json.dumps(line), flush=True)
+        lines.append(line)
+
+    Ts = [args.tokens] if args.tokens else SWEEP_T
+    Ns = [args.streams] if args.streams else SWEEP_N
+    Ds = [args.width] if args.width else SWEEP_D
+    for d in Ds:
+        for n in Ns:
+            for T in Ts:
+                alg = traffic.step_bytes("fused", T, n, d, "bf16", per_token_mix=True,
+                                         per_token_read=True)
+                P = _slots(alg)
+                Hin = gen.device_normal(gen.SEED_H + 5, (P, T, n, d), bf, device)
+                Hout = torch.empty_like(Hin)
+                y = gen.device_normal(gen.SEED_Y + 5, (P, T, d), bf, device)
+                L = gen.device_normal(gen.SEED_L + 5, (P, T, n, n), torch.float32, device)
+                rl = gen.device_normal(gen.SEED_L + 105, (P, T, n), torch.float32, device)
+                x = torch.empty((P, T, d), dtype=bf, device=device)
+                b = torch.from_numpy(gen.static_params(5, n)[2]).to(device)
+                g = torch.ones(d, dtype=torch.float32, device=device)
+
+                def call(i):
+                    j = i % P
+                    hc.write_then_read(Hin[j], y[j], L[j], b, rl[j], g, eps=eps,
+                                       mix=hc.MIX_SINKHORN_LOGITS, K=K,
+                                       read=hc.READ_SOFTMAX_LOGITS, out=Hout[j], x_next=x[j])
+                graph = T <= 4096
+                ncalls = max(P, 64) if graph else max(P, 5 if T >= 65536 else 20)
+                ms = _per_call_ms(call, ncalls, device, graph=graph)
+                small = T * n * d * 2 * 2 < 64 * 2 ** 20
+                orate, S = _oracle_point_rate(T, n, d, K, eps)
+                point_line("sweep_fused_mhc", T, n, d, ms, alg,
+                           {"buffer_sets": P, "calls": ncalls, "graph": graph,
+                            "kernel_family": "register" if (small and args.path == "auto")
+                            else args.path if args.path != "auto" else "pipelined",
+                            "oracle_tokens_per_s": orate, "oracle_sample_tokens": S})
+                del Hin, Hout, y, L, rl, x
+                torch.cuda.empty_cache()
+
+    if not (args.tokens or args.streams or args.width):
+        # static HC layer: T=4096, n=4, d=4096, per-layer a, A, b = identity + N(0, 0.02)
+        T, n, d = 4096, 4, 4096
+        a, A, b = (torch.from_numpy(v).to(device) for v in gen.static_params(2, n))
+        g = torch.ones(d, dtype=torch.float32, device=device)
+        per = {k: traffic.step_bytes(k, T, n, d, "bf16") for k in ("read", "write", "fused")}
+        P = _slots(per["read"])
+        Hs = gen.device_normal(gen.SEED_H + 2, (P, T, n, d), bf, device)
+        Ho = torch.empty_like(Hs)
+        ys = gen.device_normal(gen.SEED_Y + 2, (P, T, d), bf, device)
+        xs = torch.empty((P, T, d), dtype=bf, device=device)
+        ops = {
+            "read": (lambda i: hc.read_rmsnorm(Hs[i % P], a, g, eps=eps, x=xs[i % P]), per["read"]),
+            "write": (lambda i: hc.write_mix(Hs[i % P], ys[i % P], A, b, out=Ho[i % P]),
+                      per["write"]),
+            "unfused_pair": (lambda i: (hc.write_mix(Hs[i % P], ys[i % P], A, b, out=Ho[i % P]),
+                                        hc.read_rmsnorm(Ho[i % P], a, g, eps=eps, x=xs[i % P])),
+                             per["write"] + per["read"]),
+            "fused": (lambda i: hc.write_then_read(Hs[i % P], ys[i % P], A, b, a, g, eps=eps,
+                                                   out=Ho[i % P], x_next=xs[i % P]), per["fused"]),
+        }
+        for name, (fn, alg) in ops.items():
+            ms = _per_call_ms(fn, max(P, 64), device, graph=True)
+            point_line("static_layer_" + name, T, n, d, ms, alg, {"buffer_sets": P})
+        del Hs, Ho, ys, xs
+        torch.cuda.empty_cache()
+
+        # depth stack: 78 layers, T=8192, n=4, d=7168; static per-layer mixing,
+        # gains U(0.5, 1.5); block stand-in y = tanh(x) (torch, not timed as HC)
+        T, n, d, layers = 8192, 4, 7168, 78
+        prm = []
+        for l in range(layers + 1):
+            al, Al, bl = gen.static_params(4, n, layer=l)
+            gl = gen.uniform(gen.SEED_P + 4 + 500 + l, (d,), 0.5, 1.5)
+            prm.append(tuple(torch.from_numpy(v).to(device) for v in (al, Al, bl, gl)))
+        H0 = gen.device_normal(gen.SEED_H + 4, (T, n, d), bf, device)
+        Hb = (torch.empty_like(H0), torch.empty_like(H0))
+        x = torch.empty((T, d), dtype=bf, device=device)
+        yb = torch.empty((T, d), dtype=bf, device=device)
+        stream = torch.cuda.current_stream(device)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(layers + 1)]
+
+        def stack(timed):
+            e = ev[0]
+            if timed:
+                e[0].record(stream)
+            hc.read_rmsnorm(H0, prm[1][0], prm[1][3], eps=eps, x=x)
+            if timed:
+                e[1].record(stream)
+            src = H0
+            for l in range(1, layers + 1):
+                torch.tanh(x, out=yb)
+                dst = Hb[l % 2]
+                e = ev[l]
+                if timed:
+                    e[0].record(stream)
+                if l < layers:
+                    _, Al, bl, _ = prm[l]
+                    an, _, _, gn = prm[l + 1]
+                    hc.write_then_read(src, yb, Al, bl, an, gn, eps=eps, out=dst, x_next=x)
+                else:
+                    hc.write_mix(src, yb, prm[l][1], prm[l][2], out=dst)
+                if timed:
+                    e[1].record(stream)
+                src = dst
+
+        for _ in range(2):
+            stack(False)
+        torch.cuda.synchronize()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        stack(True)
+        s1.record(stream)
+        torch.cuda.synchronize()
+        hc_ms = [a_.elapsed_time(b_) for a_, b_ in ev]
+        stack_ms = s0.elapsed_time(s1)
+        fused_ms = statistics.mean(hc_ms[1:layers])
+        alg = traffic.step_bytes("fused", T, n, d, "bf16")
+        point_line("depth_stack_fused_layer", T, n, d, fused_ms, alg,
+                   {"layers": layers, "stack_hc_ms": sum(hc_ms), "stack_ms_with_tanh": stack_ms,
+                    "stack_tokens_per_s": T / (stack_ms / 1e3),
+                    "stack_hc_tokens_per_s": T / (sum(hc_ms) / 1e3),
+                    "note": "per-layer mean of the 77 fused write->read launches; the stack "
+                            "adds layer 1's read, layer 78's write and 78 torch tanh calls"})
+    if rank == 0:
+        return {"sweep_lines": len(lines), "device_fault": hc.device_fault(),
+                "gpu_launches": None, "peak": peak, "peak_source": peak_kind}
+    return None
+
+
 def run_ours(args):
     import torch
     from hyper_connections_stream_b200 import _lib as hc
@@ -711,11 +1003,7 @@ def run_ours(args):
         "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w["name"], "T": T, "n": n, "d": d, "K": K, "storage": "bf16",
-                   "accumulate": "fp32", "tokens_per_gpu": T, "global_tokens": ws * T,
-                   "parallelism": f"token-sharded x{ws} (no collective)",
-                   "l2": f"inputs larger than L2: {alg_bytes / 1e9:.2f} GB read+written per step "
-                         "vs 126 MB L2; stream state ping-pongs between two buffers"},
+        "config": _step_config(w, ws),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": prof, "peak_source": peak_kind,
                      "algorithmic_bytes_per_launch": alg_bytes, "kernel_ms": kern_ms,
@@ -729,6 +1017,18 @@ def run_ours(args):
     if ws == 1 and not (args.no_cpu_baseline or args.kernel_only):
         line["cpu_baseline"] = cpu_baseline(w, target_s=args.cpu_seconds)
     return line
+
+
+def _step_config(w, ws):
+    """The config dict of the step's line (both arms print the same one)."""
+    from hyper_connections_stream_b200 import traffic
+    T, n, d = w["T"], w["n"], w["d"]
+    alg_bytes = traffic.step_bytes("fused", T, n, d, "bf16", per_token_mix=True, per_token_read=True)
+    return {"workload": w["name"], "T": T, "n": n, "d": d, "K": w["K"], "storage": "bf16",
+            "accumulate": "fp32", "tokens_per_gpu": T, "global_tokens": ws * T,
+            "parallelism": f"token-sharded x{ws} (no collective)",
+            "l2": f"inputs larger than L2: {alg_bytes / 1e9:.2f} GB read+written per step "
+                  "vs 126 MB L2; stream state ping-pongs between two buffers"}
 
 
 def run_e2e(args, inp, w, device, ws):
@@ -806,10 +1106,9 @@ def _oracle_rate(w, S):
     return S / (time.perf_counter() - t0)
 
 
-def cpu_baseline(w, target_s=12.0):
-    """The oracle, as it stands, on the host cores: a bounded token sample of
-    the same workload, stepped repeatedly for about target_s seconds."""
-    import oracle
+def _oracle_timed(w, target_s):
+    """(tokens/s, sample tokens, steps, seconds) of the oracle stepping a
+    bounded token sample of the workload for about target_s seconds."""
     probe = 64
     rate = _oracle_rate(w, probe)
     S = int(max(probe, min(w["T"], rate * target_s)))
@@ -821,9 +1120,27 @@ def cpu_baseline(w, target_s=12.0):
         dt = time.perf_counter() - t0
         if dt >= target_s or reps >= 1000:
             break
-    return {"value": S * reps / dt, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+    return S * reps / dt, S, reps, dt
+
+
+def cpu_baseline(w, target_s=12.0):
+    """The oracle, as it stands, on the host cores: a bounded token sample of
+    the same workload, stepped repeatedly for about target_s seconds, with
+    OpenMP over tokens on every core; then the same on one thread for a
+    quarter of that time."""
+    import oracle
+    cores = oracle.max_threads()
+    value, S, reps, dt = _oracle_timed(w, target_s)
+    oracle.set_threads(1)
+    try:
+        v1, S1, reps1, dt1 = _oracle_timed(w, target_s / 4)
+    finally:
+        oracle.set_threads(cores)
+    return {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{S} of the workload's {w['T']} tokens (same shapes and distributions, "
-                      f"host-generated), {reps} fused step(s), {dt:.1f} s"}
+                      f"host-generated), {reps} fused step(s), {dt:.1f} s",
+            "single_thread": {"value": v1, "unit": UNIT, "cores": 1,
+                              "sample": f"{S1} tokens, {reps1} fused step(s), {dt1:.1f} s"}}
 
 
 def run_reference(args):
@@ -849,11 +1166,10 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": w["name"], "T": w["T"], "n": w["n"], "d": w["d"], "K": w["K"],
-                   "storage": "bf16", "accumulate": "fp32",
-                   "sample_tokens_per_step": S},
+        "config": _step_config(w, ws),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": f"{S} tokens of the {w['T']}-token workload per step"},
+                         "sample": f"{S} tokens of the {w['T']}-token workload per step "
+                                   "(same shapes and distributions, host-generated)"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
@@ -872,14 +1188,17 @@ def main(argv=None):
     ap.add_argument("--kernel-only", action="store_true",
                     help="device-timed kernel only (no e2e, no CPU baseline): for profiling")
     ap.add_argument("--op", choices=["step", "logits", "expand_read", "collapse", "linear_write",
-                                     "reduce_write", "backward", "decode"],
+                                     "reduce_write", "reduce_scatter", "backward", "decode", "sweep"],
                     default="step",
                     help="step: the fused HC step (the metric); logits: the tensor-core "
                          "mixing-logits kernel on the same streams; expand_read / collapse: "
                          "the stack ends on the same shape; linear_write: the block's output "
                          "projection fused with the write; reduce_write: the write fused with "
-                         "the tensor-parallel all-reduce of y (--ranks partials); backward: the "
-                         "step's backward pass; decode: per-call latency of small steps (CUDA graph)")
+                         "the tensor-parallel all-reduce of y (--ranks partials); reduce_scatter: "
+                         "its reduce-scatter form (--ranks ranks emulated on one GPU); backward: the "
+                         "step's backward pass; decode: per-call latency of small steps (CUDA graph); "
+                         "sweep: tokens/s and HBM fraction per T x n x d point, the static layer "
+                         "(read, write, unfused pair, fused) and the 78-layer depth stack")
     ap.add_argument("--path", choices=["auto", "pipelined", "register"], default="auto",
                     help="kernel family (auto = pipelined wherever it applies)")
     ap.add_argument("--ranks", type=int, default=8,
@@ -907,10 +1226,14 @@ def main(argv=None):
         line = run_linear_write(args)
     elif args.op == "reduce_write":
         line = run_reduce_write(args)
+    elif args.op == "reduce_scatter":
+        line = run_reduce_write(args, scatter=True)
     elif args.op == "backward":
         line = run_backward(args)
     elif args.op == "decode":
         line = run_decode(args)
+    elif args.op == "sweep":
+        line = run_sweep(args)
     else:
         line = run_ours(args)
     if line is not None:

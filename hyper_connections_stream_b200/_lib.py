@@ -352,12 +352,14 @@ def _addrs(name, bufs, shape, dtype):
 
 def reduce_scatter_write_then_read(parts, x_all, rank: int, H, A, b, a_next, g_next=None, *,
                                    eps: float = 1e-6, mix: int = MIX_MATRIX, K: int = 0,
-                                   read: int = READ_WEIGHTS, out=None, y_out=None):
+                                   read: int = READ_WEIGHTS, out=None, y_out=None,
+                                   T_total: int | None = None):
     """The reduce-scatter form: H is this rank's token shard [T_r, n, d] of
     the group's streams; parts and x_all list the R ranks' full [T, d] partials
     and x_next buffers (tensors or int device addresses). Reduces the rank's
     rows of the partials, writes its shard of H' (returned) and stores x_next
-    for its rows into every x_all buffer. T is inferred from the buffers."""
+    for its rows into every x_all buffer. T is inferred from the buffers
+    passed as tensors, or given as T_total when all are addresses."""
     _need_cuda("H", H)
     Tr, n, d = _streams_shape(H)
     R = len(parts)
@@ -369,7 +371,12 @@ def reduce_scatter_write_then_read(parts, x_all, rank: int, H, A, b, a_next, g_n
             T = q.shape[0]
             break
     if T is None:
-        raise ValueError("pass at least one partial or x buffer as a tensor (to give T)")
+        T = T_total
+    elif T_total is not None and int(T_total) != T:
+        raise ValueError(f"T_total = {T_total} but the buffers hold {T} rows")
+    if T is None:
+        raise ValueError("pass T_total, or at least one partial or x buffer as a tensor")
+    T = int(T)
     if not 0 <= rank < R:
         raise ValueError("0 <= rank < len(parts)")
     base, extra = divmod(T, R)

@@ -15,22 +15,25 @@ constexpr int kMaxStreams = 8;
 // bounds d of a normalising call at 512 * 8 vectors.
 constexpr int kStreamMaxThreads = 512;
 
-// Step kinds. READ / WRITE / FUSED are the residual step; the last three are
+// Step kinds. READ / WRITE / FUSED are the residual step; the next three are
 // the ends of a stack: EXPAND copies one row into the n streams, EXPAND_READ
 // also produces layer 0's block input from them, COLLAPSE mixes the n
-// streams into one row (no normalisation).
+// streams into one row (no normalisation). REDUCE is FUSED with y the sum of
+// R ranks' partial block outputs (the tensor-parallel all-reduce folded into
+// the write; pipelined family only).
 enum Kind {
     KIND_READ = 0,
     KIND_WRITE = 1,
     KIND_FUSED = 2,
     KIND_EXPAND = 3,
     KIND_EXPAND_READ = 4,
-    KIND_COLLAPSE = 5
+    KIND_COLLAPSE = 5,
+    KIND_REDUCE = 6
 };
 
 // Kinds that normalise a mixed row (a CTA-wide statistic per token).
 __host__ __device__ constexpr bool kind_normalises(int kind) {
-    return kind == KIND_READ || kind == KIND_FUSED || kind == KIND_EXPAND_READ;
+    return kind == KIND_READ || kind == KIND_FUSED || kind == KIND_EXPAND_READ || kind == KIND_REDUCE;
 }
 
 // ---------------------------------------------------------------------------
@@ -109,6 +112,15 @@ __device__ __forceinline__ float2 ffma2_rn(float2 a, float2 b, float2 c) {
         "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
         : "=f"(d.x), "=f"(d.y)
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 fadd2_rn(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
     return d;
 }
 __device__ __forceinline__ float2 fmul2_rn(float2 a, float2 b) {

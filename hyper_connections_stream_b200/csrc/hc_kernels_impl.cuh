@@ -83,16 +83,16 @@ hc_status launch_stream(const StepParams &p, const LaunchCtx &ctx, cudaStream_t 
 
 // ---- pipelined family -------------------------------------------------------------
 
+// Ring geometry for a kind whose stages hold `rows` rows of a tile.
 template <int N, typename S, int KIND>
-bool pipe_shape(const StepParams &p, PipeShape &sh, int &smem) {
+bool pipe_shape(const StepParams &p, int rows, PipeShape &sh, int &smem) {
     constexpr int V = pipe_vec_elems<N, S>();
-    constexpr int ROWS = KIND != KIND_READ ? N + 1 : N;
-    const int64_t d_h = KIND != KIND_WRITE ? p.d : 0;
+    const int64_t d_h = kind_normalises(KIND) ? p.d : 0;
     sh.tile = pipe_group_warps(N) * 32 * V;
     const int64_t ntile = (p.d + sh.tile - 1) / sh.tile;
     if (ntile > (1 << 20)) return false;
     sh.ntile = (int)ntile;
-    sh.stage_bytes = ROWS * sh.tile * (int)sizeof(S);
+    sh.stage_bytes = rows * sh.tile * (int)sizeof(S);
     // one ring per consumer group: the pipelined family needs room for two
     // stages per group; the ring then takes the kind's measured depth
     int64_t per_group = (kSmemLimit - pipe_fixed_bytes(N, 0, d_h)) /
@@ -100,7 +100,8 @@ bool pipe_shape(const StepParams &p, PipeShape &sh, int &smem) {
     if (per_group < 2) return false;
     if (per_group > kMaxStages / kPipeGroups) per_group = kMaxStages / kPipeGroups;
     const int64_t cap = KIND == KIND_WRITE ? HC_PIPE_SG_WRITE
-                        : KIND == KIND_FUSED ? HC_PIPE_SG_FUSED : HC_PIPE_SG_READ;
+                        : KIND == KIND_FUSED ? HC_PIPE_SG_FUSED
+                        : KIND == KIND_REDUCE ? HC_PIPE_SG_REDUCE : HC_PIPE_SG_READ;
     if (per_group > cap) per_group = cap;
     if (per_group < 1) per_group = 1;
     sh.stages = (int)(per_group * kPipeGroups);
@@ -109,8 +110,13 @@ bool pipe_shape(const StepParams &p, PipeShape &sh, int &smem) {
 }
 
 template <int N, typename S, int KIND>
+bool pipe_shape(const StepParams &p, PipeShape &sh, int &smem) {
+    return pipe_shape<N, S, KIND>(p, KIND != KIND_READ ? N + 1 : N, sh, smem);
+}
+
+template <int N, typename S, int KIND>
 hc_status launch_pipe(const StepParams &p, const PipeShape &sh, int smem, const LaunchCtx &ctx,
-                      cudaStream_t st) {
+                      cudaStream_t st, const PipeReduce &rd = PipeReduce{}) {
     auto kern = hc_pipe_kernel<N, S, KIND>;
     static std::atomic<int> configured[64];  // largest dynamic smem opted in so far, per device
     if (ctx.device < 0 || ctx.device >= 64)
@@ -124,7 +130,7 @@ hc_status launch_pipe(const StepParams &p, const PipeShape &sh, int smem, const 
     }
     int64_t grid = ctx.sms;
     if (grid > p.T) grid = p.T;
-    kern<<<(unsigned)grid, pipe_threads(N), smem, st>>>(p, sh, ctx.fault);
+    kern<<<(unsigned)grid, pipe_threads(N), smem, st>>>(p, sh, ctx.fault, rd);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(HC_ERR_CUDA, "hc_pipe_kernel launch: %s", cudaGetErrorString(e));
     return HC_OK;
@@ -160,6 +166,49 @@ hc_status launch_n(const StepParams &p, const LaunchCtx &ctx, cudaStream_t st) {
         return launch_stream<N, S, KIND>(p, ctx, st);
     } else {
         return launch_step_n<N, S, KIND>(p, ctx, st);
+    }
+}
+
+// ---- the fused all-reduce write (KIND_REDUCE), pipelined ------------------------
+
+template <int N, typename S>
+hc_status launch_reduce_pipe_n(const ReduceWriteArgs &ra, const bool *local, const LaunchCtx &ctx,
+                               cudaStream_t st, bool *fits) {
+    static_assert(kPipeMaxRanks == kMaxRanks, "rank limits agree");
+    PipeReduce rd{};
+    int nlocal = 0;
+    for (int r = 0; r < kPipeMaxRanks; ++r) {
+        rd.slot[r] = -1;
+        if (r < ra.R) {
+            rd.parts[r] = ra.parts[r];
+            if (local[r]) rd.slot[r] = N + nlocal++;
+        }
+        if (r < ra.nx) rd.xs[r] = ra.xs[r];
+    }
+    rd.R = ra.R;
+    rd.nx = ra.nx;
+    rd.nlocal = nlocal;
+    rd.y_out = ra.y_out;
+    rd.t0 = ra.t0;
+    PipeShape sh{};
+    int smem = 0;
+    *fits = pipe_shape<N, S, KIND_REDUCE>(ra.f, N + nlocal, sh, smem);
+    if (!*fits) return HC_OK;
+    return launch_pipe<N, S, KIND_REDUCE>(ra.f, sh, smem, ctx, st, rd);
+}
+
+template <typename S>
+hc_status launch_reduce_pipe(const ReduceWriteArgs &ra, const bool *local, const LaunchCtx &ctx,
+                             cudaStream_t st, bool *fits) {
+    switch (ra.n) {
+        case 1: return launch_reduce_pipe_n<1, S>(ra, local, ctx, st, fits);
+        case 2: return launch_reduce_pipe_n<2, S>(ra, local, ctx, st, fits);
+        case 3: return launch_reduce_pipe_n<3, S>(ra, local, ctx, st, fits);
+        case 4: return launch_reduce_pipe_n<4, S>(ra, local, ctx, st, fits);
+        case 5: return launch_reduce_pipe_n<5, S>(ra, local, ctx, st, fits);
+        case 6: return launch_reduce_pipe_n<6, S>(ra, local, ctx, st, fits);
+        case 7: return launch_reduce_pipe_n<7, S>(ra, local, ctx, st, fits);
+        default: return launch_reduce_pipe_n<8, S>(ra, local, ctx, st, fits);
     }
 }
 

@@ -82,6 +82,12 @@ struct ReduceWriteArgs {
 };
 hc_status launch_reduce_write(const ReduceWriteArgs &ra, hc_dtype dt, const LaunchCtx &ctx,
                               cudaStream_t st);
+// Its pipelined (TMA-fed) form; local[r] marks partials in this GPU's memory
+// (staged by bulk copies; the others are read with plain loads). Launches
+// nothing and sets *fits = false when the ring does not fit shared memory.
+template <typename S>
+hc_status launch_reduce_pipe(const ReduceWriteArgs &ra, const bool *local, const LaunchCtx &ctx,
+                             cudaStream_t st, bool *fits);
 
 hc_status launch_selftest_wait(int limit_us, const LaunchCtx &ctx, cudaStream_t st);
 

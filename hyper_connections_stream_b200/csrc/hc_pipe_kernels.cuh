@@ -13,6 +13,11 @@
 //               stages, writes H' with coalesced 128-bit stores, keeps h in an
 //               fp32 shared-memory row, reduces the fp64 sum of squares across
 //               its warps, then stores x.
+// KIND_REDUCE is the fused step with y the sum of R ranks' partial block
+// outputs: a stage holds the n stream rows and the partial rows that are in
+// this GPU's memory (bulk copies); partials in a peer's memory are read by
+// the consumers with plain loads. The partials are added in rank order in
+// fp32 and rounded once, so y is bit-identical on every rank.
 // Every consumer group has its own ring of stages and its own parameter
 // slots, so each mbarrier has exactly one consumer taking its phases in
 // order (a parity wait is never more than one phase ahead). The producer
@@ -56,6 +61,10 @@ namespace hc {
 #ifndef HC_PIPE_SG_READ
 #define HC_PIPE_SG_READ 16
 #endif
+// The reduce kind reads R partial rows per tile besides the n stream rows.
+#ifndef HC_PIPE_SG_REDUCE
+#define HC_PIPE_SG_REDUCE 4
+#endif
 constexpr int kPipeGroups = HC_PIPE_GROUPS;
 // Consumer warps per group: fewer for n > 4, so that each thread has the
 // registers to hold n widened 16-byte rows (launch bounds give 65536 /
@@ -94,10 +103,25 @@ struct PipeShape {
     int stage_bytes;  // bytes of one stage
 };
 
+// Extra arguments of KIND_REDUCE (unused by the other kinds).
+constexpr int kPipeMaxRanks = 8;
+struct PipeReduce {
+    const void *parts[kPipeMaxRanks];  // partial y of each rank, rows t0 .. t0 + T - 1 used
+    void *xs[kPipeMaxRanks];           // x_next destinations, same rows
+    void *y_out;                       // reduced y [T][d] of this call's tokens, or null
+    int64_t t0;                        // row of the partials and of x for token 0
+    int R;                             // ranks
+    int nx;                            // x destinations
+    int nlocal;                        // partials staged by bulk copies
+    int slot[kPipeMaxRanks];           // stage row of rank r's partial, -1: plain loads
+};
+
 // Bytes of everything in shared memory other than the ring: barriers,
 // parameter slots, reduction partials, the abort flag and, for the
-// normalising kinds, two fp32 rows h[d] per group (d_h = d, else 0): the
-// current token's and the previous token's, whose x is written meanwhile.
+// normalising kinds, one fp32 row h[d] per group (d_h = d, else 0). The row
+// serves two tokens at once: a thread reads back only its own slice
+// positions, so at each tile it first reads the previous token's h there (for
+// that token's x) and then overwrites it with the current token's.
 __host__ __device__ constexpr int64_t pipe_fixed_bytes(int n, int stages, int64_t d_h) {
     return (int64_t)stages * 16                        // full + empty barriers
            + kPipeGroups * pipe_param_slots_per_group(n) * 16  // param full + empty
@@ -106,7 +130,7 @@ __host__ __device__ constexpr int64_t pipe_fixed_bytes(int n, int stages, int64_
            + kPipeGroups * 2 * pipe_group_warps(n) * 8  // reduction partials
            + 16                                        // abort flag (padded)
            + pipe_param_replicas(n) * kGroupScratch * 4  // parameter warp scratch
-           + (int64_t)kPipeGroups * 2 * ((d_h * 4 + 15) / 16 * 16);  // h rows (2 per group)
+           + (int64_t)kPipeGroups * ((d_h * 4 + 15) / 16 * 16);  // h rows (1 per group)
 }
 
 // Elements of d one consumer thread handles per tile: one 16-byte vector
@@ -125,6 +149,12 @@ template <> struct VecIO<float, 4> {
         v[0] = make_float2(q.x, q.y);
         v[1] = make_float2(q.z, q.w);
     }
+    static __device__ __forceinline__ void load_global(const float *p, float2 (&v)[2]) {
+        const float4 q = __ldcs(reinterpret_cast<const float4 *>(p));
+        v[0] = make_float2(q.x, q.y);
+        v[1] = make_float2(q.z, q.w);
+    }
+    static __device__ __forceinline__ void round(float2 (&)[2]) {}
     static __device__ __forceinline__ void store(float *p, const float2 (&v)[2], float2 (&stored)[2]) {
         __stcs(reinterpret_cast<float4 *>(p), make_float4(v[0].x, v[0].y, v[1].x, v[1].y));
         stored[0] = v[0];
@@ -146,6 +176,17 @@ template <> struct VecIO<__nv_bfloat16, 8> {
         v[1] = widen_pair(q.y);
         v[2] = widen_pair(q.z);
         v[3] = widen_pair(q.w);
+    }
+    static __device__ __forceinline__ void load_global(const __nv_bfloat16 *p, float2 (&v)[4]) {
+        const uint4 q = __ldcs(reinterpret_cast<const uint4 *>(p));
+        v[0] = widen_pair(q.x);
+        v[1] = widen_pair(q.y);
+        v[2] = widen_pair(q.z);
+        v[3] = widen_pair(q.w);
+    }
+    static __device__ __forceinline__ void round(float2 (&v)[4]) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = widen_pair(pack_bf16x2_rn(v[e].x, v[e].y));
     }
     static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float2 (&v)[4],
                                                  float2 (&stored)[4]) {
@@ -175,6 +216,15 @@ template <> struct VecIO<__nv_bfloat16, 4> {
         v[0] = widen_pair(q.x);
         v[1] = widen_pair(q.y);
     }
+    static __device__ __forceinline__ void load_global(const __nv_bfloat16 *p, float2 (&v)[2]) {
+        const uint2 q = __ldcs(reinterpret_cast<const uint2 *>(p));
+        v[0] = widen_pair(q.x);
+        v[1] = widen_pair(q.y);
+    }
+    static __device__ __forceinline__ void round(float2 (&v)[2]) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) v[e] = widen_pair(pack_bf16x2_rn(v[e].x, v[e].y));
+    }
     static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float2 (&v)[2],
                                                  float2 (&stored)[2]) {
         uint2 q;
@@ -194,13 +244,14 @@ template <> struct VecIO<__nv_bfloat16, 4> {
 
 template <int N, typename S, int KIND>
 __global__ void __launch_bounds__(pipe_threads(N), 1)
-hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
+hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
     constexpr int V = pipe_vec_elems<N, S>();
     constexpr int VB = V * (int)sizeof(S);  // bytes per thread per row of a tile
     constexpr int NN = N * N;
     constexpr bool WRITE = KIND != KIND_READ;
     constexpr bool READ = KIND != KIND_WRITE;
-    constexpr int ROWS = WRITE ? N + 1 : N;
+    constexpr bool REDUCE = KIND == KIND_REDUCE;
+    const int ROWS = REDUCE ? N + rd.nlocal : WRITE ? N + 1 : N;
     constexpr int PSTRIDE = NN + 2 * N;  // A transposed (column j at j*N) | b | a
     constexpr int GW = pipe_group_warps(N);
     constexpr int NG = kPipeGroups;
@@ -291,7 +342,16 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
                 const S *src = H + t * N * d + k0;
 #pragma unroll
                 for (int i = 0; i < N; ++i) load(st + i * row_bytes, src + i * d, rb, &full[s]);
-                if constexpr (WRITE) load(st + N * row_bytes, Y + t * d + k0, rb, &full[s]);
+                if constexpr (REDUCE) {
+                    const int64_t off = (rd.t0 + t) * d + k0;
+#pragma unroll
+                    for (int q = 0; q < kPipeMaxRanks; ++q)
+                        if (q < rd.R && rd.slot[q] >= 0)
+                            load(st + rd.slot[q] * row_bytes, static_cast<const S *>(rd.parts[q]) + off,
+                                 rb, &full[s]);
+                } else if constexpr (WRITE) {
+                    load(st + N * row_bytes, Y + t * d + k0, rb, &full[s]);
+                }
                 ++nq[r];
                 if (++slot_r[r] == SG) {
                     slot_r[r] = 0;
@@ -424,6 +484,8 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
     // token i-1's x, one tile after each of token i's tiles: a warp arrives at
     // the group reduction of token i-1 and goes on to token i's first tile
     // before it waits for the other warps' sums, so the wait overlaps work.
+    // Both tokens share the group's h row: at each tile a thread reads token
+    // i-1's h at its own slice positions before it stores token i's there.
     const int cw = warp - 2;
     const int g = cw / GW;
     const int gw = cw - g * GW;
@@ -431,12 +493,14 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
     uint64_t *gfull = full + g * SG;
     uint64_t *gempty = empty + g * SG;
     unsigned char *gring = ring + (size_t)g * SG * sh.stage_bytes;
+    float *hrow = hrow_base + g * hrow_stride;
     S *Ho = static_cast<S *>(p.Hout);
     S *X = static_cast<S *>(p.x);
     int slot = 0;      // ring position of this group's next tile
     uint32_t ph = 0;   // its phase parity
     const int64_t Mg = M > g ? (M - 1 - g) / NG + 1 : 0;  // tokens of this group
     float r_prev = 0.0f;
+    constexpr int VP = V / 2;  // element pairs per thread
 
     for (int64_t i = 0; i <= Mg; ++i) {
         const bool cur = i < Mg;                 // token i to mix
@@ -444,8 +508,6 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
         const int64_t m = g + i * NG;
         const int64_t t = blockIdx.x + m * G;
         const int64_t t_prev = t - (int64_t)NG * G;
-        float *hcur = hrow_base + (g * 2 + (int)(i & 1)) * hrow_stride;
-        const float *hprev = hrow_base + (g * 2 + (int)((i + 1) & 1)) * hrow_stride;
         const int ps = g * PSG + (int)(i % PSG);
         float bv[N], av[N];
         const float *P = params + ps * PSTRIDE;
@@ -465,6 +527,7 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
         for (int j = 0; j < ntile; ++j) {
             const int64_t k = (int64_t)j * tile + (int64_t)gt * V;
             const bool active = k < d;
+            float2 hr[VP];  // token i's h at this thread's slice of tile j
             if (cur) {
                 const int cs = slot;
                 const bool w = mbar_wait_bounded(&gfull[cs], ph, abort_flag, fault, FAULT_WAIT_FULL);
@@ -477,17 +540,48 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
                     ph ^= 1u;
                 }
                 const unsigned char *st = gring + (size_t)cs * sh.stage_bytes + (size_t)gt * VB;
-                constexpr int VP = V / 2;  // element pairs per thread
                 float2 h[N][VP], yv[VP];
                 if (active) {
 #pragma unroll
                     for (int ii = 0; ii < N; ++ii) VecIO<S, V>::load_smem(st + ii * row_bytes, h[ii]);
-                    if constexpr (WRITE) VecIO<S, V>::load_smem(st + N * row_bytes, yv);
+                    if constexpr (REDUCE) {
+                        // the all-reduce of y: partials added in rank order
+                        const int64_t off = (rd.t0 + t) * d + k;
+#pragma unroll
+                        for (int q = 0; q < kPipeMaxRanks; ++q) {
+                            if (q < rd.R) {
+                                float2 pv[VP];
+                                if (rd.slot[q] >= 0)
+                                    VecIO<S, V>::load_smem(st + rd.slot[q] * row_bytes, pv);
+                                else
+                                    VecIO<S, V>::load_global(static_cast<const S *>(rd.parts[q]) + off, pv);
+                                if (q == 0) {
+#pragma unroll
+                                    for (int e = 0; e < VP; ++e) yv[e] = pv[e];
+                                } else {
+#pragma unroll
+                                    for (int e = 0; e < VP; ++e) yv[e] = fadd2_rn(yv[e], pv[e]);
+                                }
+                            }
+                        }
+                    } else if constexpr (WRITE) {
+                        VecIO<S, V>::load_smem(st + N * row_bytes, yv);
+                    }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&gempty[cs]);  // stage data is in registers
                 if (active) {
-                    float2 hr[VP];
+                    if constexpr (REDUCE) {
+                        // one rounding to the storage dtype (what a stored y holds)
+                        if (rd.y_out) {
+                            float2 stored[VP];
+                            VecIO<S, V>::store(static_cast<S *>(rd.y_out) + t * d + k, yv, stored);
+#pragma unroll
+                            for (int e = 0; e < VP; ++e) yv[e] = stored[e];
+                        } else {
+                            VecIO<S, V>::round(yv);
+                        }
+                    }
                     if constexpr (WRITE) {
                         S *Hot = Ho + t * N * d + k;
 #pragma unroll
@@ -539,11 +633,6 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
                             ss = __fma_rn(hx, hx, ss);
                             ss = __fma_rn(hy, hy, ss);
                         }
-                        // keep h for the normalisation (this thread reads it back itself)
-#pragma unroll
-                        for (int e = 0; e < VP; e += 2)
-                            *reinterpret_cast<float4 *>(hcur + k + 2 * e) =
-                                make_float4(hr[e].x, hr[e].y, hr[e + 1].x, hr[e + 1].y);
                     }
                 }
             }
@@ -564,13 +653,12 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
                         r_prev = __double2float_rn(1.0 / sqrt(tot / (double)d + (double)p.eps));
                     }
                     if (active) {
-                        constexpr int VP = V / 2;
                         float gv[V];
                         float2 hv[VP], xv[VP];
                         load_gain<V>(p.g, k, gv);
 #pragma unroll
                         for (int e = 0; e < VP; e += 2) {
-                            const float4 f = *reinterpret_cast<const float4 *>(hprev + k + 2 * e);
+                            const float4 f = *reinterpret_cast<const float4 *>(hrow + k + 2 * e);
                             hv[e] = make_float2(f.x, f.y);
                             hv[e + 1] = make_float2(f.z, f.w);
                         }
@@ -578,8 +666,24 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault) {
 #pragma unroll
                         for (int e = 0; e < VP; ++e)
                             xv[e] = fmul2_rn(fmul2_rn(hv[e], r2), make_float2(gv[2 * e], gv[2 * e + 1]));
-                        VecIO<S, V>::store(X + t_prev * d + k, xv);
+                        if constexpr (REDUCE) {
+                            // x_next to every destination (the all-gather of the
+                            // reduce-scatter form: peers' buffers take plain stores)
+                            const int64_t off = (rd.t0 + t_prev) * d + k;
+#pragma unroll
+                            for (int q = 0; q < kPipeMaxRanks; ++q)
+                                if (q < rd.nx) VecIO<S, V>::store(static_cast<S *>(rd.xs[q]) + off, xv);
+                        } else {
+                            VecIO<S, V>::store(X + t_prev * d + k, xv);
+                        }
                     }
+                }
+                // keep token i's h for its normalisation (after token i-1's read above)
+                if (cur && active) {
+#pragma unroll
+                    for (int e = 0; e < VP; e += 2)
+                        *reinterpret_cast<float4 *>(hrow + k + 2 * e) =
+                            make_float4(hr[e].x, hr[e].y, hr[e + 1].x, hr[e + 1].y);
                 }
             }
         }

@@ -21,15 +21,21 @@
 // only, writes its shard of H', and stores that shard's x_next into every
 // rank's x buffer (the all-gather, as plain stores to peer memory).
 //
-// The kernel reads and writes peer memory with plain loads and stores (no
-// TMA, no multicast) and never waits on another rank: the caller orders each
+// Peer memory is read and written with plain loads and stores only (bulk
+// copies, never multicast, read this GPU's own memory), and no kernel ever
+// waits on another rank: the caller orders each
 // partial's writes before the call, and every later read of x or overwrite
 // of a partial after every rank's call (the host layer does this with two
 // barriers). With buffers of one GPU it is the same computation over all
 // ranks' data, one launch per rank.
 //
-// One CTA per token at a time (grid-stride), threads own 16-byte column
-// slices; h stays in registers until the CTA's fp64 sum of squares is known.
+// Two kernel families, as for the step: the pipelined one (hc_pipe_kernel,
+// KIND_REDUCE: bulk copies of the stream rows and of the local partial rows
+// into shared-memory rings, warp-specialised) for large calls, and the
+// register-streaming one below for decode-sized calls and shapes whose ring
+// does not fit: one CTA per token at a time (grid-stride), threads own
+// 16-byte column slices, and h stays in registers until the CTA's fp64 sum
+// of squares is known.
 #include "hc_launch.h"
 
 namespace hc {
@@ -246,6 +252,32 @@ hc_status rw_dispatch(const ReduceWriteArgs &ra, const LaunchCtx &ctx, cudaStrea
 
 hc_status launch_reduce_write(const ReduceWriteArgs &ra, hc_dtype dt, const LaunchCtx &ctx,
                               cudaStream_t st) {
+    // Decode-sized calls (under ~64 MiB of stream traffic) skip the pipeline's
+    // set-up, as the step kinds do; hc_set_path forces either family.
+    const int64_t es = dt == HC_BF16 ? 2 : 4;
+    const bool small = ra.f.T * (int64_t)ra.n * ra.f.d * es * 2 < (int64_t(64) << 20);
+    if (ctx.path == 1 || (ctx.path == 0 && !small)) {
+        // partials in this GPU's own memory are staged by bulk copies; any
+        // other (a peer's memory, or memory the runtime cannot place) takes
+        // plain loads
+        bool local[kMaxRanks] = {};
+        for (int r = 0; r < ra.R; ++r) {
+            cudaPointerAttributes at{};
+            const cudaError_t e = cudaPointerGetAttributes(&at, ra.parts[r]);
+            if (e != cudaSuccess) {
+                (void)cudaGetLastError();  // not a device pointer the runtime knows: plain loads
+                continue;
+            }
+            local[r] = at.type == cudaMemoryTypeDevice && at.device == ctx.device;
+        }
+        bool fits = false;
+        const hc_status s = dt == HC_BF16 ? launch_reduce_pipe<__nv_bfloat16>(ra, local, ctx, st, &fits)
+                                          : launch_reduce_pipe<float>(ra, local, ctx, st, &fits);
+        if (s != HC_OK || fits) return s;
+        if (ctx.path == 1)
+            return set_error(HC_ERR_UNSUPPORTED, "pipelined kernels do not cover d = %lld with R = %d here",
+                             (long long)ra.f.d, ra.R);
+    }
     return dt == HC_BF16 ? rw_dispatch<__nv_bfloat16>(ra, ctx, st) : rw_dispatch<float>(ra, ctx, st);
 }
 

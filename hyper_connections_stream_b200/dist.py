@@ -76,6 +76,7 @@ class PeerPartials:
             open_ = open_ or hc.ipc_open
             close = close or hc.ipc_close
         self._close = close
+        self.local = local
         self.rank = dist.get_rank(group)
         self.world = dist.get_world_size(group)
         handle, offset = export(local)
@@ -140,6 +141,11 @@ def reduce_scatter_step(peers_y: PeerPartials, peers_x: PeerPartials, H_shard, A
         call = hc.reduce_scatter_write_then_read
     if sync is None:
         sync = lambda: torch.cuda.current_stream().synchronize()  # noqa: E731
+    # the pointer lists are plain addresses: the group's token count comes
+    # from this rank's own partial buffer
+    shape = getattr(peers_y.local, "shape", None)
+    if shape is not None:
+        kw.setdefault("T_total", int(shape[0]))
     sync()
     dist.barrier(group)
     out = call(peers_y.pointers, peers_x.pointers, peers_y.rank, H_shard, A, b, a_next, g_next, **kw)

@@ -279,19 +279,25 @@ HC_API size_t hc_write_then_read_backward_workspace_bytes(hc_dtype dt, int64_t T
 
 /*
  * hc_write_then_read_backward without a workspace argument: the pages have no
- * counterpart to this; it is an interface convenience of this library. The
- * gain gradient's per-CTA partials go to a 16 MiB scratch array that lives in
- * the library's device image (one per device); the call allocates nothing.
+ * counterpart to this; it is an interface addition of this library for
+ * callers that cannot allocate device memory when they call it -- runtimes
+ * that reserve a GPU's memory up front in their own pool and have no buffer
+ * to lend, and latency-critical loops where cudaMalloc, which can synchronise
+ * the device, is not acceptable. The gain gradient's per-CTA partials go to a
+ * 16 MiB scratch array that lives in the library's device image (one per
+ * device, held until the process exits); the call allocates nothing.
  * Arguments and results are those of hc_write_then_read_backward.
- *   - Calls needing more than 16 MiB of partials (more SMs x d x 4 bytes)
- *     return HC_ERR_UNSUPPORTED without launching anything.
+ *   - The partials take hc_write_then_read_backward_workspace_bytes(dt, T, n,
+ *     d) bytes; a call with dg fits when that is at most 16 MiB (16777216).
+ *     Larger calls return HC_ERR_UNSUPPORTED without launching anything; use
+ *     the workspace form for them. Invalid arguments get the statuses of
+ *     hc_write_then_read_backward.
  *   - The scratch is shared by every call on a device: two calls whose
  *     executions overlap (different streams without ordering between them)
  *     race on it and corrupt dg. Order such calls, or use the workspace form.
  *   - The first call on a device (with dg) looks the scratch address up on
- *     the host (cudaGetSymbolAddress) and sets kernel attributes; make one
- *     call before capturing work into a graph if that setup must not happen
- *     during capture.
+ *     the host (cudaGetSymbolAddress, with that device current) and sets
+ *     kernel attributes; make that first call before any stream capture.
  *   - No part of the scratch has to start at zero.
  */
 HC_API hc_status hc_write_then_read_backward_noalloc(

@@ -27,6 +27,8 @@ def test_reference_arm_prints_one_complete_line():
     assert (d["n_gpus"], d["steps"], d["warmup"]) == (1, 1, 3)
     assert d["dtype"] == "bf16" and d["data"] == "synthetic" and d["vs_baseline"] is None
     assert d["config"]["workload"] and (d["config"]["n"], d["config"]["d"]) == (4, 7168)
+    # the same config dict as the product arm prints
+    assert d["config"] == bench._step_config(bench.WORKLOAD, 1)
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,

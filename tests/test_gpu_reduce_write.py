@@ -7,6 +7,12 @@ waits on another rank, so one GPU runs the whole computation of every rank.
 The oracle sums the partials in rank order in fp32, rounds once, and runs its
 fused step on that y.
 
+Every case runs under each kernel family (chosen by size, pipelined, register
+streaming). The pipelined kernel stages partials in this GPU's memory with
+bulk copies and reads any other partial with plain loads; a case with some
+partials in managed memory (which the library does not stage) covers the
+plain-load branch on one GPU.
+
 Bars: y bit-exact always (no parameter enters it); H' and x_next bit-exact
 with the matrix and weights given (the same fp32 chains on both sides); with
 Sinkhorn and softmax logits within the fused step's bars (2e-2 bf16 / 1e-5
@@ -28,17 +34,22 @@ pytestmark = pytest.mark.gpu
 EPS = 1e-6
 
 
-@pytest.fixture(scope="module")
-def hc():
+@pytest.fixture(scope="module", params=["auto", "pipelined", "register"])
+def hc(request):
+    """The binding with the kernel family chosen by call size, or forced to the
+    pipelined (bulk-copy rings) or the register-streaming kernel."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from hyper_connections_stream_b200 import build
     build.build()
     import hyper_connections_stream_b200._lib as L
     L.lib()
+    L.set_path({"auto": L.PATH_AUTO, "pipelined": L.PATH_PIPELINED,
+                "register": L.PATH_REGISTER}[request.param])
     yield L
     torch.cuda.synchronize()
     assert L.device_fault() == 0
+    L.set_path(L.PATH_AUTO)
 
 
 def _case(T, n, d, R, dt, logits, per_token, seed):
@@ -157,6 +168,59 @@ def test_full_size_sampled(hc):
     assert_close(Hs, Hr, dt, "H'", token_axes=2)
     assert_close(to_host(x[it], dt), xr, dt, "x_next")
     assert np.mean(Hs == Hr) > 0.999
+
+
+class _Managed:
+    """A [T, d] buffer in CUDA managed memory (device-accessible, but not
+    device memory of this GPU, so the library reads it with plain loads)."""
+
+    def __init__(self, src: torch.Tensor):
+        from cuda.bindings import runtime as rt
+        self._rt = rt
+        self.bytes = src.numel() * src.element_size()
+        err, self.ptr = rt.cudaMallocManaged(self.bytes, rt.cudaMemAttachGlobal)
+        assert err == rt.cudaError_t.cudaSuccess, err
+        torch.cuda.synchronize()
+        err, = rt.cudaMemcpy(self.ptr, src.data_ptr(), self.bytes, rt.cudaMemcpyKind.cudaMemcpyDefault)
+        assert err == rt.cudaError_t.cudaSuccess, err
+
+    def free(self):
+        torch.cuda.synchronize()
+        err, = self._rt.cudaFree(self.ptr)
+        assert err == self._rt.cudaError_t.cudaSuccess, err
+
+
+@pytest.mark.parametrize("T,n,d,R,dt,logits,managed", [
+    (600, 4, 7168, 8, "bf16", True, (1, 4, 7)),
+    (400, 2, 2048, 3, "f32", False, (0,)),
+    (700, 8, 1032, 5, "bf16", False, (0, 1, 2, 3, 4)),
+])
+def test_partials_read_with_plain_loads(hc, T, n, d, R, dt, logits, managed):
+    """Partials outside this GPU's device memory (here managed memory, as a
+    peer mapping would be) take the consumers' plain-load branch, in rank
+    order with the staged ones: same bits as the oracle."""
+    parts, H, A, b, a, g = _case(T, n, d, R, dt, logits, True, seed=3600 + T + R)
+    dparts = [to_dev(p, dt) for p in parts]
+    held = {r: _Managed(dparts[r]) for r in managed}
+    try:
+        mixed = [held[r].ptr if r in held else dparts[r] for r in range(R)]
+        y_out = torch.empty((T, d), dtype=TORCH_DT[dt], device="cuda")
+        Hp, x = hc.reduce_write_then_read(
+            mixed, to_dev(H, dt), f32_dev(A), f32_dev(b), f32_dev(a), f32_dev(g), eps=EPS,
+            mix=hc.MIX_SINKHORN_LOGITS if logits else hc.MIX_MATRIX, K=20,
+            read=hc.READ_SOFTMAX_LOGITS if logits else hc.READ_WEIGHTS, y_out=y_out)
+        torch.cuda.synchronize()
+    finally:
+        for m in held.values():
+            m.free()
+    Hr, xr, yr = oracle.reduce_write_then_read(parts, H, A, b, a, g, EPS, dt, K=20,
+                                               mix_logits=logits, read_logits=logits)
+    assert np.array_equal(to_host(y_out, dt), yr)
+    if logits:
+        assert_close(to_host(Hp, dt), Hr, dt, "H'", token_axes=2)
+        assert_close(to_host(x, dt), xr, dt, "x_next")
+    else:
+        assert np.array_equal(to_host(Hp, dt), Hr) and np.array_equal(to_host(x, dt), xr)
 
 
 def test_rejections(hc):
