@@ -60,7 +60,9 @@ KERNEL_SOURCES = {
     "expand_read_n4_d7168_bf16_T16384": ["hc_stream_kernels.cuh", "hc_device.cuh",
                                          "hc_kernels_impl.cuh", "hc_k_bf16_ends.cu"],
     "linear_write_n4_d7168_k7168_bf16_T16384": ["hc_linear_write.cu", "hc_tc.cuh", "hc_sync.cuh"],
-    "backward_mhc_n4_d7168_bf16_T16384": ["hc_backward.cu", "hc_device.cuh", "hc_sync.cuh"],
+    "backward_mhc_n4_d7168_bf16_T16384": ["hc_backward.cu", "hc_backward_pipe.cuh",
+                                          "hc_backward_common.cuh", "hc_pipe_kernels.cuh",
+                                          "hc_device.cuh", "hc_sync.cuh"],
     "reduce_write_r8_mhc_n4_d7168_bf16_T16384": ["hc_pipe_kernels.cuh", "hc_device.cuh",
                                                  "hc_sync.cuh", "hc_kernels_impl.cuh",
                                                  "hc_k_bf16_reduce.cu", "hc_reduce_write.cu"],
@@ -558,6 +560,7 @@ def run_backward(args):
     ws, rank, local = _dist_env()
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
+    _set_path(args)
     w = dict(WORKLOAD)
     if args.tokens:
         w["T"] = args.tokens
@@ -587,11 +590,12 @@ def run_backward(args):
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
-    for i in range(args.steps):
-        ev[i][0].record(stream)
-        step()
-        ev[i][1].record(stream)
-    torch.cuda.synchronize()
+    with ClockSampler(_gpu_uuid(device)) as clk:
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
     step_ms = statistics.mean(s_.elapsed_time(e) for s_, e in ev)
     total_ms = ev[0][0].elapsed_time(ev[-1][1])
     s = 2
@@ -613,6 +617,7 @@ def run_backward(args):
                      if (T, n) == (16384, 4) else None,
                      "peak_source": peak_kind,
                      "algorithmic_bytes_per_step": alg_bytes, "step_ms": step_ms},
+        "clocks": clk.summary(), "kernel_path": args.path,
         "gpu_launches": 3 * args.steps, "device_fault": hc.device_fault(),
     }
 

@@ -95,7 +95,9 @@ bool pipe_shape(const StepParams &p, int rows, PipeShape &sh, int &smem) {
     sh.stage_bytes = rows * sh.tile * (int)sizeof(S);
     // one ring per consumer group: the pipelined family needs room for two
     // stages per group; the ring then takes the kind's measured depth
-    int64_t per_group = (kSmemLimit - pipe_fixed_bytes(N, 0, d_h)) /
+    constexpr int srows = N + (KIND == KIND_FUSED ? 1 : 0);
+    const int64_t st_bytes = KIND == KIND_READ ? 0 : pipe_store_bytes(N, srows, V * (int)sizeof(S));
+    int64_t per_group = (kSmemLimit - pipe_fixed_bytes(N, 0, d_h) - st_bytes) /
                         ((int64_t)kPipeGroups * (sh.stage_bytes + 16));
     if (per_group < 2) return false;
     if (per_group > kMaxStages / kPipeGroups) per_group = kMaxStages / kPipeGroups;
@@ -105,7 +107,7 @@ bool pipe_shape(const StepParams &p, int rows, PipeShape &sh, int &smem) {
     if (per_group > cap) per_group = cap;
     if (per_group < 1) per_group = 1;
     sh.stages = (int)(per_group * kPipeGroups);
-    smem = (int)((int64_t)sh.stages * sh.stage_bytes + pipe_fixed_bytes(N, sh.stages, d_h));
+    smem = (int)((int64_t)sh.stages * sh.stage_bytes + pipe_fixed_bytes(N, sh.stages, d_h) + st_bytes);
     return true;
 }
 

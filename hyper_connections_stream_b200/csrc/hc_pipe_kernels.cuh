@@ -48,6 +48,18 @@ namespace hc {
 #ifndef HC_PIPE_L2_HINT
 #define HC_PIPE_L2_HINT 0
 #endif
+// 1: consumer warps stage their rounded H' (and x) slices in shared memory
+// and write them with bulk copies (cp.async.bulk shared -> global) instead of
+// 16-byte register stores.
+#ifndef HC_PIPE_TMA_STORE
+#define HC_PIPE_TMA_STORE 0
+#endif
+// 1: the parameter warp projects its first batch with shuffle exchanges
+// (shortest latency; the consumers wait on it), later batches through shared
+// memory (highest throughput).
+#ifndef HC_PIPE_FIRST_SHFL
+#define HC_PIPE_FIRST_SHFL 0
+#endif
 // Ring stages per consumer group, by kind. Shallow read-ahead keeps DRAM
 // reads and writes balanced for the kinds that write as much as they read
 // (measured on B200 at n = 4, d = 7168, bf16: write 2, fused 3); the read
@@ -133,6 +145,12 @@ __host__ __device__ constexpr int64_t pipe_fixed_bytes(int n, int stages, int64_
            + (int64_t)kPipeGroups * ((d_h * 4 + 15) / 16 * 16);  // h rows (1 per group)
 }
 
+// Bulk-store staging (HC_PIPE_TMA_STORE): one slot per consumer warp of
+// `rows` rows x 32 lanes x `vb` bytes.
+__host__ __device__ constexpr int64_t pipe_store_bytes(int n, int rows, int vb) {
+    return HC_PIPE_TMA_STORE ? (int64_t)kPipeGroups * pipe_group_warps(n) * rows * 32 * vb : 0;
+}
+
 // Elements of d one consumer thread handles per tile: one 16-byte vector
 // (n > 4 runs fewer, register-richer consumer threads to afford it).
 template <int N, typename S>
@@ -169,6 +187,32 @@ __device__ __forceinline__ float2 widen_pair(uint32_t w) {
     widen_bf16x2(w, f.x, f.y);
     return f;
 }
+// Round VE fp32 values (pairs) to the storage dtype: the 16 bytes to store
+// and the widened values a later read of them would see.
+template <typename S, int VE> struct VecPack;
+template <> struct VecPack<float, 4> {
+    static __device__ __forceinline__ uint4 pack(const float2 (&v)[2], float2 (&stored)[2]) {
+        stored[0] = v[0];
+        stored[1] = v[1];
+        return make_uint4(__float_as_uint(v[0].x), __float_as_uint(v[0].y), __float_as_uint(v[1].x),
+                          __float_as_uint(v[1].y));
+    }
+};
+template <> struct VecPack<__nv_bfloat16, 8> {
+    static __device__ __forceinline__ uint4 pack(const float2 (&v)[4], float2 (&stored)[4]) {
+        uint4 q;
+        q.x = pack_bf16x2_rn(v[0].x, v[0].y);
+        q.y = pack_bf16x2_rn(v[1].x, v[1].y);
+        q.z = pack_bf16x2_rn(v[2].x, v[2].y);
+        q.w = pack_bf16x2_rn(v[3].x, v[3].y);
+        stored[0] = widen_pair(q.x);
+        stored[1] = widen_pair(q.y);
+        stored[2] = widen_pair(q.z);
+        stored[3] = widen_pair(q.w);
+        return q;
+    }
+};
+
 template <> struct VecIO<__nv_bfloat16, 8> {
     static __device__ __forceinline__ void load_smem(const unsigned char *p, float2 (&v)[4]) {
         const uint4 q = *reinterpret_cast<const uint4 *>(p);
@@ -242,6 +286,112 @@ template <> struct VecIO<__nv_bfloat16, 4> {
     }
 };
 
+// The parameter warp of the pipelined kernels. Token m of the CTA (token
+// blockIdx.x + m * G) belongs to consumer group m % NG as that group's token
+// m / NG, whose parameters go to slot (m % NG) * PSG + (m / NG) % PSG of
+// `params` (PSTRIDE = n*n + 2n floats: A transposed, column j at j * n, then
+// b, then a), published on pfull and reclaimed through pempty (each with one
+// arrival per use: this warp, resp. the group's consumer warps).
+template <int N, bool WRITE, bool READ, int NG, int PSG>
+__device__ __forceinline__ void pipe_param_warp(const StepParams &p, int64_t M, int64_t G, float *params,
+                                                uint64_t *pfull, uint64_t *pempty, float *pscratch,
+                                                volatile int *abort_flag, int *fault, int lane) {
+    constexpr int NN = N * N;
+    constexpr int PSTRIDE = NN + 2 * N;
+    constexpr int PB = pipe_param_batch(N);
+    // ---------------- per-token parameters ----------------
+    // Batch replica rb, lane group lane / GL prepares token
+    // m0 + rb * TPW + lane / GL. The next batch's inputs are loaded
+    // before the current batch is projected, hiding their latency.
+    constexpr int GL = Group<N>::GL, EPL = Group<N>::EPL, TPW = Group<N>::TPW;
+    constexpr int R = pipe_param_replicas(N);
+    static_assert(R * TPW == PB, "a batch is R warps' worth of lane groups");
+    const int q = lane & (GL - 1);
+    float nmv[R][EPL], nlv[R], nbv[R];
+    auto fetch = [&](int64_t m0) {
+#pragma unroll
+        for (int rb = 0; rb < R; ++rb) {
+            const int64_t m = m0 + rb * TPW + lane / GL;
+            const bool live = m < M;
+            const int64_t t = blockIdx.x + m * G;
+#pragma unroll
+            for (int r = 0; r < EPL; ++r) {
+                const int e = q + GL * r;
+                nmv[rb][r] = (WRITE && live && e < NN) ? p.A[t * p.A_s + e] : 0.0f;
+            }
+            nbv[rb] = (WRITE && live && q < N) ? p.b[t * p.b_s + q] : 0.0f;
+            nlv[rb] = (READ && live && q < N) ? p.a[t * p.a_s + q] : 0.0f;
+        }
+    };
+    fetch(0);
+    for (int64_t m0 = 0; m0 < M; m0 += PB) {
+        float mv[R][EPL], lv[R], bvv[R];
+#pragma unroll
+        for (int rb = 0; rb < R; ++rb) {
+#pragma unroll
+            for (int r = 0; r < EPL; ++r) mv[rb][r] = nmv[rb][r];
+            lv[rb] = nlv[rb];
+            bvv[rb] = nbv[rb];
+        }
+        if (m0 + PB < M) fetch(m0 + PB);
+        bool w = true;
+#pragma unroll
+        for (int rb = 0; rb < R; ++rb) {
+            const int64_t m = m0 + rb * TPW + lane / GL;
+            const int64_t i = m / NG;  // token ordinal within its group
+            const int ps = (int)(m % NG) * PSG + (int)(i % PSG);
+            if (m < M && i >= PSG)
+                w = w && mbar_wait_bounded(&pempty[ps], (uint32_t)(((i / PSG) & 1) ^ 1), abort_flag,
+                                           fault, FAULT_WAIT_PARAM);
+        }
+        if (!__all_sync(0xffffffffu, w)) break;
+        if constexpr (WRITE) {
+            if (p.mix_logits) {
+                // the consumers wait on the first batch: project it with the
+                // shortest-latency exchange (same results bit for bit)
+                if (HC_PIPE_FIRST_SHFL && m0 == 0)
+                    group_sinkhorn<N, R, true>(mv, pscratch, lane, p.K);
+                else
+                    group_sinkhorn<N, R, false>(mv, pscratch, lane, p.K);
+            }
+        }
+        if constexpr (READ) {
+            if (p.read_logits) {
+#pragma unroll
+                for (int rb = 0; rb < R; ++rb) lv[rb] = group_softmax<N>(lv[rb], pscratch, lane);
+            }
+        }
+#pragma unroll
+        for (int rb = 0; rb < R; ++rb) {
+            const int64_t m = m0 + rb * TPW + lane / GL;
+            if (m >= M) continue;
+            const int64_t i = m / NG;
+            const int ps = (int)(m % NG) * PSG + (int)(i % PSG);
+            float *P = params + ps * PSTRIDE;
+            if constexpr (WRITE) {
+#pragma unroll
+                for (int r = 0; r < EPL; ++r) {
+                    const int e = q + GL * r;  // A[i][j], i = e / N, j = e % N
+                    if (e < NN) P[(e % N) * N + e / N] = mv[rb][r];
+                }
+                if (q < N) P[NN + q] = bvv[rb];
+            }
+            if constexpr (READ) {
+                if (q < N) P[NN + N + q] = lv[rb];
+            }
+        }
+        __syncwarp();
+#pragma unroll
+        for (int rb = 0; rb < R; ++rb) {
+            const int64_t m = m0 + rb * TPW + lane / GL;
+            if (m < M && q == 0) {
+                const int64_t i = m / NG;
+                mbar_arrive(&pfull[(int)(m % NG) * PSG + (int)(i % PSG)]);
+            }
+        }
+    }
+}
+
 template <int N, typename S, int KIND>
 __global__ void __launch_bounds__(pipe_threads(N), 1)
 hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
@@ -274,6 +424,13 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
     float *hrow_base = pscratch + pipe_param_replicas(N) * kGroupScratch;  // 16-byte aligned
     const int64_t d = p.d;
     const int64_t hrow_stride = READ ? (d + 3) / 4 * 4 : 0;  // floats per group row
+    // bulk-store staging (HC_PIPE_TMA_STORE, write kinds): per consumer warp
+    // SROWS rows of 32 lanes x VB bytes (H' rows, then x unless the kind sends
+    // x to several destinations)
+    constexpr bool TSTORE = HC_PIPE_TMA_STORE && WRITE;
+    constexpr bool STAGE_X = TSTORE && READ && !REDUCE;
+    constexpr int SROWS = N + (STAGE_X ? 1 : 0);
+    unsigned char *stage_base = reinterpret_cast<unsigned char *>(hrow_base + NG * hrow_stride);
     const int SG = sh.stages / NG;  // stages per group ring
 
     const int warp = threadIdx.x >> 5;
@@ -391,90 +548,8 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
     }
 
     if (warp == 1) {
-        // ---------------- per-token parameters ----------------
-        // Batch replica rb, lane group lane / GL prepares token
-        // m0 + rb * TPW + lane / GL. The next batch's inputs are loaded
-        // before the current batch is projected, hiding their latency.
-        constexpr int GL = Group<N>::GL, EPL = Group<N>::EPL, TPW = Group<N>::TPW;
-        constexpr int R = pipe_param_replicas(N);
-        static_assert(R * TPW == PB, "a batch is R warps' worth of lane groups");
-        const int q = lane & (GL - 1);
-        float nmv[R][EPL], nlv[R], nbv[R];
-        auto fetch = [&](int64_t m0) {
-#pragma unroll
-            for (int rb = 0; rb < R; ++rb) {
-                const int64_t m = m0 + rb * TPW + lane / GL;
-                const bool live = m < M;
-                const int64_t t = blockIdx.x + m * G;
-#pragma unroll
-                for (int r = 0; r < EPL; ++r) {
-                    const int e = q + GL * r;
-                    nmv[rb][r] = (WRITE && live && e < NN) ? p.A[t * p.A_s + e] : 0.0f;
-                }
-                nbv[rb] = (WRITE && live && q < N) ? p.b[t * p.b_s + q] : 0.0f;
-                nlv[rb] = (READ && live && q < N) ? p.a[t * p.a_s + q] : 0.0f;
-            }
-        };
-        fetch(0);
-        for (int64_t m0 = 0; m0 < M; m0 += PB) {
-            float mv[R][EPL], lv[R], bvv[R];
-#pragma unroll
-            for (int rb = 0; rb < R; ++rb) {
-#pragma unroll
-                for (int r = 0; r < EPL; ++r) mv[rb][r] = nmv[rb][r];
-                lv[rb] = nlv[rb];
-                bvv[rb] = nbv[rb];
-            }
-            if (m0 + PB < M) fetch(m0 + PB);
-            bool w = true;
-#pragma unroll
-            for (int rb = 0; rb < R; ++rb) {
-                const int64_t m = m0 + rb * TPW + lane / GL;
-                const int64_t i = m / NG;  // token ordinal within its group
-                const int ps = (int)(m % NG) * PSG + (int)(i % PSG);
-                if (m < M && i >= PSG)
-                    w = w && mbar_wait_bounded(&pempty[ps], (uint32_t)(((i / PSG) & 1) ^ 1), abort_flag,
-                                               fault, FAULT_WAIT_PARAM);
-            }
-            if (!__all_sync(0xffffffffu, w)) break;
-            if constexpr (WRITE) {
-                if (p.mix_logits) group_sinkhorn<N, R, false>(mv, pscratch, lane, p.K);
-            }
-            if constexpr (READ) {
-                if (p.read_logits) {
-#pragma unroll
-                    for (int rb = 0; rb < R; ++rb) lv[rb] = group_softmax<N>(lv[rb], pscratch, lane);
-                }
-            }
-#pragma unroll
-            for (int rb = 0; rb < R; ++rb) {
-                const int64_t m = m0 + rb * TPW + lane / GL;
-                if (m >= M) continue;
-                const int64_t i = m / NG;
-                const int ps = (int)(m % NG) * PSG + (int)(i % PSG);
-                float *P = params + ps * PSTRIDE;
-                if constexpr (WRITE) {
-#pragma unroll
-                    for (int r = 0; r < EPL; ++r) {
-                        const int e = q + GL * r;  // A[i][j], i = e / N, j = e % N
-                        if (e < NN) P[(e % N) * N + e / N] = mv[rb][r];
-                    }
-                    if (q < N) P[NN + q] = bvv[rb];
-                }
-                if constexpr (READ) {
-                    if (q < N) P[NN + N + q] = lv[rb];
-                }
-            }
-            __syncwarp();
-#pragma unroll
-            for (int rb = 0; rb < R; ++rb) {
-                const int64_t m = m0 + rb * TPW + lane / GL;
-                if (m < M && q == 0) {
-                    const int64_t i = m / NG;
-                    mbar_arrive(&pfull[(int)(m % NG) * PSG + (int)(i % PSG)]);
-                }
-            }
-        }
+        pipe_param_warp<N, WRITE, READ, NG, PSG>(p, M, G, params, pfull, pempty, pscratch, abort_flag,
+                                                 fault, lane);
         return;
     }
 
@@ -494,6 +569,7 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
     uint64_t *gempty = empty + g * SG;
     unsigned char *gring = ring + (size_t)g * SG * sh.stage_bytes;
     float *hrow = hrow_base + g * hrow_stride;
+    unsigned char *wst = stage_base + (size_t)cw * SROWS * 32 * VB;  // this warp's staging slot
     S *Ho = static_cast<S *>(p.Hout);
     S *X = static_cast<S *>(p.x);
     int slot = 0;      // ring position of this group's next tile
@@ -570,6 +646,11 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&gempty[cs]);  // stage data is in registers
+                if constexpr (TSTORE) {
+                    // the previous tile's bulk stores have read the staging slot
+                    if (lane == 0) bulk_wait_read<0>();
+                    __syncwarp();
+                }
                 if (active) {
                     if constexpr (REDUCE) {
                         // one rounding to the storage dtype (what a stored y holds)
@@ -603,7 +684,12 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
                             const float2 cb = make_float2(bv[jj], bv[jj]);
 #pragma unroll
                             for (int e = 0; e < VP; ++e) acc[e] = ffma2_rn(cb, yv[e], acc[e]);
-                            VecIO<S, V>::store(Hot + jj * d, acc, stored);
+                            if constexpr (TSTORE) {
+                                *reinterpret_cast<uint4 *>(wst + (jj * 32 + lane) * VB) =
+                                    VecPack<S, V>::pack(acc, stored);
+                            } else {
+                                VecIO<S, V>::store(Hot + jj * d, acc, stored);
+                            }
                             if constexpr (READ) {
                                 const float2 ca = make_float2(av[jj], av[jj]);
                                 if (jj == 0) {
@@ -638,6 +724,12 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
             }
             if constexpr (READ) {
                 if (prev) {
+                    if constexpr (STAGE_X) {
+                        if (!cur) {  // no stage wait above: free the staging slot here
+                            if (lane == 0) bulk_wait_read<0>();
+                            __syncwarp();
+                        }
+                    }
                     if (j == 0) {
                         // token i-1's sum of squares, reduced over the group's warps
                         const bool w = mbar_wait_bounded(&redbar[g], (uint32_t)((i - 1) & 1), abort_flag,
@@ -673,6 +765,10 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
 #pragma unroll
                             for (int q = 0; q < kPipeMaxRanks; ++q)
                                 if (q < rd.nx) VecIO<S, V>::store(static_cast<S *>(rd.xs[q]) + off, xv);
+                        } else if constexpr (STAGE_X) {
+                            float2 unused[VP];
+                            *reinterpret_cast<uint4 *>(wst + (N * 32 + lane) * VB) =
+                                VecPack<S, V>::pack(xv, unused);
                         } else {
                             VecIO<S, V>::store(X + t_prev * d + k, xv);
                         }
@@ -684,6 +780,27 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
                     for (int e = 0; e < VP; e += 2)
                         *reinterpret_cast<float4 *>(hrow + k + 2 * e) =
                             make_float4(hr[e].x, hr[e].y, hr[e + 1].x, hr[e + 1].y);
+                }
+            }
+            if constexpr (TSTORE) {
+                // the warp's staged rows go out as bulk copies of its active lanes'
+                // contiguous 32 x VB bytes per row
+                const int64_t kw0 = (int64_t)j * tile + (int64_t)gw * 32 * V;
+                const int64_t left = (d - kw0) / V;
+                const uint32_t nb = (uint32_t)((left < 32 ? (left > 0 ? left : 0) : 32) * VB);
+                const bool sx = STAGE_X && prev;
+                if (nb != 0 && (cur || sx)) {
+                    fence_proxy_async_smem();  // this lane's staging writes -> async proxy
+                    __syncwarp();
+                    if (lane == 0) {
+                        if (cur) {
+#pragma unroll
+                            for (int jj = 0; jj < N; ++jj)
+                                bulk_store(Ho + (t * N + jj) * d + kw0, wst + jj * 32 * VB, nb);
+                        }
+                        if (sx) bulk_store(X + t_prev * d + kw0, wst + N * 32 * VB, nb);
+                        bulk_commit();
+                    }
                 }
             }
         }
@@ -700,6 +817,9 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
                 }
             }
         }
+    }
+    if constexpr (TSTORE) {
+        if (lane == 0) bulk_wait_all();  // staged rows written before the CTA exits
     }
 }
 
