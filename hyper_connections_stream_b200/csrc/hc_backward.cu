@@ -22,7 +22,11 @@
 //                        Sinkhorn backward with the 2K+1 iterates kept in
 //                        shared memory; in place on dA / da.
 //   hc_dg_reduce_kernel  sums the per-CTA gain partials in a fixed order.
+#include <atomic>
+
 #include "hc_launch.h"
+#include "hc_backward_common.cuh"
+#include "hc_backward_pipe.cuh"
 
 namespace hc {
 
@@ -36,158 +40,6 @@ constexpr int kBwThreads = 256;  // largest CTA of the step kernel (255 register
         hc_status _st = (expr);         \
         if (_st != HC_OK) return _st;   \
     } while (0)
-
-// VE fp32 gains (1 when g is null); k is a multiple of VE.
-template <int VE>
-__device__ __forceinline__ void bw_load_gain(const float *g, int64_t k, float (&gv)[VE]) {
-    if (g == nullptr) {
-#pragma unroll
-        for (int e = 0; e < VE; ++e) gv[e] = 1.0f;
-    } else if constexpr (VE == 2) {
-        const float2 q = __ldg(reinterpret_cast<const float2 *>(g + k));
-        gv[0] = q.x;
-        gv[1] = q.y;
-    } else {
-#pragma unroll
-        for (int e = 0; e < VE; e += 4) {
-            const float4 q = __ldg(reinterpret_cast<const float4 *>(g + k + e));
-            gv[e] = q.x; gv[e + 1] = q.y; gv[e + 2] = q.z; gv[e + 3] = q.w;
-        }
-    }
-}
-
-// VE-element vectors of the storage dtype (16 or 8 bytes), widened to fp32.
-template <typename S, int VE> struct BwVec;
-template <> struct BwVec<float, 4> {
-    static __device__ __forceinline__ void load(const float *p, float (&v)[4]) {
-        const float4 q = __ldcs(reinterpret_cast<const float4 *>(p));
-        v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
-    }
-    static __device__ __forceinline__ void store(float *p, const float (&v)[4]) {
-        __stcs(reinterpret_cast<float4 *>(p), make_float4(v[0], v[1], v[2], v[3]));
-    }
-    static __device__ __forceinline__ void round(float (&)[4]) {}
-    static __device__ __forceinline__ void store_smem(float *p, const float (&v)[4]) {
-        *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
-    }
-    static __device__ __forceinline__ void load_smem(const float *p, float (&v)[4]) {
-        const float4 q = *reinterpret_cast<const float4 *>(p);
-        v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
-    }
-};
-template <> struct BwVec<float, 2> {
-    static __device__ __forceinline__ void load(const float *p, float (&v)[2]) {
-        const float2 q = __ldcs(reinterpret_cast<const float2 *>(p));
-        v[0] = q.x; v[1] = q.y;
-    }
-    static __device__ __forceinline__ void store(float *p, const float (&v)[2]) {
-        __stcs(reinterpret_cast<float2 *>(p), make_float2(v[0], v[1]));
-    }
-    static __device__ __forceinline__ void round(float (&)[2]) {}
-    static __device__ __forceinline__ void store_smem(float *p, const float (&v)[2]) {
-        *reinterpret_cast<float2 *>(p) = make_float2(v[0], v[1]);
-    }
-    static __device__ __forceinline__ void load_smem(const float *p, float (&v)[2]) {
-        const float2 q = *reinterpret_cast<const float2 *>(p);
-        v[0] = q.x; v[1] = q.y;
-    }
-};
-template <> struct BwVec<__nv_bfloat16, 4> {
-    static __device__ __forceinline__ void load(const __nv_bfloat16 *p, float (&v)[4]) {
-        const uint2 q = __ldcs(reinterpret_cast<const uint2 *>(p));
-        widen_bf16x2(q.x, v[0], v[1]); widen_bf16x2(q.y, v[2], v[3]);
-    }
-    static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float (&v)[4]) {
-        uint2 q;
-        q.x = pack_bf16x2_rn(v[0], v[1]); q.y = pack_bf16x2_rn(v[2], v[3]);
-        __stcs(reinterpret_cast<uint2 *>(p), q);
-    }
-    static __device__ __forceinline__ void round(float (&v)[4]) {
-#pragma unroll
-        for (int e = 0; e < 4; e += 2) widen_bf16x2(pack_bf16x2_rn(v[e], v[e + 1]), v[e], v[e + 1]);
-    }
-    // shared-memory copies of values already rounded to bf16 (exact)
-    static __device__ __forceinline__ void store_smem(__nv_bfloat16 *p, const float (&v)[4]) {
-        uint2 q;
-        q.x = pack_bf16x2_rn(v[0], v[1]); q.y = pack_bf16x2_rn(v[2], v[3]);
-        *reinterpret_cast<uint2 *>(p) = q;
-    }
-    static __device__ __forceinline__ void load_smem(const __nv_bfloat16 *p, float (&v)[4]) {
-        const uint2 q = *reinterpret_cast<const uint2 *>(p);
-        widen_bf16x2(q.x, v[0], v[1]); widen_bf16x2(q.y, v[2], v[3]);
-    }
-};
-
-// 8-byte vectors for bf16 (16 bytes would double the per-slice registers and
-// halve the CTAs per SM); 16-byte fp32 vectors up to n = 4.
-template <typename S> constexpr int bw_vec_elems(int n) {
-    return sizeof(S) == 2 ? 4 : (n <= 4 ? 4 : 2);
-}
-
-struct BwKernelParams {
-    StepParams f;
-    const void *dHout;
-    const void *dx;
-    void *dH;
-    void *dy;
-    float *gA, *gb, *ga;  // per-token sums (gradients w.r.t. the matrix / weights)
-    float *dg_part;       // [gridDim.x][d] or null
-};
-
-// The forward of one VE-slice: H' as stored (hs) and h, exactly as the
-// forward kernels compute them (fp32 FMA chains in stream order, storage
-// rounding of H').
-template <int N, typename S, int VE>
-__device__ __forceinline__ void bw_forward_slice(const S *Ht, const S *Yt, int64_t d, int64_t k,
-                                                 const float *At, const float *bt, const float *at,
-                                                 float (&hv)[N][VE], float (&yv)[VE],
-                                                 float (&hs)[N][VE], float (&h)[VE]) {
-    using V = BwVec<S, VE>;
-#pragma unroll
-    for (int i = 0; i < N; ++i) V::load(Ht + i * d + k, hv[i]);
-    V::load(Yt + k, yv);
-    // paired fp32 FMAs: each element's chain is the scalar one, bit for bit
-#pragma unroll
-    for (int e = 0; e < VE; ++e) h[e] = -0.0f;
-#pragma unroll
-    for (int j = 0; j < N; ++j) {
-#pragma unroll
-        for (int e = 0; e < VE; e += 2) {
-            float2 acc = make_float2(-0.0f, -0.0f);
-#pragma unroll
-            for (int i = 0; i < N; ++i)
-                acc = ffma2_rn(make_float2(At[i * N + j], At[i * N + j]),
-                               make_float2(hv[i][e], hv[i][e + 1]), acc);
-            acc = ffma2_rn(make_float2(bt[j], bt[j]), make_float2(yv[e], yv[e + 1]), acc);
-            hs[j][e] = acc.x;
-            hs[j][e + 1] = acc.y;
-        }
-        V::round(hs[j]);
-#pragma unroll
-        for (int e = 0; e < VE; e += 2) {
-            const float2 hh = ffma2_rn(make_float2(at[j], at[j]), make_float2(hs[j][e], hs[j][e + 1]),
-                                       make_float2(h[e], h[e + 1]));
-            h[e] = hh.x;
-            h[e + 1] = hh.y;
-        }
-    }
-}
-
-// Stream j of H' as the forward stores it, from the loaded H and y slices.
-template <int N, typename S, int VE>
-__device__ __forceinline__ void bw_stream_out(const float (&hv)[N][VE], const float (&yv)[VE],
-                                              const float *At, const float *bt, int j,
-                                              float (&hs)[VE]) {
-#pragma unroll
-    for (int e = 0; e < VE; ++e) hs[e] = -0.0f;
-#pragma unroll
-    for (int i = 0; i < N; ++i)
-#pragma unroll
-        for (int e = 0; e < VE; ++e) hs[e] = __fmaf_rn(At[i * N + j], hv[i][e], hs[e]);
-#pragma unroll
-    for (int e = 0; e < VE; ++e) hs[e] = __fmaf_rn(bt[j], yv[e], hs[e]);
-    BwVec<S, VE>::round(hs);
-}
 
 // Two CTAs per SM (128 registers a thread) up to n = 5; the n*n per-thread
 // sums of larger n need the full register file.
@@ -571,9 +423,36 @@ struct StepBw {
         if (e != cudaSuccess) return set_error(HC_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
         return HC_OK;
     }
+    // The TMA-fed kernel (hc_backward_pipe.cuh): bf16, n <= 4, only when the
+    // pipelined path is forced (hc_set_path), and when its token buffer, dH'
+    // ring, parked H' and gain partial fit shared memory (checked with the
+    // ring, so the choice does not depend on dH'). It reads exactly the
+    // minimum from DRAM but issues ~18 % more instructions per token than the
+    // register kernel, which measured faster at T = 16384, n = 4, d = 7168
+    // (1.11 against 1.19 ms), so the automatic choice is the register kernel.
+    static bool pipelined(int64_t T, int64_t d, bool want_dg, const LaunchCtx &ctx, BwPipeShape &ps) {
+        (void)T;
+        if constexpr (sizeof(S) != 2 || N > 4) {
+            return false;
+        } else {
+            if (ctx.path != 1) return false;
+            const int64_t ntile = (d + kBwpTile - 1) / kBwpTile;
+            if (ntile > 64) return false;
+            ps.ntile = (int)ntile;
+            ps.gstages = kBwpGradStages;
+            return bwp_smem_bytes<N>(ps.ntile, ps.gstages, want_dg) <= (int64_t)kSmemLimitLogits;
+        }
+    }
     // Launch shape; the grid is what the gain-gradient workspace is sized by.
     static hc_status plan(int64_t T, int64_t d, bool want_dg, const LaunchCtx &ctx, int &NT,
                           int64_t &grid) {
+        BwPipeShape ps{};
+        if (pipelined(T, d, want_dg, ctx, ps)) {
+            NT = kBwpThreads;
+            grid = ctx.sms < T ? ctx.sms : T;
+            if (grid < 1) grid = 1;
+            return HC_OK;
+        }
         shape(d, NT);
         const size_t dyn = dyn_bytes(d, want_dg);
         if (dyn > (size_t)kSmemLimitLogits - 48 * 1024)
@@ -601,6 +480,39 @@ struct StepBw {
         int NT = 0;
         int64_t grid = 0;
         HC_BW_TRY(plan(a.f.T, a.f.d, want_dg, ctx, NT, grid));
+        BwPipeShape ps{};
+        if (pipelined(a.f.T, a.f.d, want_dg, ctx, ps)) {
+            if constexpr (sizeof(S) == 2 && N <= 4) {
+                if (!a.dHout) ps.gstages = 0;
+                const int64_t smem = bwp_smem_bytes<N>(ps.ntile, ps.gstages, want_dg);
+                auto kern = hc_bwd_pipe_kernel<N>;
+                static std::atomic<int> configured[64];  // largest opt-in so far, per device
+                if (ctx.device < 0 || ctx.device >= 64)
+                    return set_error(HC_ERR_UNSUPPORTED, "device ordinal %d >= 64", ctx.device);
+                if (smem > configured[ctx.device].load()) {
+                    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                         (int)smem);
+                    if (e != cudaSuccess)
+                        return set_error(HC_ERR_CUDA, "backward smem attribute: %s", cudaGetErrorString(e));
+                    configured[ctx.device].store((int)smem);
+                }
+                BwPipeParams pp{};
+                pp.f = a.f;
+                pp.dHout = a.dHout;
+                pp.dx = a.dx;
+                pp.dH = a.dH;
+                pp.dy = a.dy;
+                pp.gA = a.dA;
+                pp.gb = a.db;
+                pp.ga = a.da;
+                pp.dg_part = want_dg ? static_cast<float *>(a.workspace) : nullptr;
+                kern<<<(unsigned)grid, kBwpThreads, (size_t)smem, st>>>(pp, ps, ctx.fault);
+                cudaError_t e = cudaGetLastError();
+                if (e != cudaSuccess)
+                    return set_error(HC_ERR_CUDA, "hc_bwd_pipe_kernel launch: %s", cudaGetErrorString(e));
+                return launch_tail(a, ctx, st, grid, hist, pthreads);
+            }
+        }
         BwKernelParams bp{};
         bp.f = a.f;
         bp.dHout = a.dHout;
@@ -618,6 +530,13 @@ struct StepBw {
             hc_step_bwd_kernel<N, S, VE, false><<<(unsigned)grid, NT, dyn, st>>>(bp);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return set_error(HC_ERR_CUDA, "hc_step_bwd_kernel launch: %s", cudaGetErrorString(e));
+        return launch_tail(a, ctx, st, grid, hist, pthreads);
+    }
+    // The parameter backward (softmax, Sinkhorn) and the gain reduction over
+    // the step kernel's `grid` partial rows.
+    static hc_status launch_tail(const BackwardArgs &a, const LaunchCtx &ctx, cudaStream_t st,
+                                 int64_t grid, size_t hist, int pthreads) {
+        cudaError_t e;
         if (a.f.mix_logits || a.f.read_logits) {
             auto pk = hc_param_bwd_kernel<N>;
             e = cudaFuncSetAttribute(pk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist);

@@ -84,20 +84,18 @@ hc_status launch_stream(const StepParams &p, const LaunchCtx &ctx, cudaStream_t 
 // ---- pipelined family -------------------------------------------------------------
 
 // Ring geometry for a kind whose stages hold `rows` rows of a tile.
-template <int N, typename S, int KIND>
+template <int N, typename S, int KIND, int GW = pipe_group_warps(N)>
 bool pipe_shape(const StepParams &p, int rows, PipeShape &sh, int &smem) {
     constexpr int V = pipe_vec_elems<N, S>();
     const int64_t d_h = kind_normalises(KIND) ? p.d : 0;
-    sh.tile = pipe_group_warps(N) * 32 * V;
+    sh.tile = GW * 32 * V;
     const int64_t ntile = (p.d + sh.tile - 1) / sh.tile;
     if (ntile > (1 << 20)) return false;
     sh.ntile = (int)ntile;
     sh.stage_bytes = rows * sh.tile * (int)sizeof(S);
     // one ring per consumer group: the pipelined family needs room for two
     // stages per group; the ring then takes the kind's measured depth
-    constexpr int srows = N + (KIND == KIND_FUSED ? 1 : 0);
-    const int64_t st_bytes = KIND == KIND_READ ? 0 : pipe_store_bytes(N, srows, V * (int)sizeof(S));
-    int64_t per_group = (kSmemLimit - pipe_fixed_bytes(N, 0, d_h) - st_bytes) /
+    int64_t per_group = (kSmemLimit - pipe_fixed_bytes(N, 0, d_h, GW)) /
                         ((int64_t)kPipeGroups * (sh.stage_bytes + 16));
     if (per_group < 2) return false;
     if (per_group > kMaxStages / kPipeGroups) per_group = kMaxStages / kPipeGroups;
@@ -107,7 +105,7 @@ bool pipe_shape(const StepParams &p, int rows, PipeShape &sh, int &smem) {
     if (per_group > cap) per_group = cap;
     if (per_group < 1) per_group = 1;
     sh.stages = (int)(per_group * kPipeGroups);
-    smem = (int)((int64_t)sh.stages * sh.stage_bytes + pipe_fixed_bytes(N, sh.stages, d_h) + st_bytes);
+    smem = (int)((int64_t)sh.stages * sh.stage_bytes + pipe_fixed_bytes(N, sh.stages, d_h, GW));
     return true;
 }
 
@@ -116,10 +114,10 @@ bool pipe_shape(const StepParams &p, PipeShape &sh, int &smem) {
     return pipe_shape<N, S, KIND>(p, KIND != KIND_READ ? N + 1 : N, sh, smem);
 }
 
-template <int N, typename S, int KIND>
+template <int N, typename S, int KIND, int GW = pipe_group_warps(N)>
 hc_status launch_pipe(const StepParams &p, const PipeShape &sh, int smem, const LaunchCtx &ctx,
                       cudaStream_t st, const PipeReduce &rd = PipeReduce{}) {
-    auto kern = hc_pipe_kernel<N, S, KIND>;
+    auto kern = hc_pipe_kernel<N, S, KIND, GW>;
     static std::atomic<int> configured[64];  // largest dynamic smem opted in so far, per device
     if (ctx.device < 0 || ctx.device >= 64)
         return set_error(HC_ERR_UNSUPPORTED, "device ordinal %d >= 64", ctx.device);
@@ -132,7 +130,7 @@ hc_status launch_pipe(const StepParams &p, const PipeShape &sh, int smem, const 
     }
     int64_t grid = ctx.sms;
     if (grid > p.T) grid = p.T;
-    kern<<<(unsigned)grid, pipe_threads(N), smem, st>>>(p, sh, ctx.fault, rd);
+    kern<<<(unsigned)grid, pipe_threads_gw(GW), smem, st>>>(p, sh, ctx.fault, rd);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(HC_ERR_CUDA, "hc_pipe_kernel launch: %s", cudaGetErrorString(e));
     return HC_OK;

@@ -48,17 +48,11 @@ namespace hc {
 #ifndef HC_PIPE_L2_HINT
 #define HC_PIPE_L2_HINT 0
 #endif
-// 1: consumer warps stage their rounded H' (and x) slices in shared memory
-// and write them with bulk copies (cp.async.bulk shared -> global) instead of
-// 16-byte register stores.
-#ifndef HC_PIPE_TMA_STORE
-#define HC_PIPE_TMA_STORE 0
-#endif
 // 1: the parameter warp projects its first batch with shuffle exchanges
 // (shortest latency; the consumers wait on it), later batches through shared
-// memory (highest throughput).
+// memory (highest throughput). Same results bit for bit either way.
 #ifndef HC_PIPE_FIRST_SHFL
-#define HC_PIPE_FIRST_SHFL 0
+#define HC_PIPE_FIRST_SHFL 1
 #endif
 // Ring stages per consumer group, by kind. Shallow read-ahead keeps DRAM
 // reads and writes balanced for the kinds that write as much as they read
@@ -87,6 +81,8 @@ __host__ __device__ constexpr int pipe_group_warps(int n) {
 __host__ __device__ constexpr int pipe_threads(int n) {
     return 64 + kPipeGroups * pipe_group_warps(n) * 32;
 }
+// Threads of a pipelined CTA with gw consumer warps per group.
+__host__ __device__ constexpr int pipe_threads_gw(int gw) { return 64 + kPipeGroups * gw * 32; }
 // The parameter warp prepares kParamReplicas warps' worth of lane groups at a
 // time (4 tokens for n = 3, 4; 2 for n >= 5); each group's slot ring holds at
 // least 8 of its tokens, and two batches, so preparation runs ahead.
@@ -134,28 +130,28 @@ struct PipeReduce {
 // serves two tokens at once: a thread reads back only its own slice
 // positions, so at each tile it first reads the previous token's h there (for
 // that token's x) and then overwrites it with the current token's.
-__host__ __device__ constexpr int64_t pipe_fixed_bytes(int n, int stages, int64_t d_h) {
+__host__ __device__ constexpr int64_t pipe_fixed_bytes(int n, int stages, int64_t d_h,
+                                                       int gw = -1) {
     return (int64_t)stages * 16                        // full + empty barriers
            + kPipeGroups * pipe_param_slots_per_group(n) * 16  // param full + empty
            + (kPipeGroups + 1) / 2 * 16                // group reduction barriers
            + kPipeGroups * pipe_param_slots_per_group(n) * (n * n + 2 * n) * 4  // slots
-           + kPipeGroups * 2 * pipe_group_warps(n) * 8  // reduction partials
+           + kPipeGroups * 2 * (gw > 0 ? gw : pipe_group_warps(n)) * 8  // reduction partials
            + 16                                        // abort flag (padded)
            + pipe_param_replicas(n) * kGroupScratch * 4  // parameter warp scratch
            + (int64_t)kPipeGroups * ((d_h * 4 + 15) / 16 * 16);  // h rows (1 per group)
 }
 
-// Bulk-store staging (HC_PIPE_TMA_STORE): one slot per consumer warp of
-// `rows` rows x 32 lanes x `vb` bytes.
-__host__ __device__ constexpr int64_t pipe_store_bytes(int n, int rows, int vb) {
-    return HC_PIPE_TMA_STORE ? (int64_t)kPipeGroups * pipe_group_warps(n) * rows * 32 * vb : 0;
-}
 
 // Elements of d one consumer thread handles per tile: one 16-byte vector
-// (n > 4 runs fewer, register-richer consumer threads to afford it).
+// (n > 4 runs fewer, register-richer consumer threads to afford it), or with
+// HC_PIPE_WIDE_HALF an 8-byte bf16 half vector for n > 4.
+#ifndef HC_PIPE_WIDE_HALF
+#define HC_PIPE_WIDE_HALF 0
+#endif
 template <int N, typename S>
 __host__ __device__ constexpr int pipe_vec_elems() {
-    return StorageTraits<S>::V;
+    return (HC_PIPE_WIDE_HALF && N > 4 && sizeof(S) == 2) ? 4 : StorageTraits<S>::V;
 }
 
 // Shared-memory loads and streaming global stores of VE storage elements,
@@ -187,32 +183,6 @@ __device__ __forceinline__ float2 widen_pair(uint32_t w) {
     widen_bf16x2(w, f.x, f.y);
     return f;
 }
-// Round VE fp32 values (pairs) to the storage dtype: the 16 bytes to store
-// and the widened values a later read of them would see.
-template <typename S, int VE> struct VecPack;
-template <> struct VecPack<float, 4> {
-    static __device__ __forceinline__ uint4 pack(const float2 (&v)[2], float2 (&stored)[2]) {
-        stored[0] = v[0];
-        stored[1] = v[1];
-        return make_uint4(__float_as_uint(v[0].x), __float_as_uint(v[0].y), __float_as_uint(v[1].x),
-                          __float_as_uint(v[1].y));
-    }
-};
-template <> struct VecPack<__nv_bfloat16, 8> {
-    static __device__ __forceinline__ uint4 pack(const float2 (&v)[4], float2 (&stored)[4]) {
-        uint4 q;
-        q.x = pack_bf16x2_rn(v[0].x, v[0].y);
-        q.y = pack_bf16x2_rn(v[1].x, v[1].y);
-        q.z = pack_bf16x2_rn(v[2].x, v[2].y);
-        q.w = pack_bf16x2_rn(v[3].x, v[3].y);
-        stored[0] = widen_pair(q.x);
-        stored[1] = widen_pair(q.y);
-        stored[2] = widen_pair(q.z);
-        stored[3] = widen_pair(q.w);
-        return q;
-    }
-};
-
 template <> struct VecIO<__nv_bfloat16, 8> {
     static __device__ __forceinline__ void load_smem(const unsigned char *p, float2 (&v)[4]) {
         const uint4 q = *reinterpret_cast<const uint4 *>(p);
@@ -285,6 +255,30 @@ template <> struct VecIO<__nv_bfloat16, 4> {
         __stcs(reinterpret_cast<uint2 *>(p), q);
     }
 };
+
+// The n floats of a mixing-matrix column from a parameter slot, with the
+// widest shared-memory loads the column's alignment allows (slots start on
+// 16 bytes; a column starts at 4 n bytes into its slot): one LDS.128 per
+// four values for n % 4 == 0, one LDS.64 per pair for even n.
+template <int N>
+__device__ __forceinline__ void load_column(const float *c, float (&col)[N]) {
+    if constexpr (N % 4 == 0) {
+#pragma unroll
+        for (int q = 0; q < N; q += 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(c + q);
+            col[q] = v.x; col[q + 1] = v.y; col[q + 2] = v.z; col[q + 3] = v.w;
+        }
+    } else if constexpr (N % 2 == 0) {
+#pragma unroll
+        for (int q = 0; q < N; q += 2) {
+            const float2 v = *reinterpret_cast<const float2 *>(c + q);
+            col[q] = v.x; col[q + 1] = v.y;
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < N; ++q) col[q] = c[q];
+    }
+}
 
 // The parameter warp of the pipelined kernels. Token m of the CTA (token
 // blockIdx.x + m * G) belongs to consumer group m % NG as that group's token
@@ -392,8 +386,8 @@ __device__ __forceinline__ void pipe_param_warp(const StepParams &p, int64_t M, 
     }
 }
 
-template <int N, typename S, int KIND>
-__global__ void __launch_bounds__(pipe_threads(N), 1)
+template <int N, typename S, int KIND, int GW = pipe_group_warps(N)>
+__global__ void __launch_bounds__(pipe_threads_gw(GW), 1)
 hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
     constexpr int V = pipe_vec_elems<N, S>();
     constexpr int VB = V * (int)sizeof(S);  // bytes per thread per row of a tile
@@ -403,7 +397,6 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
     constexpr bool REDUCE = KIND == KIND_REDUCE;
     const int ROWS = REDUCE ? N + rd.nlocal : WRITE ? N + 1 : N;
     constexpr int PSTRIDE = NN + 2 * N;  // A transposed (column j at j*N) | b | a
-    constexpr int GW = pipe_group_warps(N);
     constexpr int NG = kPipeGroups;
     constexpr int PSG = pipe_param_slots_per_group(N);
     constexpr int kParamSlots = NG * PSG;
@@ -424,13 +417,6 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
     float *hrow_base = pscratch + pipe_param_replicas(N) * kGroupScratch;  // 16-byte aligned
     const int64_t d = p.d;
     const int64_t hrow_stride = READ ? (d + 3) / 4 * 4 : 0;  // floats per group row
-    // bulk-store staging (HC_PIPE_TMA_STORE, write kinds): per consumer warp
-    // SROWS rows of 32 lanes x VB bytes (H' rows, then x unless the kind sends
-    // x to several destinations)
-    constexpr bool TSTORE = HC_PIPE_TMA_STORE && WRITE;
-    constexpr bool STAGE_X = TSTORE && READ && !REDUCE;
-    constexpr int SROWS = N + (STAGE_X ? 1 : 0);
-    unsigned char *stage_base = reinterpret_cast<unsigned char *>(hrow_base + NG * hrow_stride);
     const int SG = sh.stages / NG;  // stages per group ring
 
     const int warp = threadIdx.x >> 5;
@@ -569,7 +555,6 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
     uint64_t *gempty = empty + g * SG;
     unsigned char *gring = ring + (size_t)g * SG * sh.stage_bytes;
     float *hrow = hrow_base + g * hrow_stride;
-    unsigned char *wst = stage_base + (size_t)cw * SROWS * 32 * VB;  // this warp's staging slot
     S *Ho = static_cast<S *>(p.Hout);
     S *X = static_cast<S *>(p.x);
     int slot = 0;      // ring position of this group's next tile
@@ -646,11 +631,6 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&gempty[cs]);  // stage data is in registers
-                if constexpr (TSTORE) {
-                    // the previous tile's bulk stores have read the staging slot
-                    if (lane == 0) bulk_wait_read<0>();
-                    __syncwarp();
-                }
                 if (active) {
                     if constexpr (REDUCE) {
                         // one rounding to the storage dtype (what a stored y holds)
@@ -667,10 +647,9 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
                         S *Hot = Ho + t * N * d + k;
 #pragma unroll
                         for (int jj = 0; jj < N; ++jj) {
-                            // column jj of A: A[0][jj] .. A[N-1][jj]
+                            // column jj of A: A[0][jj] .. A[N-1][jj] (contiguous in the slot)
                             float col[N];
-#pragma unroll
-                            for (int ii = 0; ii < N; ++ii) col[ii] = P[jj * N + ii];
+                            load_column<N>(P + jj * N, col);
                             float2 acc[VP], stored[VP];
                             const float2 c0 = make_float2(col[0], col[0]);
 #pragma unroll
@@ -684,12 +663,7 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
                             const float2 cb = make_float2(bv[jj], bv[jj]);
 #pragma unroll
                             for (int e = 0; e < VP; ++e) acc[e] = ffma2_rn(cb, yv[e], acc[e]);
-                            if constexpr (TSTORE) {
-                                *reinterpret_cast<uint4 *>(wst + (jj * 32 + lane) * VB) =
-                                    VecPack<S, V>::pack(acc, stored);
-                            } else {
-                                VecIO<S, V>::store(Hot + jj * d, acc, stored);
-                            }
+                            VecIO<S, V>::store(Hot + jj * d, acc, stored);
                             if constexpr (READ) {
                                 const float2 ca = make_float2(av[jj], av[jj]);
                                 if (jj == 0) {
@@ -724,12 +698,6 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
             }
             if constexpr (READ) {
                 if (prev) {
-                    if constexpr (STAGE_X) {
-                        if (!cur) {  // no stage wait above: free the staging slot here
-                            if (lane == 0) bulk_wait_read<0>();
-                            __syncwarp();
-                        }
-                    }
                     if (j == 0) {
                         // token i-1's sum of squares, reduced over the group's warps
                         const bool w = mbar_wait_bounded(&redbar[g], (uint32_t)((i - 1) & 1), abort_flag,
@@ -765,10 +733,6 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
 #pragma unroll
                             for (int q = 0; q < kPipeMaxRanks; ++q)
                                 if (q < rd.nx) VecIO<S, V>::store(static_cast<S *>(rd.xs[q]) + off, xv);
-                        } else if constexpr (STAGE_X) {
-                            float2 unused[VP];
-                            *reinterpret_cast<uint4 *>(wst + (N * 32 + lane) * VB) =
-                                VecPack<S, V>::pack(xv, unused);
                         } else {
                             VecIO<S, V>::store(X + t_prev * d + k, xv);
                         }
@@ -780,27 +744,6 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
                     for (int e = 0; e < VP; e += 2)
                         *reinterpret_cast<float4 *>(hrow + k + 2 * e) =
                             make_float4(hr[e].x, hr[e].y, hr[e + 1].x, hr[e + 1].y);
-                }
-            }
-            if constexpr (TSTORE) {
-                // the warp's staged rows go out as bulk copies of its active lanes'
-                // contiguous 32 x VB bytes per row
-                const int64_t kw0 = (int64_t)j * tile + (int64_t)gw * 32 * V;
-                const int64_t left = (d - kw0) / V;
-                const uint32_t nb = (uint32_t)((left < 32 ? (left > 0 ? left : 0) : 32) * VB);
-                const bool sx = STAGE_X && prev;
-                if (nb != 0 && (cur || sx)) {
-                    fence_proxy_async_smem();  // this lane's staging writes -> async proxy
-                    __syncwarp();
-                    if (lane == 0) {
-                        if (cur) {
-#pragma unroll
-                            for (int jj = 0; jj < N; ++jj)
-                                bulk_store(Ho + (t * N + jj) * d + kw0, wst + jj * 32 * VB, nb);
-                        }
-                        if (sx) bulk_store(X + t_prev * d + kw0, wst + N * 32 * VB, nb);
-                        bulk_commit();
-                    }
                 }
             }
         }
@@ -817,9 +760,6 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
                 }
             }
         }
-    }
-    if constexpr (TSTORE) {
-        if (lane == 0) bulk_wait_all();  // staged rows written before the CTA exits
     }
 }
 

@@ -36,17 +36,23 @@ def _param_bar(key, dt, mix, read):
     return DA_BF16_LOGITS if (key == "da" and dt == "bf16" and (mix or read)) else 2e-4
 
 
-@pytest.fixture(scope="module")
-def hc():
+@pytest.fixture(scope="module", params=["auto", "pipelined", "register"])
+def hc(request):
+    """The binding with the backward's step kernel chosen automatically (the
+    register kernel), forced to the TMA-fed kernel (bf16, n <= 4; other calls
+    keep the register kernel) or forced to the register kernel."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from hyper_connections_stream_b200 import build
     build.build()
     import hyper_connections_stream_b200._lib as L
     L.lib()
+    L.set_path({"auto": L.PATH_AUTO, "pipelined": L.PATH_PIPELINED,
+                "register": L.PATH_REGISTER}[request.param])
     yield L
     torch.cuda.synchronize()
     assert L.device_fault() == 0
+    L.set_path(L.PATH_AUTO)
 
 
 def _inputs(T, n, d, dt, mix, read, per_token, seed, with_dHout=True):
