@@ -959,11 +959,37 @@ def run_ours(args):
     except Exception:
         pass
 
+    # The timed steps are captured once in a CUDA graph (the way a layer loop
+    # is deployed: no host time between launches) and replayed once untimed;
+    # the timed region is one replay between two events. --stream-launch times
+    # plain stream launches with events around every step instead.
+    graph = None
+    if not args.stream_launch:
+        side = torch.cuda.Stream(device)
+        side.wait_stream(stream)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            for i in range(args.steps):
+                step(bufs[i % 2], bufs[(i + 1) % 2])
+        graph.replay()
+        torch.cuda.synchronize()
+
     def timed():
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
         _barrier(ws)
         torch.cuda.synchronize()
+        if graph is not None:
+            a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with ClockSampler(uuid if rank == 0 else None) as clk:
+                a_.record(stream)
+                graph.replay()
+                b_.record(stream)
+                torch.cuda.synchronize()
+            _barrier(ws)
+            total_ms = a_.elapsed_time(b_)
+            return total_ms, [total_ms / args.steps], clk.summary()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
         with ClockSampler(uuid if rank == 0 else None) as clk:
             for i in range(args.steps):
                 ev[i][0].record(stream)
@@ -994,6 +1020,7 @@ def run_ours(args):
     prof = (_profiled_traffic("fused_mhc_n4_d7168_bf16_T16384")
             if (T, n, d) == (WORKLOAD["T"], WORKLOAD["n"], WORKLOAD["d"]) else None)
 
+    del graph
     # end to end through the public API with host buffers
     e2e = None if args.kernel_only else run_e2e(args, inp, w, device, ws)
 
@@ -1015,6 +1042,9 @@ def run_ours(args):
                      "frac_of_8TBs": achieved / 8000.0},
         "e2e": e2e,
         "gpu_launches": args.steps * ws,
+        "launch": "stream launches, events around every step" if args.stream_launch
+        else f"CUDA graph of the {args.steps} timed steps, replayed once (one warm replay before); "
+             "events around the replay",
         "kernel_path": args.path,
         "device_fault": hc.device_fault(),
         "clocks": clocks,
@@ -1204,6 +1234,9 @@ def main(argv=None):
                          "step's backward pass; decode: per-call latency of small steps (CUDA graph); "
                          "sweep: tokens/s and HBM fraction per T x n x d point, the static layer "
                          "(read, write, unfused pair, fused) and the 78-layer depth stack")
+    ap.add_argument("--stream-launch", action="store_true",
+                    help="time the step with plain stream launches and events around every step "
+                         "(default: the timed steps replayed from one CUDA graph)")
     ap.add_argument("--path", choices=["auto", "pipelined", "register"], default="auto",
                     help="kernel family (auto = pipelined wherever it applies)")
     ap.add_argument("--ranks", type=int, default=8,
