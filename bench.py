@@ -63,6 +63,9 @@ KERNEL_SOURCES = {
     "backward_mhc_n4_d7168_bf16_T16384": ["hc_backward.cu", "hc_backward_pipe.cuh",
                                           "hc_backward_common.cuh", "hc_pipe_kernels.cuh",
                                           "hc_device.cuh", "hc_sync.cuh"],
+    "backward_pipe_mhc_n4_d7168_bf16_T16384": ["hc_backward.cu", "hc_backward_pipe.cuh",
+                                               "hc_backward_common.cuh", "hc_pipe_kernels.cuh",
+                                               "hc_device.cuh", "hc_sync.cuh"],
     "reduce_write_r8_mhc_n4_d7168_bf16_T16384": ["hc_pipe_kernels.cuh", "hc_device.cuh",
                                                  "hc_sync.cuh", "hc_kernels_impl.cuh",
                                                  "hc_k_bf16_reduce.cu", "hc_reduce_write.cu"],
@@ -613,7 +616,9 @@ def run_backward(args):
                    "l2": "inputs and outputs > L2; the binding allocates the gradient outputs"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak,
-                     "traffic": _profiled_traffic("backward_mhc_n4_d7168_bf16_T16384")
+                     "traffic": _profiled_traffic(("backward_pipe_mhc_n4_d7168_bf16_T16384"
+                                                   if args.path == "pipelined" else
+                                                   "backward_mhc_n4_d7168_bf16_T16384"))
                      if (T, n) == (16384, 4) else None,
                      "peak_source": peak_kind,
                      "algorithmic_bytes_per_step": alg_bytes, "step_ms": step_ms},

@@ -130,7 +130,7 @@ hc_status launch_pipe(const StepParams &p, const PipeShape &sh, int smem, const 
     }
     int64_t grid = ctx.sms;
     if (grid > p.T) grid = p.T;
-    kern<<<(unsigned)grid, pipe_threads_gw(GW), smem, st>>>(p, sh, ctx.fault, rd);
+    kern<<<(unsigned)grid, pipe_threads_gw(GW, pipe_param_warps(N)), smem, st>>>(p, sh, ctx.fault, rd);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(HC_ERR_CUDA, "hc_pipe_kernel launch: %s", cudaGetErrorString(e));
     return HC_OK;

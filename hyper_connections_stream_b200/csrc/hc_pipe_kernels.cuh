@@ -72,17 +72,46 @@ namespace hc {
 #define HC_PIPE_SG_REDUCE 4
 #endif
 constexpr int kPipeGroups = HC_PIPE_GROUPS;
+// Geometry for n > 5. Two Sinkhorn elements per lane and one token per warp
+// make the projection cost about four times the instructions per token of
+// n <= 5, and one parameter warp could not keep pace with the streams (at
+// n = 6, d = 4096 the step ran at half the copy rate with K = 20 and at 88 %
+// with K = 1). So several parameter warps share the token batches, and for
+// n = 7, 8 the consumer groups narrow to four warps to keep the register
+// budget (measured on B200: n = 6, d = 7168: 0.662 -> 0.600 ms; d = 4096:
+// 0.593 -> 0.390 ms; n = 8, d = 4096: 0.688 -> 0.485 ms; n = 8, d = 7168
+// within 1 %).
+#ifndef HC_PIPE_GROUP_WARPS_6
+#define HC_PIPE_GROUP_WARPS_6 5
+#endif
+#ifndef HC_PIPE_PARAM_WARPS_6
+#define HC_PIPE_PARAM_WARPS_6 2
+#endif
+#ifndef HC_PIPE_GROUP_WARPS_78
+#define HC_PIPE_GROUP_WARPS_78 4
+#endif
+#ifndef HC_PIPE_PARAM_WARPS_78
+#define HC_PIPE_PARAM_WARPS_78 3
+#endif
 // Consumer warps per group: fewer for n > 4, so that each thread has the
 // registers to hold n widened 16-byte rows (launch bounds give 65536 /
-// threads registers a thread: 128 at 7 warps per group, 170 at 5).
+// threads registers a thread, the threads counted in whole 128-thread
+// quarters: 128 at 16 warps, 170 at 12).
 __host__ __device__ constexpr int pipe_group_warps(int n) {
-    return n > 4 ? HC_PIPE_GROUP_WARPS_WIDE : HC_PIPE_GROUP_WARPS;
+    return n > 6 ? HC_PIPE_GROUP_WARPS_78 : n == 6 ? HC_PIPE_GROUP_WARPS_6
+                 : n > 4 ? HC_PIPE_GROUP_WARPS_WIDE : HC_PIPE_GROUP_WARPS;
+}
+__host__ __device__ constexpr int pipe_param_warps(int n) {
+    return n > 6 ? HC_PIPE_PARAM_WARPS_78 : n == 6 ? HC_PIPE_PARAM_WARPS_6 : 1;
 }
 __host__ __device__ constexpr int pipe_threads(int n) {
-    return 64 + kPipeGroups * pipe_group_warps(n) * 32;
+    return 32 * (1 + pipe_param_warps(n)) + kPipeGroups * pipe_group_warps(n) * 32;
 }
-// Threads of a pipelined CTA with gw consumer warps per group.
-__host__ __device__ constexpr int pipe_threads_gw(int gw) { return 64 + kPipeGroups * gw * 32; }
+// Threads of a pipelined CTA with gw consumer warps per group and npw
+// parameter warps (plus the producer warp).
+__host__ __device__ constexpr int pipe_threads_gw(int gw, int npw = 1) {
+    return 32 * (1 + npw) + kPipeGroups * gw * 32;
+}
 // The parameter warp prepares kParamReplicas warps' worth of lane groups at a
 // time (4 tokens for n = 3, 4; 2 for n >= 5); each group's slot ring holds at
 // least 8 of its tokens, and two batches, so preparation runs ahead.
@@ -96,9 +125,11 @@ __host__ __device__ constexpr int pipe_param_batch(int n) {
     return pipe_param_replicas(n) *
            (n * n <= 1 ? 32 : n * n <= 2 ? 16 : n * n <= 4 ? 8 : n * n <= 8 ? 4 : n * n <= 16 ? 2 : 1);
 }
+// Slots per group: at least 8 of its tokens, and one batch more than the
+// parameter warps prepare at once, so preparation runs ahead.
 __host__ __device__ constexpr int pipe_param_slots_per_group(int n) {
-    return (((2 * pipe_param_batch(n) + kPipeGroups - 1) / kPipeGroups > 8
-                 ? (2 * pipe_param_batch(n) + kPipeGroups - 1) / kPipeGroups
+    return ((((pipe_param_warps(n) + 1) * pipe_param_batch(n) + kPipeGroups - 1) / kPipeGroups > 8
+                 ? ((pipe_param_warps(n) + 1) * pipe_param_batch(n) + kPipeGroups - 1) / kPipeGroups
                  : 8) + 1) & ~1;  // even
 }
 constexpr int kMaxStages = 32;
@@ -138,7 +169,7 @@ __host__ __device__ constexpr int64_t pipe_fixed_bytes(int n, int stages, int64_
            + kPipeGroups * pipe_param_slots_per_group(n) * (n * n + 2 * n) * 4  // slots
            + kPipeGroups * 2 * (gw > 0 ? gw : pipe_group_warps(n)) * 8  // reduction partials
            + 16                                        // abort flag (padded)
-           + pipe_param_replicas(n) * kGroupScratch * 4  // parameter warp scratch
+           + pipe_param_warps(n) * pipe_param_replicas(n) * kGroupScratch * 4  // parameter warps' scratch
            + (int64_t)kPipeGroups * ((d_h * 4 + 15) / 16 * 16);  // h rows (1 per group)
 }
 
@@ -289,7 +320,8 @@ __device__ __forceinline__ void load_column(const float *c, float (&col)[N]) {
 template <int N, bool WRITE, bool READ, int NG, int PSG>
 __device__ __forceinline__ void pipe_param_warp(const StepParams &p, int64_t M, int64_t G, float *params,
                                                 uint64_t *pfull, uint64_t *pempty, float *pscratch,
-                                                volatile int *abort_flag, int *fault, int lane) {
+                                                volatile int *abort_flag, int *fault, int lane,
+                                                int pw = 0, int npw = 1) {
     constexpr int NN = N * N;
     constexpr int PSTRIDE = NN + 2 * N;
     constexpr int PB = pipe_param_batch(N);
@@ -317,8 +349,9 @@ __device__ __forceinline__ void pipe_param_warp(const StepParams &p, int64_t M, 
             nlv[rb] = (READ && live && q < N) ? p.a[t * p.a_s + q] : 0.0f;
         }
     };
-    fetch(0);
-    for (int64_t m0 = 0; m0 < M; m0 += PB) {
+    // parameter warp pw of npw takes batches pw, pw + npw, ...
+    fetch((int64_t)pw * PB);
+    for (int64_t m0 = (int64_t)pw * PB; m0 < M; m0 += (int64_t)npw * PB) {
         float mv[R][EPL], lv[R], bvv[R];
 #pragma unroll
         for (int rb = 0; rb < R; ++rb) {
@@ -327,7 +360,7 @@ __device__ __forceinline__ void pipe_param_warp(const StepParams &p, int64_t M, 
             lv[rb] = nlv[rb];
             bvv[rb] = nbv[rb];
         }
-        if (m0 + PB < M) fetch(m0 + PB);
+        if (m0 + (int64_t)npw * PB < M) fetch(m0 + (int64_t)npw * PB);
         bool w = true;
 #pragma unroll
         for (int rb = 0; rb < R; ++rb) {
@@ -343,7 +376,7 @@ __device__ __forceinline__ void pipe_param_warp(const StepParams &p, int64_t M, 
             if (p.mix_logits) {
                 // the consumers wait on the first batch: project it with the
                 // shortest-latency exchange (same results bit for bit)
-                if (HC_PIPE_FIRST_SHFL && m0 == 0)
+                if (HC_PIPE_FIRST_SHFL && m0 < (int64_t)npw * PB)
                     group_sinkhorn<N, R, true>(mv, pscratch, lane, p.K);
                 else
                     group_sinkhorn<N, R, false>(mv, pscratch, lane, p.K);
@@ -387,7 +420,7 @@ __device__ __forceinline__ void pipe_param_warp(const StepParams &p, int64_t M, 
 }
 
 template <int N, typename S, int KIND, int GW = pipe_group_warps(N)>
-__global__ void __launch_bounds__(pipe_threads_gw(GW), 1)
+__global__ void __launch_bounds__(pipe_threads_gw(GW, pipe_param_warps(N)), 1)
 hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
     constexpr int V = pipe_vec_elems<N, S>();
     constexpr int VB = V * (int)sizeof(S);  // bytes per thread per row of a tile
@@ -414,7 +447,8 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
     int *abort_word = reinterpret_cast<int *>(sred + NG * 2 * GW);
     volatile int *abort_flag = abort_word;
     float *pscratch = reinterpret_cast<float *>(abort_word + 4);  // parameter warp scratch
-    float *hrow_base = pscratch + pipe_param_replicas(N) * kGroupScratch;  // 16-byte aligned
+    constexpr int NPW = pipe_param_warps(N);
+    float *hrow_base = pscratch + NPW * pipe_param_replicas(N) * kGroupScratch;  // 16-byte aligned
     const int64_t d = p.d;
     const int64_t hrow_stride = READ ? (d + 3) / 4 * 4 : 0;  // floats per group row
     const int SG = sh.stages / NG;  // stages per group ring
@@ -533,9 +567,10 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
         return;
     }
 
-    if (warp == 1) {
-        pipe_param_warp<N, WRITE, READ, NG, PSG>(p, M, G, params, pfull, pempty, pscratch, abort_flag,
-                                                 fault, lane);
+    if (warp >= 1 && warp <= NPW) {
+        pipe_param_warp<N, WRITE, READ, NG, PSG>(
+            p, M, G, params, pfull, pempty, pscratch + (warp - 1) * pipe_param_replicas(N) * kGroupScratch,
+            abort_flag, fault, lane, warp - 1, NPW);
         return;
     }
 
@@ -547,7 +582,7 @@ hc_pipe_kernel(StepParams p, PipeShape sh, int *fault, PipeReduce rd) {
     // before it waits for the other warps' sums, so the wait overlaps work.
     // Both tokens share the group's h row: at each tile a thread reads token
     // i-1's h at its own slice positions before it stores token i's there.
-    const int cw = warp - 2;
+    const int cw = warp - 1 - NPW;
     const int g = cw / GW;
     const int gw = cw - g * GW;
     const int gt = gw * 32 + lane;
