@@ -145,10 +145,24 @@ hc_status launch_step_n(const StepParams &p, const LaunchCtx &ctx, cudaStream_t 
         return set_error(HC_ERR_UNSUPPORTED, "pipelined kernels do not cover d = %lld here",
                          (long long)p.d);
     // Small calls (decode-sized batches) finish sooner without the pipeline's
-    // set-up: below ~64 MiB of stream traffic the register-streaming family
-    // wins on B200 (measured crossover: n = 4, d = 7168 at ~450 tokens;
-    // d = 4096 at ~1000; n = 8 at ~600).
-    const bool small = p.T * (int64_t)N * p.d * (int64_t)sizeof(S) * 2 < (int64_t(64) << 20);
+    // set-up. For the fused step the pipeline needs enough tokens per CTA to
+    // amortise its fill and the first parameter batches: a per-n token count
+    // (wider n: costlier Sinkhorn), times a factor when more than an eighth
+    // of the last pipelined tile would idle. Fitted to a crossover measurement
+    // of both families (B200, bf16, graph-replayed calls, T = 256 ... 8192,
+    // n in {2, 4, 5, 6, 8}, d in {4096, 7168}). The other kinds use the
+    // stream-traffic rule they were measured with: below ~64 MiB the
+    // register-streaming family wins.
+    bool small = p.T * (int64_t)N * p.d * (int64_t)sizeof(S) * 2 < (int64_t(64) << 20);
+    if constexpr (KIND == KIND_FUSED) {
+        constexpr int64_t tmin_n[9] = {0, 512, 512, 256, 256, 1024, 4096, 2048, 2048};
+        constexpr int64_t ragged_x[9] = {0, 16, 16, 4, 4, 16, 4, 4, 4};
+        constexpr int64_t per_tile = (int64_t)pipe_group_warps(N) * 32;  // slices per tile
+        const int64_t nvec = p.d / pipe_vec_elems<N, S>();
+        const int64_t slots = (nvec + per_tile - 1) / per_tile * per_tile;
+        const bool ragged = (slots - nvec) * 8 > slots;
+        small = p.T < tmin_n[N] * (ragged ? ragged_x[N] : 1);
+    }
     if (ctx.path == 2 || !pipe_ok || (ctx.path == 0 && small)) {
         if (kind_normalises(KIND) && p.d > (int64_t)kStreamMaxThreads * 8 * StorageTraits<S>::V)
             return set_error(HC_ERR_UNSUPPORTED, "d = %lld too large", (long long)p.d);

@@ -6,9 +6,11 @@
 //               tile by tile into shared-memory stages with plain bulk copies
 //               (cp.async.bulk, this GPU's own memory, no multicast),
 //               completing on the stage's "full" mbarrier;
-//   warp 1      parameters: lane groups compute the per-token Sinkhorn
-//               projection / read softmax ahead of use into parameter slots;
-//   warps 2..   consumer groups (kPipeGroups x pipe_group_warps(n) warps); group
+//   warps 1..   parameters (pipe_param_warps(n) warps: one for n <= 5, more
+//               for wider n, taking token batches round-robin): lane groups
+//               compute the per-token Sinkhorn projection / read softmax
+//               ahead of use into parameter slots;
+//   the rest    consumer groups (kPipeGroups x pipe_group_warps(n) warps); group
 //               r owns tokens r, r + kPipeGroups, ... of the CTA, reads the
 //               stages, writes H' with coalesced 128-bit stores, keeps h in an
 //               fp32 shared-memory row, reduces the fp64 sum of squares across
