@@ -12,12 +12,14 @@
 //
 // Kernels:
 //   hc_step_bwd_kernel   one CTA per token at a time (grid-stride), threads own
-//                        column slices. Phase 1 recomputes H' (as stored) and
-//                        h and reduces sum h^2 and sum g dx h (fp64); phase 2
-//                        reloads the token (L2-resident by then), forms dh, G,
-//                        dH, dy and the per-token sums (fp32 per thread, fp64
-//                        across warps); the gain gradient accumulates per CTA
-//                        in shared memory and goes to the workspace at exit.
+//                        column slices, their global rows staged ahead through
+//                        a per-thread cp.async ring. Phase 1 recomputes H' (as
+//                        stored) and h, reduces sum h^2 and sum g dx h (fp64)
+//                        and the two da sums, and parks h in shared memory;
+//                        phase 2 re-reads H, y, dx (L2-resident by then),
+//                        reads dH', forms dh, G, dH, dy and the dA / db sums
+//                        (fp32 per thread, fp64 across warps); the gain
+//                        gradient accumulates in the CTA's workspace row.
 //   hc_param_bwd_kernel  lane group per token: the softmax backward, and the
 //                        Sinkhorn backward with the 2K+1 iterates kept in
 //                        shared memory; in place on dA / da.
@@ -33,7 +35,7 @@ namespace hc {
 namespace {
 
 constexpr int kBwTB = 32;       // parameter slots per batch
-constexpr int kBwThreads = 256;  // largest CTA of the step kernel (255 registers a thread)
+constexpr int kBwThreads = 256;  // largest CTA of the step kernel
 
 #define HC_BW_TRY(expr)                 \
     do {                                \
@@ -41,20 +43,39 @@ constexpr int kBwThreads = 256;  // largest CTA of the step kernel (255 register
         if (_st != HC_OK) return _st;   \
     } while (0)
 
-// Two CTAs per SM (128 registers a thread) up to n = 5; the n*n per-thread
-// sums of larger n need the full register file.
-// STAGE: phase 1 parks the token's H' (as stored, bf16) in shared memory and
-// phase 2 reads it back instead of rebuilding it (bf16 storage, when it fits).
-template <int N, typename S, int VE, bool STAGE>
+// One CTA per token at a time (grid-stride over tokens), threads own VE-wide
+// column slices; two CTAs per SM (128 registers a thread) up to n = 5, the
+// n*n per-thread sums of larger n need the full register file.
+//
+// Phase 1 recomputes H' (as stored) and h, reduces sum h^2 and sum g dx h
+// (fp64), and forms the read-weight gradient while H' is live:
+//   da_j = sum_k dh H'_j = r sum_k (g dx) H'_j - (r^3/d)(sum g dx h) sum_k h H'_j
+// (both sums finished once r and the coefficient are known). Phase 2 then
+// needs h but not H': PARK keeps h (fp32, d * 4 bytes) in shared memory from
+// phase 1 (each thread reads back only the slots it wrote), otherwise phase 2
+// rebuilds h from H and y. Phase 2 re-reads H, y and dx (from L2), reads dH',
+// and forms dh, G, dH, dy and the dA / db sums (fp32 per thread, dA paired
+// over stream pairs; one halving exchange per warp, fp64 across warps). The
+// gain gradient accumulates in this CTA's workspace row.
+//
+// RING > 0: each thread stages the global rows of its next RING - 1 slices
+// (H, y, dx and, in phase 2, dH') in its own shared-memory slots with
+// cp.async, in the order the loops consume them (phase 1 then phase 2 of
+// each token, tokens in order), so every thread keeps loads in flight while
+// it computes instead of waiting for each slice's loads.
+template <int N, typename S, int VE, bool PARK, int RING>
 __global__ void __launch_bounds__(kBwThreads, (N <= 5 ? 2 : 1))
 hc_step_bwd_kernel(BwKernelParams bp) {
     const StepParams &p = bp.f;
     constexpr int NN = N * N;
-    constexpr int NR = NN + 2 * N;  // per-token sums: dA, db, da
+    constexpr int NS = NN + N;  // phase-2 sums: dA, db
+    constexpr int NP = (N + 1) / 2;
+    static_assert(RING == 0 || (RING >= 2 && PARK), "a ring needs two stages and the parked h");
     using V = BwVec<S, VE>;
     __shared__ float sA[kBwTB * NN], sb[kBwTB * N], sa[kBwTB * N];
     __shared__ double sred[2][kBwThreads / 32];
-    __shared__ float pred[kBwThreads / 32][NR];
+    __shared__ float pred1[kBwThreads / 32][2 * N];
+    __shared__ float pred[kBwThreads / 32][NS];
     __shared__ float swork[kBwThreads / 32 * kGroupScratch];
     extern __shared__ __align__(16) unsigned char bw_dyn[];
 
@@ -75,10 +96,74 @@ hc_step_bwd_kernel(BwKernelParams bp) {
     S *DH = static_cast<S *>(bp.dH);
     S *DY = static_cast<S *>(bp.dy);
     const bool want_dg = bp.dg_part != nullptr;
-    float *sdg = reinterpret_cast<float *>(bw_dyn);  // [d]: this CTA's gain-gradient partial
-    S *shs = reinterpret_cast<S *>(bw_dyn + (want_dg ? d * 4 : 0));  // [N][d] stored H' (STAGE)
+    // The gain partial accumulates in this CTA's workspace row (L2-resident:
+    // grid x d x 4 bytes); each thread reads and writes only the slots of its
+    // own slices, in program order.
+    float *sdg = want_dg ? bp.dg_part + (int64_t)blockIdx.x * d : nullptr;
     if (want_dg)
-        for (int64_t k = tid; k < d; k += NT) sdg[k] = 0.0f;
+        for (int64_t c = tid; c < nvec; c += NT) {
+            const float z[VE] = {};
+            bw_st_f32<VE>(sdg + c * VE, z);
+        }
+    unsigned char *dyn_rest = bw_dyn;
+    float *shp = reinterpret_cast<float *>(dyn_rest);  // [d] parked h
+
+    // Staging ring: [RING slots][2N + 2 rows: H, y, dx, dH'][NT threads]
+    // chunks of VE elements, so a warp's copies of one row land contiguously.
+    constexpr int RR = 2 * N + 2;
+    constexpr int CB = VE * (int)sizeof(S);
+    const int ROW = NT * CB;
+    unsigned char *ring0 = dyn_rest + (PARK ? d * 4 : 0);
+    auto slot = [&](int st, int row) -> unsigned char * {
+        return ring0 + ((size_t)(st * RR + row) * NT + tid) * CB;
+    };
+    // next slice to stage: slice pc of phase pph of token blockIdx.x + pm G
+    int64_t pm = 0, pc = tid;
+    int pph = 0, ist = 0, cst = 0;
+    auto stage_next = [&]() {
+        if constexpr (RING > 0) {
+            const int64_t tq = blockIdx.x + pm * G;
+            if (pc < nvec && tq < p.T) {
+                const int64_t k = pc * VE;
+#pragma unroll
+                for (int i = 0; i < N; ++i)
+                    bw_cp_async<CB>(smem_addr(slot(ist, i)), H + (tq * N + i) * d + k);
+                bw_cp_async<CB>(smem_addr(slot(ist, N)), Y + tq * d + k);
+                bw_cp_async<CB>(smem_addr(slot(ist, N + 1)), DX + tq * d + k);
+                if (pph == 1 && DHO) {
+#pragma unroll
+                    for (int j = 0; j < N; ++j)
+                        bw_cp_async<CB>(smem_addr(slot(ist, N + 2 + j)), DHO + (tq * N + j) * d + k);
+                }
+            }
+            bw_cp_commit();  // possibly empty: one group per slice keeps the count
+            ist = ist + 1 == RING ? 0 : ist + 1;
+            pc += NT;
+            if (pc >= nvec) {
+                pc = tid;
+                if (pph == 0) {
+                    pph = 1;
+                } else {
+                    pph = 0;
+                    ++pm;
+                }
+            }
+        }
+    };
+    // The slot of the next slice to compute, once its copies have landed;
+    // then the slice RING - 1 ahead is staged into the slot read last.
+    // (Measured: per-token row bases with constant slot offsets issue 18 %
+    // fewer instructions but ran 10 % slower, as did staging before the wait.)
+    auto take = [&]() -> const unsigned char * {
+        bw_cp_wait<RING >= 2 ? RING - 2 : 0>();
+        stage_next();
+        const int st = cst;
+        cst = cst + 1 == RING ? 0 : cst + 1;
+        return slot(st, 0);
+    };
+    if constexpr (RING > 0) {
+        for (int q = 0; q < RING - 1; ++q) stage_next();
+    }
 
     for (int64_t m0 = 0;; m0 += TB) {
         const int64_t first = blockIdx.x + m0 * G;
@@ -92,18 +177,41 @@ hc_step_bwd_kernel(BwKernelParams bp) {
             const float *At = sA + tt * NN, *bt = sb + tt * N, *at = sa + tt * N;
             const S *Ht = H + t * N * d, *Yt = Y + t * d, *DXt = DX + t * d;
 
-            // ---- phase 1: the token's statistics ----
+            // ---- phase 1: the token's statistics and the da sums ----
             double ss = 0.0, sg = 0.0;
+            float2 s1[N], s2[N];
+#pragma unroll
+            for (int j = 0; j < N; ++j) {
+                s1[j] = make_float2(0.0f, 0.0f);
+                s2[j] = make_float2(0.0f, 0.0f);
+            }
             for (int64_t c = tid; c < nvec; c += NT) {
                 const int64_t k = c * VE;
                 float hv[N][VE], yv[VE], hs[N][VE], h[VE], dxv[VE], gv[VE];
-                bw_forward_slice<N, S, VE>(Ht, Yt, d, k, At, bt, at, hv, yv, hs, h);
-                if constexpr (STAGE) {
+                if constexpr (RING > 0) {
+                    const unsigned char *sp = take();
 #pragma unroll
-                    for (int j = 0; j < N; ++j) V::store_smem(shs + j * d + k, hs[j]);
+                    for (int i = 0; i < N; ++i) bw_ld_stage<S, VE>(sp + i * ROW, hv[i]);
+                    bw_ld_stage<S, VE>(sp + N * ROW, yv);
+                    bw_ld_stage<S, VE>(sp + (N + 1) * ROW, dxv);
+                    bw_forward_from<N, S, VE>(hv, yv, At, bt, at, hs, h);
+                } else {
+                    bw_forward_slice<N, S, VE>(Ht, Yt, d, k, At, bt, at, hv, yv, hs, h);
+                    V::load(DXt + k, dxv);
                 }
-                V::load(DXt + k, dxv);
+                if constexpr (PARK) bw_st_f32<VE>(shp + k, h);
                 bw_load_gain<VE>(p.g, k, gv);
+#pragma unroll
+                for (int e = 0; e < VE; e += 2) {
+                    const float2 gdx = fmul2_rn(make_float2(gv[e], gv[e + 1]), make_float2(dxv[e], dxv[e + 1]));
+                    const float2 h2 = make_float2(h[e], h[e + 1]);
+#pragma unroll
+                    for (int j = 0; j < N; ++j) {
+                        const float2 hs2 = make_float2(hs[j][e], hs[j][e + 1]);
+                        s1[j] = ffma2_rn(gdx, hs2, s1[j]);
+                        s2[j] = ffma2_rn(h2, hs2, s2[j]);
+                    }
+                }
 #pragma unroll
                 for (int e = 0; e < VE; ++e) {
                     const double he = (double)h[e];
@@ -115,6 +223,26 @@ hc_step_bwd_kernel(BwKernelParams bp) {
             for (int off = 16; off > 0; off >>= 1) {
                 ss += __shfl_xor_sync(0xffffffffu, ss, off);
                 sg += __shfl_xor_sync(0xffffffffu, sg, off);
+            }
+            {
+                float v1[2 * N];
+#pragma unroll
+                for (int j = 0; j < N; ++j) {
+                    v1[j] = __fadd_rn(s1[j].x, s1[j].y);
+                    v1[N + j] = __fadd_rn(s2[j].x, s2[j].y);
+                }
+                if constexpr (2 * N <= 32) {
+                    bw_warp_sums_to<2 * N>(v1, pred1[warp], lane);
+                } else
+                {
+#pragma unroll
+                    for (int v = 0; v < 2 * N; ++v) {
+                        float val = v1[v];
+#pragma unroll
+                        for (int off = 16; off > 0; off >>= 1) val += __shfl_xor_sync(0xffffffffu, val, off);
+                        if (lane == 0) pred1[warp][v] = val;
+                    }
+                }
             }
             if (lane == 0) {
                 sred[0][warp] = ss;
@@ -129,53 +257,74 @@ hc_step_bwd_kernel(BwKernelParams bp) {
             const float r = __double2float_rn(1.0 / sqrt(tss / (double)d + (double)p.eps));
             const double rd = (double)r;
             const float coef = (float)(rd * rd * rd * tsg / (double)d);
-
-            // ---- phase 2: gradients (the token is re-read from L2) ----
-            // per-thread partial sums, two lanes of a pair each (added at the end)
-            float pA[NN];
-            float2 pb2[N], pa2[N];
-#pragma unroll
-            for (int v = 0; v < NN; ++v) pA[v] = 0.0f;
-#pragma unroll
-            for (int j = 0; j < N; ++j) {
-                pb2[j] = make_float2(0.0f, 0.0f);
-                pa2[j] = make_float2(0.0f, 0.0f);
+            if (tid < N) {
+                double S1 = 0.0, S2 = 0.0;
+                for (int w = 0; w < nwarps; ++w) {
+                    S1 += (double)pred1[w][tid];
+                    S2 += (double)pred1[w][N + tid];
+                }
+                bp.ga[t * N + tid] = (float)(rd * S1 - (double)coef * S2);
             }
+
+            // ---- phase 2: gradients (H, y, dx and dH' read; the first three from L2) ----
+            float2 pA2[N][NP];
+#pragma unroll
+            for (int i = 0; i < N; ++i)
+#pragma unroll
+                for (int q = 0; q < NP; ++q) pA2[i][q] = make_float2(0.0f, 0.0f);
+            float2 pb2[N];
+#pragma unroll
+            for (int j = 0; j < N; ++j) pb2[j] = make_float2(0.0f, 0.0f);
+            const float2 r2 = make_float2(r, r), nc2 = make_float2(-coef, -coef);
             for (int64_t c = tid; c < nvec; c += NT) {
                 const int64_t k = c * VE;
-                float hv[N][VE], yv[VE], h[VE], dh[VE];
+                float hv[N][VE], yv[VE], h[VE], dh[VE], dxv[VE];
+                const unsigned char *sp = nullptr;
+                if constexpr (RING > 0) {
+                    sp = take();
 #pragma unroll
-                for (int i = 0; i < N; ++i) V::load(Ht + i * d + k, hv[i]);
-                V::load(Yt + k, yv);
-                // h from the stored H' (parked in phase 1, or each stream rebuilt)
-                float hsk[STAGE ? N : 1][VE];
+                    for (int i = 0; i < N; ++i) bw_ld_stage<S, VE>(sp + i * ROW, hv[i]);
+                    bw_ld_stage<S, VE>(sp + N * ROW, yv);
+                    bw_ld_stage<S, VE>(sp + (N + 1) * ROW, dxv);
+                } else {
 #pragma unroll
-                for (int e = 0; e < VE; ++e) h[e] = -0.0f;
+                    for (int i = 0; i < N; ++i) V::load(Ht + i * d + k, hv[i]);
+                    V::load(Yt + k, yv);
+                    V::load(DXt + k, dxv);
+                }
+                if constexpr (PARK) {
+                    bw_ld_f32<VE>(shp + k, h);
+                } else {
 #pragma unroll
-                for (int j = 0; j < N; ++j) {
-                    float hs[VE];
-                    if constexpr (STAGE) {
-                        V::load_smem(shs + j * d + k, hsk[j]);
+                    for (int e = 0; e < VE; ++e) h[e] = -0.0f;
 #pragma unroll
-                        for (int e = 0; e < VE; ++e) hs[e] = hsk[j][e];
-                    } else {
+                    for (int j = 0; j < N; ++j) {
+                        float hs[VE];
                         bw_stream_out<N, S, VE>(hv, yv, At, bt, j, hs);
-                    }
 #pragma unroll
-                    for (int e = 0; e < VE; ++e) h[e] = __fmaf_rn(at[j], hs[e], h[e]);
+                        for (int e = 0; e < VE; ++e) h[e] = __fmaf_rn(at[j], hs[e], h[e]);
+                    }
                 }
                 {
-                    float dxv[VE], gv[VE];
-                    V::load(DXt + k, dxv);
+                    float gv[VE];
                     bw_load_gain<VE>(p.g, k, gv);
+                    float sd[VE];
+                    if (want_dg) bw_ld_f32<VE>(sdg + k, sd);
 #pragma unroll
-                    for (int e = 0; e < VE; ++e)
-                        dh[e] = __fmaf_rn(-coef, h[e], __fmul_rn(__fmul_rn(r, gv[e]), dxv[e]));
-                    if (want_dg) {
-#pragma unroll
-                        for (int e = 0; e < VE; ++e)
-                            sdg[k + e] = __fmaf_rn(__fmul_rn(dxv[e], h[e]), r, sdg[k + e]);
+                    for (int e = 0; e < VE; e += 2) {
+                        const float2 dx2 = make_float2(dxv[e], dxv[e + 1]);
+                        const float2 h2 = make_float2(h[e], h[e + 1]);
+                        const float2 u = fmul2_rn(fmul2_rn(r2, make_float2(gv[e], gv[e + 1])), dx2);
+                        const float2 dh2 = ffma2_rn(nc2, h2, u);
+                        dh[e] = dh2.x;
+                        dh[e + 1] = dh2.y;
+                        if (want_dg) {
+                            const float2 s = ffma2_rn(fmul2_rn(dx2, h2), r2, make_float2(sd[e], sd[e + 1]));
+                            sd[e] = s.x;
+                            sd[e + 1] = s.y;
+                        }
                     }
+                    if (want_dg) bw_st_f32<VE>(sdg + k, sd);
                 }
                 float dHacc[N][VE], dyacc[VE];
 #pragma unroll
@@ -185,78 +334,92 @@ hc_step_bwd_kernel(BwKernelParams bp) {
 #pragma unroll
                     for (int e = 0; e < VE; ++e) dHacc[i][e] = 0.0f;
 #pragma unroll
-                for (int j = 0; j < N; ++j) {
-                    float hs[VE], Gj[VE];
-                    if constexpr (STAGE) {
+                for (int jp = 0; jp < NP; ++jp) {
+                    float Gq[2][VE];
 #pragma unroll
-                        for (int e = 0; e < VE; ++e) hs[e] = hsk[j][e];
-                    } else {
-                        bw_stream_out<N, S, VE>(hv, yv, At, bt, j, hs);
-                    }
-                    if (DHO) {
-                        V::load(DHO + (t * N + j) * d + k, Gj);
-                    } else {
+                    for (int q = 0; q < 2; ++q) {
+                        const int j = 2 * jp + q;
+                        if (j >= N) break;
+                        if (DHO) {
+                            if constexpr (RING > 0) bw_ld_stage<S, VE>(sp + (N + 2 + j) * ROW, Gq[q]);
+                            else V::load(DHO + (t * N + j) * d + k, Gq[q]);
+                        } else {
 #pragma unroll
-                        for (int e = 0; e < VE; ++e) Gj[e] = 0.0f;
-                    }
+                            for (int e = 0; e < VE; ++e) Gq[q][e] = 0.0f;
+                        }
 #pragma unroll
-                    for (int e = 0; e < VE; e += 2) {
-                        const float2 dh2 = make_float2(dh[e], dh[e + 1]);
-                        const float2 G2 = ffma2_rn(make_float2(at[j], at[j]), dh2,
-                                                   make_float2(Gj[e], Gj[e + 1]));
-                        Gj[e] = G2.x;
-                        Gj[e + 1] = G2.y;
-                        pa2[j] = ffma2_rn(dh2, make_float2(hs[e], hs[e + 1]), pa2[j]);
-                        pb2[j] = ffma2_rn(make_float2(yv[e], yv[e + 1]), G2, pb2[j]);
-                        const float2 dy2 = ffma2_rn(make_float2(bt[j], bt[j]), G2,
-                                                    make_float2(dyacc[e], dyacc[e + 1]));
-                        dyacc[e] = dy2.x;
-                        dyacc[e + 1] = dy2.y;
+                        for (int e = 0; e < VE; e += 2) {
+                            const float2 G2 = ffma2_rn(make_float2(at[j], at[j]), make_float2(dh[e], dh[e + 1]),
+                                                       make_float2(Gq[q][e], Gq[q][e + 1]));
+                            Gq[q][e] = G2.x;
+                            Gq[q][e + 1] = G2.y;
+                            pb2[j] = ffma2_rn(make_float2(yv[e], yv[e + 1]), G2, pb2[j]);
+                            const float2 dy2 = ffma2_rn(make_float2(bt[j], bt[j]), G2,
+                                                        make_float2(dyacc[e], dyacc[e + 1]));
+                            dyacc[e] = dy2.x;
+                            dyacc[e + 1] = dy2.y;
 #pragma unroll
-                        for (int i = 0; i < N; ++i) {
-                            const float aij = At[i * N + j];
-                            pA[i * N + j] = __fmaf_rn(hv[i][e + 1], G2.y,
-                                                      __fmaf_rn(hv[i][e], G2.x, pA[i * N + j]));
-                            const float2 dH2 = ffma2_rn(make_float2(aij, aij), G2,
-                                                        make_float2(dHacc[i][e], dHacc[i][e + 1]));
-                            dHacc[i][e] = dH2.x;
-                            dHacc[i][e + 1] = dH2.y;
+                            for (int i = 0; i < N; ++i) {
+                                const float aij = At[i * N + j];
+                                const float2 dH2 = ffma2_rn(make_float2(aij, aij), G2,
+                                                            make_float2(dHacc[i][e], dHacc[i][e + 1]));
+                                dHacc[i][e] = dH2.x;
+                                dHacc[i][e + 1] = dH2.y;
+                            }
                         }
                     }
+                    // dA[i][2jp], dA[i][2jp+1]: one paired FMA per element, each
+                    // half the scalar chain over the slice's elements in order
+#pragma unroll
+                    for (int e = 0; e < VE; ++e)
+#pragma unroll
+                        for (int i = 0; i < N; ++i) {
+                            if (2 * jp + 1 < N)
+                                pA2[i][jp] = ffma2_rn(make_float2(hv[i][e], hv[i][e]),
+                                                      make_float2(Gq[0][e], Gq[1][e]), pA2[i][jp]);
+                            else
+                                pA2[i][jp].x = __fmaf_rn(hv[i][e], Gq[0][e], pA2[i][jp].x);
+                        }
                 }
 #pragma unroll
                 for (int i = 0; i < N; ++i) V::store(DH + (t * N + i) * d + k, dHacc[i]);
                 V::store(DY + t * d + k, dyacc);
             }
-            // per-token sums: warp trees (fp32), then the warps in order (fp64)
+            // per-token sums: warp sums (fp32), then the warps in order (fp64)
+            {
+                float v2[NS];
 #pragma unroll
-            for (int v = 0; v < NR; ++v) {
-                float val;
-                if (v < NN) {
-                    val = pA[v];
-                } else {
-                    const float2 pv = v < NN + N ? pb2[v - NN] : pa2[v - NN - N];
-                    val = __fadd_rn(pv.x, pv.y);
+                for (int i = 0; i < N; ++i)
+#pragma unroll
+                    for (int j = 0; j < N; ++j) {
+                        v2[i * N + j] = (j & 1) ? pA2[i][j >> 1].y : pA2[i][j >> 1].x;
+                    }
+#pragma unroll
+                for (int j = 0; j < N; ++j) v2[NN + j] = __fadd_rn(pb2[j].x, pb2[j].y);
+                if constexpr (NS <= 32) {
+                    bw_warp_sums_to<NS>(v2, pred[warp], lane);
+                } else
+                {
+#pragma unroll
+                    for (int v = 0; v < NS; ++v) {
+                        float val = v2[v];
+#pragma unroll
+                        for (int off = 16; off > 0; off >>= 1) val += __shfl_xor_sync(0xffffffffu, val, off);
+                        if (lane == 0) pred[warp][v] = val;
+                    }
                 }
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) val += __shfl_xor_sync(0xffffffffu, val, off);
-                if (lane == 0) pred[warp][v] = val;
             }
             __syncthreads();
-            if (tid < NR) {
+            if (tid < NS) {
                 double acc = 0.0;
                 for (int w = 0; w < nwarps; ++w) acc += (double)pred[w][tid];
                 const float out = (float)acc;
                 if (tid < NN) bp.gA[t * NN + tid] = out;
-                else if (tid < NN + N) bp.gb[t * N + (tid - NN)] = out;
-                else bp.ga[t * N + (tid - NN - N)] = out;
+                else bp.gb[t * N + (tid - NN)] = out;
             }
         }
     }
-    if (want_dg) {
-        __syncthreads();
-        for (int64_t k = tid; k < d; k += NT) bp.dg_part[(int64_t)blockIdx.x * d + k] = sdg[k];
-    }
+    if constexpr (RING > 0) bw_cp_wait_all();
 }
 
 // Per token, in place: da <- softmax backward of da (read logits), dA <- the
@@ -395,28 +558,52 @@ hc_dg_reduce_kernel(const float *part, int rows, int64_t d, float *dg) {
     }
 }
 
+#ifndef HC_BW_RING
+#define HC_BW_RING 3  // cp.async staging stages of the step kernel (0: none)
+#endif
+
 template <int N, typename S>
 struct StepBw {
     static constexpr int VE = bw_vec_elems<S>(N);
-    // Shared-memory budget of the dynamic part: two CTAs per SM up to n = 5.
-    static constexpr size_t kDynBudget = N <= 5 ? 96 * 1024 : 176 * 1024;
-    static bool stage(int64_t d, bool want_dg) {
-        return sizeof(S) == 2 && (size_t)N * d * 2 + (want_dg ? (size_t)d * 4 : 0) <= kDynBudget;
+    // Shared-memory budget of the dynamic part: two CTAs per SM up to n = 5
+    // (2 x (104 KB + static + 1 KB reserved) <= 228 KB).
+    static constexpr size_t kDynBudget = N <= 5 ? 104 * 1024 : 176 * 1024;
+    static constexpr int kRing = HC_BW_RING;
+    static_assert(kRing == 0 || kRing >= 2, "two staging stages at least");
+    static size_t park_bytes(int64_t d) { return (size_t)d * 4; }  // h, fp32
+    static size_t ring_bytes(int NT) { return (size_t)kRing * (2 * N + 2) * NT * VE * sizeof(S); }
+    // 0: nothing staged; 1: h parked; 2: h parked and the rows staged through
+    // the cp.async ring -- the deepest that fits the budget.
+    static int mode(int64_t d, int NT) {
+        if (park_bytes(d) > kDynBudget) return 0;
+        if (kRing > 0 && park_bytes(d) + ring_bytes(NT) <= kDynBudget) return 2;
+        return 1;
     }
-    static size_t dyn_bytes(int64_t d, bool want_dg) {
-        return (want_dg ? (size_t)d * 4 : 0) + (stage(d, want_dg) ? (size_t)N * d * 2 : 0);
+    static size_t dyn_bytes(int64_t d, int NT) {
+        const int md = mode(d, NT);
+        return (md >= 1 ? park_bytes(d) : 0) + (md == 2 ? ring_bytes(NT) : 0);
+    }
+    template <int MD>
+    static auto kernel() {
+        return hc_step_bwd_kernel<N, S, VE, (MD >= 1), (MD == 2 ? kRing : 0)>;
     }
     static hc_status shape(int64_t d, int &NT) {
         const int64_t nvec = d / VE;
         int64_t nt = nvec < kBwThreads ? nvec : kBwThreads;
         nt = (nt + 31) / 32 * 32;
+        // a CTA size that divides the row's slices, when one is near the largest
+        for (int64_t c = nt; c >= nt / 2 && c >= 32 && nvec >= kBwThreads; c -= 32)
+            if (nvec % c == 0) {
+                nt = c;
+                break;
+            }
         if (nt < 32) nt = 32;
         NT = (int)nt;
         return HC_OK;
     }
-    template <bool ST>
+    template <int MD>
     static hc_status occupancy(int NT, size_t dyn, int &per_sm) {
-        auto kern = hc_step_bwd_kernel<N, S, VE, ST>;
+        auto kern = kernel<MD>();
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
         if (e != cudaSuccess) return set_error(HC_ERR_CUDA, "backward smem attribute: %s", cudaGetErrorString(e));
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NT, dyn);
@@ -427,9 +614,9 @@ struct StepBw {
     // pipelined path is forced (hc_set_path), and when its token buffer, dH'
     // ring, parked H' and gain partial fit shared memory (checked with the
     // ring, so the choice does not depend on dH'). It reads exactly the
-    // minimum from DRAM but issues ~18 % more instructions per token than the
-    // register kernel, which measured faster at T = 16384, n = 4, d = 7168
-    // (1.11 against 1.19 ms), so the automatic choice is the register kernel.
+    // minimum from DRAM, but the staged step kernel measured faster at
+    // T = 16384, n = 4, d = 7168 (0.99 against 1.19 ms), so the automatic
+    // choice is the step kernel.
     static bool pipelined(int64_t T, int64_t d, bool want_dg, const LaunchCtx &ctx, BwPipeShape &ps) {
         (void)T;
         if constexpr (sizeof(S) != 2 || N > 4) {
@@ -454,11 +641,13 @@ struct StepBw {
             return HC_OK;
         }
         shape(d, NT);
-        const size_t dyn = dyn_bytes(d, want_dg);
-        if (dyn > (size_t)kSmemLimitLogits - 48 * 1024)
+        const size_t dyn = dyn_bytes(d, NT);
+        if (dyn > (size_t)kSmemLimitLogits - 16 * 1024)
             return set_error(HC_ERR_UNSUPPORTED, "d = %lld too large for the backward", (long long)d);
         int per_sm = 0;
-        HC_BW_TRY(stage(d, want_dg) ? occupancy<true>(NT, dyn, per_sm) : occupancy<false>(NT, dyn, per_sm));
+        const int md = mode(d, NT);
+        HC_BW_TRY(md == 2 ? occupancy<2>(NT, dyn, per_sm)
+                          : md == 1 ? occupancy<1>(NT, dyn, per_sm) : occupancy<0>(NT, dyn, per_sm));
         if (per_sm < 1) per_sm = 1;
         grid = (int64_t)ctx.sms * per_sm;
         if (grid > T) grid = T;
@@ -523,11 +712,14 @@ struct StepBw {
         bp.gb = a.db;
         bp.ga = a.da;
         bp.dg_part = want_dg ? static_cast<float *>(a.workspace) : nullptr;
-        const size_t dyn = dyn_bytes(a.f.d, want_dg);
-        if (stage(a.f.d, want_dg))
-            hc_step_bwd_kernel<N, S, VE, true><<<(unsigned)grid, NT, dyn, st>>>(bp);
+        const size_t dyn = dyn_bytes(a.f.d, NT);
+        const int md = mode(a.f.d, NT);
+        if (md == 2)
+            kernel<2>()<<<(unsigned)grid, NT, dyn, st>>>(bp);
+        else if (md == 1)
+            kernel<1>()<<<(unsigned)grid, NT, dyn, st>>>(bp);
         else
-            hc_step_bwd_kernel<N, S, VE, false><<<(unsigned)grid, NT, dyn, st>>>(bp);
+            kernel<0>()<<<(unsigned)grid, NT, dyn, st>>>(bp);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return set_error(HC_ERR_CUDA, "hc_step_bwd_kernel launch: %s", cudaGetErrorString(e));
         return launch_tail(a, ctx, st, grid, hist, pthreads);

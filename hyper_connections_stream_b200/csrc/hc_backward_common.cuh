@@ -104,18 +104,14 @@ struct BwKernelParams {
     float *dg_part;       // [gridDim.x][d] or null
 };
 
-// The forward of one VE-slice: H' as stored (hs) and h, exactly as the
-// forward kernels compute them (fp32 FMA chains in stream order, storage
-// rounding of H').
+// The forward of one VE-slice from its widened H and y values: H' as stored
+// (hs) and h, exactly as the forward kernels compute them (fp32 FMA chains in
+// stream order, storage rounding of H').
 template <int N, typename S, int VE>
-__device__ __forceinline__ void bw_forward_slice(const S *Ht, const S *Yt, int64_t d, int64_t k,
-                                                 const float *At, const float *bt, const float *at,
-                                                 float (&hv)[N][VE], float (&yv)[VE],
-                                                 float (&hs)[N][VE], float (&h)[VE]) {
+__device__ __forceinline__ void bw_forward_from(const float (&hv)[N][VE], const float (&yv)[VE],
+                                                const float *At, const float *bt, const float *at,
+                                                float (&hs)[N][VE], float (&h)[VE]) {
     using V = BwVec<S, VE>;
-#pragma unroll
-    for (int i = 0; i < N; ++i) V::load(Ht + i * d + k, hv[i]);
-    V::load(Yt + k, yv);
     // paired fp32 FMAs: each element's chain is the scalar one, bit for bit
 #pragma unroll
     for (int e = 0; e < VE; ++e) h[e] = -0.0f;
@@ -140,6 +136,110 @@ __device__ __forceinline__ void bw_forward_slice(const S *Ht, const S *Yt, int64
             h[e] = hh.x;
             h[e + 1] = hh.y;
         }
+    }
+}
+
+// The same, loading the slice's H and y rows from global memory first.
+template <int N, typename S, int VE>
+__device__ __forceinline__ void bw_forward_slice(const S *Ht, const S *Yt, int64_t d, int64_t k,
+                                                 const float *At, const float *bt, const float *at,
+                                                 float (&hv)[N][VE], float (&yv)[VE],
+                                                 float (&hs)[N][VE], float (&h)[VE]) {
+    using V = BwVec<S, VE>;
+#pragma unroll
+    for (int i = 0; i < N; ++i) V::load(Ht + i * d + k, hv[i]);
+    V::load(Yt + k, yv);
+    bw_forward_from<N, S, VE>(hv, yv, At, bt, at, hs, h);
+}
+
+// Per-thread asynchronous copies (cp.async, no registers held while in
+// flight) of CB = 8 or 16 bytes to a shared-memory address (32-bit, shared
+// window) from global memory; each thread waits on its
+// own groups and reads back only what it copied, so no barrier is needed.
+template <int CB>
+__device__ __forceinline__ void bw_cp_async(unsigned sa, const void *gmem) {
+    static_assert(CB == 8 || CB == 16, "chunk of 8 or 16 bytes");
+    if constexpr (CB == 16)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
+    else
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void bw_cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int NW>
+__device__ __forceinline__ void bw_cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(NW) : "memory"); }
+__device__ __forceinline__ void bw_cp_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// A VE-element storage vector from shared memory, widened to fp32.
+template <typename S, int VE>
+__device__ __forceinline__ void bw_ld_stage(const unsigned char *p, float (&v)[VE]) {
+    if constexpr (sizeof(S) == 2) {
+        const uint2 q = *reinterpret_cast<const uint2 *>(p);
+        widen_bf16x2(q.x, v[0], v[1]);
+        widen_bf16x2(q.y, v[2], v[3]);
+    } else if constexpr (VE == 4) {
+        const float4 q = *reinterpret_cast<const float4 *>(p);
+        v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+    } else {
+        const float2 q = *reinterpret_cast<const float2 *>(p);
+        v[0] = q.x; v[1] = q.y;
+    }
+}
+
+__host__ __device__ constexpr int bw_pow2_ceil(int m) {
+    int p = 1;
+    while (p < m) p *= 2;
+    return p;
+}
+
+// Warp sums of M per-lane values in one halving exchange: at each step the
+// lanes with the offset's bit set keep the upper half of their values and
+// send the lower half, the others the reverse, so P - 1 shuffles (P = M
+// rounded up to a power of two, <= 32) replace M butterflies of five. Value m
+// ends in lane m * (32 / P) and its copies (the remaining butterfly steps);
+// dst[m] is written from there. Summation order: a fixed tree per launch
+// shape, so the result is reproducible.
+template <int M>
+__device__ __forceinline__ void bw_warp_sums_to(const float (&v)[M], float *dst, int lane) {
+    static_assert(M <= 32, "at most 32 values per exchange");
+    constexpr int P = bw_pow2_ceil(M);
+    float w[P];
+#pragma unroll
+    for (int m = 0; m < P; ++m) w[m] = m < M ? v[m] : 0.0f;
+    int o = 16;
+#pragma unroll
+    for (int h = P / 2; h >= 1; h /= 2) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int m = 0; m < h; ++m) {
+            const float send = up ? w[m] : w[m + h];
+            const float keep = up ? w[m + h] : w[m];
+            w[m] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+        o >>= 1;
+    }
+    float s = w[0];
+#pragma unroll
+    for (; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    // lane bits 4, 3, ... (one per halving) spell the value index
+    constexpr int span = 32 / P;
+    const int idx = lane / span;
+    if (lane % span == 0 && idx < M) dst[idx] = s;
+}
+
+// VE fp32 values to and from shared memory (16- or 8-byte accesses).
+template <int VE>
+__device__ __forceinline__ void bw_st_f32(float *p, const float (&v)[VE]) {
+    if constexpr (VE == 4) *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    else *reinterpret_cast<float2 *>(p) = make_float2(v[0], v[1]);
+}
+template <int VE>
+__device__ __forceinline__ void bw_ld_f32(const float *p, float (&v)[VE]) {
+    if constexpr (VE == 4) {
+        const float4 q = *reinterpret_cast<const float4 *>(p);
+        v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+    } else {
+        const float2 q = *reinterpret_cast<const float2 *>(p);
+        v[0] = q.x; v[1] = q.y;
     }
 }
 
