@@ -565,9 +565,15 @@ hc_dg_reduce_kernel(const float *part, int rows, int64_t d, float *dg) {
 template <int N, typename S>
 struct StepBw {
     static constexpr int VE = bw_vec_elems<S>(N);
-    // Shared-memory budget of the dynamic part: two CTAs per SM up to n = 5
-    // (2 x (104 KB + static + 1 KB reserved) <= 228 KB).
-    static constexpr size_t kDynBudget = N <= 5 ? 104 * 1024 : 176 * 1024;
+    // Static shared memory of the step kernel, and the dynamic budget that
+    // leaves room for two CTAs per SM up to n = 5 (228 KB per SM, 1 KB
+    // reserved per CTA), one CTA above.
+    static constexpr size_t kStatic = 4 * ((size_t)kBwTB * (N * N + 2 * N)) + 16 * (kBwThreads / 32) +
+                                      4 * (kBwThreads / 32) * (size_t)(2 * N + N * N + N) +
+                                      4 * (kBwThreads / 32) * (size_t)kGroupScratch;
+    static constexpr size_t kSmemPerSm = 228 * 1024;
+    static constexpr size_t kDynBudget =
+        N <= 5 ? kSmemPerSm / 2 - 1024 - kStatic - 256 : (size_t)kSmemLimitLogits - kStatic - 1024;
     static constexpr int kRing = HC_BW_RING;
     static_assert(kRing == 0 || kRing >= 2, "two staging stages at least");
     static size_t park_bytes(int64_t d) { return (size_t)d * 4; }  // h, fp32
