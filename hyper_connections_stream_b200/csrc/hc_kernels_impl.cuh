@@ -109,9 +109,35 @@ bool pipe_shape(const StepParams &p, int rows, PipeShape &sh, int &smem) {
     return true;
 }
 
-template <int N, typename S, int KIND>
+template <int N, typename S, int KIND, int GW = pipe_group_warps(N)>
 bool pipe_shape(const StepParams &p, PipeShape &sh, int &smem) {
-    return pipe_shape<N, S, KIND>(p, KIND != KIND_READ ? N + 1 : N, sh, smem);
+    return pipe_shape<N, S, KIND, GW>(p, KIND != KIND_READ ? N + 1 : N, sh, smem);
+}
+
+// The other consumer-group width a call may take: eight warps at n <= 2
+// (576 threads fit the register file there), chosen when it pads the row's
+// slices less than the default width does -- d = 4096 in bf16 is two tiles
+// of 2048 instead of three of 1792 (measured at n = 2, T = 16384: 71.7 ->
+// 78.1 % of copy; at d = 7168, where seven-warp tiles fit exactly, the
+// default stays).
+template <int N>
+constexpr int pipe_alt_group_warps() { return N <= 2 ? 8 : pipe_group_warps(N); }
+
+template <int N, typename S>
+int64_t pipe_padded_slices(int64_t d, int gw) {
+    const int64_t nvec = d / pipe_vec_elems<N, S>();
+    const int64_t per = (int64_t)gw * 32;
+    return (nvec + per - 1) / per * per;
+}
+
+template <int N, typename S>
+bool pipe_take_alt(int64_t d) {
+    if constexpr (pipe_alt_group_warps<N>() == pipe_group_warps(N)) {
+        return false;
+    } else {
+        return pipe_padded_slices<N, S>(d, pipe_alt_group_warps<N>()) <
+               pipe_padded_slices<N, S>(d, pipe_group_warps(N));
+    }
 }
 
 template <int N, typename S, int KIND, int GW = pipe_group_warps(N)>
@@ -138,9 +164,11 @@ hc_status launch_pipe(const StepParams &p, const PipeShape &sh, int smem, const 
 
 template <int N, typename S, int KIND>
 hc_status launch_step_n(const StepParams &p, const LaunchCtx &ctx, cudaStream_t st) {
+    constexpr int GWA = pipe_alt_group_warps<N>();
+    const bool alt = pipe_take_alt<N, S>(p.d);
     PipeShape sh{};
     int smem = 0;
-    const bool pipe_ok = pipe_shape<N, S, KIND>(p, sh, smem);
+    const bool pipe_ok = alt ? pipe_shape<N, S, KIND, GWA>(p, sh, smem) : pipe_shape<N, S, KIND>(p, sh, smem);
     if (ctx.path == 1 && !pipe_ok)
         return set_error(HC_ERR_UNSUPPORTED, "pipelined kernels do not cover d = %lld here",
                          (long long)p.d);
@@ -157,9 +185,9 @@ hc_status launch_step_n(const StepParams &p, const LaunchCtx &ctx, cudaStream_t 
     if constexpr (KIND == KIND_FUSED) {
         constexpr int64_t tmin_n[9] = {0, 512, 512, 256, 256, 1024, 4096, 2048, 2048};
         constexpr int64_t ragged_x[9] = {0, 16, 16, 4, 4, 16, 4, 4, 4};
-        constexpr int64_t per_tile = (int64_t)pipe_group_warps(N) * 32;  // slices per tile
+        // raggedness of the default width, which the thresholds were fitted on
         const int64_t nvec = p.d / pipe_vec_elems<N, S>();
-        const int64_t slots = (nvec + per_tile - 1) / per_tile * per_tile;
+        const int64_t slots = pipe_padded_slices<N, S>(p.d, pipe_group_warps(N));
         const bool ragged = (slots - nvec) * 8 > slots;
         small = p.T < tmin_n[N] * (ragged ? ragged_x[N] : 1);
     }
@@ -168,6 +196,7 @@ hc_status launch_step_n(const StepParams &p, const LaunchCtx &ctx, cudaStream_t 
             return set_error(HC_ERR_UNSUPPORTED, "d = %lld too large", (long long)p.d);
         return launch_stream<N, S, KIND>(p, ctx, st);
     }
+    if (alt) return launch_pipe<N, S, KIND, GWA>(p, sh, smem, ctx, st);
     return launch_pipe<N, S, KIND>(p, sh, smem, ctx, st);
 }
 
@@ -206,8 +235,12 @@ hc_status launch_reduce_pipe_n(const ReduceWriteArgs &ra, const bool *local, con
     rd.t0 = ra.t0;
     PipeShape sh{};
     int smem = 0;
-    *fits = pipe_shape<N, S, KIND_REDUCE>(ra.f, N + nlocal, sh, smem);
+    constexpr int GWA = pipe_alt_group_warps<N>();
+    const bool alt = pipe_take_alt<N, S>(ra.f.d);
+    *fits = alt ? pipe_shape<N, S, KIND_REDUCE, GWA>(ra.f, N + nlocal, sh, smem)
+                : pipe_shape<N, S, KIND_REDUCE>(ra.f, N + nlocal, sh, smem);
     if (!*fits) return HC_OK;
+    if (alt) return launch_pipe<N, S, KIND_REDUCE, GWA>(ra.f, sh, smem, ctx, st, rd);
     return launch_pipe<N, S, KIND_REDUCE>(ra.f, sh, smem, ctx, st, rd);
 }
 
