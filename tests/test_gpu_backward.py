@@ -113,6 +113,10 @@ def _check(hc, T, n, d, dt, mix, read, per_token, seed, with_dHout=True, K=20):
     (97, 3, 1544, "bf16", True, True, False),
     (61, 5, 2056, "bf16", True, True, True),
     (2000, 4, 1024, "bf16", True, True, True),
+    # wide rows: h parked without the staging ring (d = 16384), and h rebuilt
+    # in phase 2 because even the parked row does not fit (d = 32768)
+    (20, 4, 16384, "bf16", True, True, True),
+    (9, 2, 32768, "bf16", False, True, True),
 ])
 def test_backward_matches_oracle(hc, T, n, d, dt, mix, read, per_token):
     _check(hc, T, n, d, dt, mix, read, per_token, seed=1200 + T + n)
