@@ -281,6 +281,29 @@ def test_shape_sweep_mhc(hc, T, n, d):
 # Edge cases
 # ---------------------------------------------------------------------------
 
+@pytest.mark.parametrize("n", [1, 2])
+@pytest.mark.parametrize("dt,d", [("bf16", 4096), ("bf16", 2048), ("f32", 4096)])
+def test_eight_warp_groups_every_kind(hc, n, dt, d):
+    """Widths at which n <= 2 takes eight-warp consumer groups in the
+    pipelined family (they pad the row's slices less than seven do): the
+    read, the write and the fused step, bit-exact against the oracle with
+    static parameters, over a ragged token count."""
+    T = 300
+    H = gen.streams(60 + n, T, n, d, dt)
+    y = gen.block_out(60 + n, T, d, dt)
+    a, A, b = gen.static_params(61 + n, n)
+    a2, _, _ = gen.static_params(61 + n, n, layer=1)
+    g = gen.gain(62 + n, d)
+    Hd, yd = to_dev(H, dt), to_dev(y, dt)
+    x = to_host(hc.read_rmsnorm(Hd, f32_dev(a), f32_dev(g), eps=EPS), dt)
+    assert_bitwise(x, oracle.read_rmsnorm(H, a, g, EPS, dt), "read")
+    Hw_ref = oracle.write_mix(H, y, A, b, dt)
+    assert_bitwise(to_host(hc.write_mix(Hd, yd, f32_dev(A), f32_dev(b)), dt), Hw_ref, "write")
+    H2, x2 = hc.write_then_read(Hd, yd, f32_dev(A), f32_dev(b), f32_dev(a2), f32_dev(g), eps=EPS)
+    assert_bitwise(to_host(H2, dt), Hw_ref, "fused H'")
+    assert_bitwise(to_host(x2, dt), oracle.read_rmsnorm(Hw_ref, a2, g, EPS, dt), "fused x")
+
+
 @pytest.mark.parametrize("n", list(range(1, 9)))
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
 def test_every_n_ragged_d_per_token_params(hc, n, dt):

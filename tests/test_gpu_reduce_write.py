@@ -90,6 +90,9 @@ def _run(hc, parts, H, A, b, a, g, dt, logits, K=20, want_y=True, inplace=False)
     (50, 8, 1032, 2, "bf16", True),
     (300, 3, 2056, 5, "f32", True),
     (1, 5, 264, 7, "bf16", False),
+    # n <= 2 at widths where the pipelined kernel takes eight-warp groups
+    (300, 2, 4096, 8, "bf16", True),
+    (77, 1, 4096, 3, "f32", False),
 ])
 def test_static_parameters_bitwise(hc, T, n, d, R, dt, per_token):
     parts, H, A, b, a, g = _case(T, n, d, R, dt, False, per_token, seed=3000 + 7 * T + R)
