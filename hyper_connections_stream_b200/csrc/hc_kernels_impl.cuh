@@ -114,14 +114,18 @@ bool pipe_shape(const StepParams &p, PipeShape &sh, int &smem) {
     return pipe_shape<N, S, KIND, GW>(p, KIND != KIND_READ ? N + 1 : N, sh, smem);
 }
 
-// The other consumer-group width a call may take: eight warps at n <= 2
-// (576 threads fit the register file there), chosen when it pads the row's
-// slices less than the default width does -- d = 4096 in bf16 is two tiles
-// of 2048 instead of three of 1792 (measured at n = 2, T = 16384: 71.7 ->
-// 78.1 % of copy; at d = 7168, where seven-warp tiles fit exactly, the
-// default stays).
-template <int N>
-constexpr int pipe_alt_group_warps() { return N <= 2 ? 8 : pipe_group_warps(N); }
+// The other consumer-group width a call may take: eight warps (576 threads;
+// the compiler fits every kind in 96 registers without spills there), chosen
+// when it pads the row's slices less than the default width does -- d =
+// 4096 in bf16 is two tiles of 2048 instead of three of 1792. The read and
+// write kinds take it up to n = 4 (static layer, T = 4096, n = 4, d = 4096:
+// read 43.7 -> 40.7 us, write 52.4 -> 48.5 us); the fused and all-reduce
+// kinds, whose consumers then run on fewer registers, at n <= 2 (n = 2,
+// T = 16384: 71.7 -> 78.1 % of copy) and at n = 3, 4 only for calls of up to
+// 8192 tokens (n = 4: T = 1024 +5 %, T = 4096 +3 %, but T = 16384 -1 %).
+// Where seven-warp tiles fit exactly (d = 7168) the default stays.
+template <int N, int KIND>
+constexpr int pipe_alt_group_warps() { return N <= 4 ? 8 : pipe_group_warps(N); }
 
 template <int N, typename S>
 int64_t pipe_padded_slices(int64_t d, int gw) {
@@ -130,12 +134,13 @@ int64_t pipe_padded_slices(int64_t d, int gw) {
     return (nvec + per - 1) / per * per;
 }
 
-template <int N, typename S>
-bool pipe_take_alt(int64_t d) {
-    if constexpr (pipe_alt_group_warps<N>() == pipe_group_warps(N)) {
+template <int N, typename S, int KIND>
+bool pipe_take_alt(int64_t d, int64_t T) {
+    if constexpr (pipe_alt_group_warps<N, KIND>() == pipe_group_warps(N)) {
         return false;
     } else {
-        return pipe_padded_slices<N, S>(d, pipe_alt_group_warps<N>()) <
+        if (!(KIND == KIND_READ || KIND == KIND_WRITE) && N > 2 && T > 8192) return false;
+        return pipe_padded_slices<N, S>(d, pipe_alt_group_warps<N, KIND>()) <
                pipe_padded_slices<N, S>(d, pipe_group_warps(N));
     }
 }
@@ -164,8 +169,8 @@ hc_status launch_pipe(const StepParams &p, const PipeShape &sh, int smem, const 
 
 template <int N, typename S, int KIND>
 hc_status launch_step_n(const StepParams &p, const LaunchCtx &ctx, cudaStream_t st) {
-    constexpr int GWA = pipe_alt_group_warps<N>();
-    const bool alt = pipe_take_alt<N, S>(p.d);
+    constexpr int GWA = pipe_alt_group_warps<N, KIND>();
+    const bool alt = pipe_take_alt<N, S, KIND>(p.d, p.T);
     PipeShape sh{};
     int smem = 0;
     const bool pipe_ok = alt ? pipe_shape<N, S, KIND, GWA>(p, sh, smem) : pipe_shape<N, S, KIND>(p, sh, smem);
@@ -235,8 +240,8 @@ hc_status launch_reduce_pipe_n(const ReduceWriteArgs &ra, const bool *local, con
     rd.t0 = ra.t0;
     PipeShape sh{};
     int smem = 0;
-    constexpr int GWA = pipe_alt_group_warps<N>();
-    const bool alt = pipe_take_alt<N, S>(ra.f.d);
+    constexpr int GWA = pipe_alt_group_warps<N, KIND_REDUCE>();
+    const bool alt = pipe_take_alt<N, S, KIND_REDUCE>(ra.f.d, ra.f.T);
     *fits = alt ? pipe_shape<N, S, KIND_REDUCE, GWA>(ra.f, N + nlocal, sh, smem)
                 : pipe_shape<N, S, KIND_REDUCE>(ra.f, N + nlocal, sh, smem);
     if (!*fits) return HC_OK;

@@ -281,13 +281,14 @@ def test_shape_sweep_mhc(hc, T, n, d):
 # Edge cases
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("n", [1, 2])
+@pytest.mark.parametrize("n", [1, 2, 3, 4])
 @pytest.mark.parametrize("dt,d", [("bf16", 4096), ("bf16", 2048), ("f32", 4096)])
 def test_eight_warp_groups_every_kind(hc, n, dt, d):
-    """Widths at which n <= 2 takes eight-warp consumer groups in the
-    pipelined family (they pad the row's slices less than seven do): the
-    read, the write and the fused step, bit-exact against the oracle with
-    static parameters, over a ragged token count."""
+    """Widths at which the pipelined family takes eight-warp consumer groups
+    (they pad the row's slices less than seven do; read and write kinds up to
+    n = 4, the fused step up to n = 2): the read, the write and the fused
+    step, bit-exact against the oracle with static parameters, over a ragged
+    token count."""
     T = 300
     H = gen.streams(60 + n, T, n, d, dt)
     y = gen.block_out(60 + n, T, d, dt)
