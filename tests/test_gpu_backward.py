@@ -117,6 +117,9 @@ def _check(hc, T, n, d, dt, mix, read, per_token, seed, with_dHout=True, K=20):
     # in phase 2 because even the parked row does not fit (d = 32768)
     (20, 4, 16384, "bf16", True, True, True),
     (9, 2, 32768, "bf16", False, True, True),
+    # fp32 beyond n = 4 (two-element vectors, 8-byte staging copies)
+    (23, 6, 1000, "f32", True, True, True),
+    (19, 8, 520, "f32", True, False, True),
 ])
 def test_backward_matches_oracle(hc, T, n, d, dt, mix, read, per_token):
     _check(hc, T, n, d, dt, mix, read, per_token, seed=1200 + T + n)
