@@ -105,15 +105,14 @@ hc_step_bwd_kernel(BwKernelParams bp) {
             const float z[VE] = {};
             bw_st_f32<VE>(sdg + c * VE, z);
         }
-    unsigned char *dyn_rest = bw_dyn;
-    float *shp = reinterpret_cast<float *>(dyn_rest);  // [d] parked h
+    float *shp = reinterpret_cast<float *>(bw_dyn);  // [d] parked h
 
     // Staging ring: [RING slots][2N + 2 rows: H, y, dx, dH'][NT threads]
     // chunks of VE elements, so a warp's copies of one row land contiguously.
     constexpr int RR = 2 * N + 2;
     constexpr int CB = VE * (int)sizeof(S);
     const int ROW = NT * CB;
-    unsigned char *ring0 = dyn_rest + (PARK ? d * 4 : 0);
+    unsigned char *ring0 = bw_dyn + (PARK ? d * 4 : 0);
     auto slot = [&](int st, int row) -> unsigned char * {
         return ring0 + ((size_t)(st * RR + row) * NT + tid) * CB;
     };
@@ -233,8 +232,7 @@ hc_step_bwd_kernel(BwKernelParams bp) {
                 }
                 if constexpr (2 * N <= 32) {
                     bw_warp_sums_to<2 * N>(v1, pred1[warp], lane);
-                } else
-                {
+                } else {
 #pragma unroll
                     for (int v = 0; v < 2 * N; ++v) {
                         float val = v1[v];
@@ -398,8 +396,7 @@ hc_step_bwd_kernel(BwKernelParams bp) {
                 for (int j = 0; j < N; ++j) v2[NN + j] = __fadd_rn(pb2[j].x, pb2[j].y);
                 if constexpr (NS <= 32) {
                     bw_warp_sums_to<NS>(v2, pred[warp], lane);
-                } else
-                {
+                } else {
 #pragma unroll
                     for (int v = 0; v < NS; ++v) {
                         float val = v2[v];
