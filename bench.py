@@ -818,12 +818,11 @@ def run_sweep(args):
                 graph = T <= 4096
                 ncalls = max(P, 64) if graph else max(P, 5 if T >= 65536 else 20)
                 ms = _per_call_ms(call, ncalls, device, graph=graph)
-                small = T * n * d * 2 * 2 < 64 * 2 ** 20
+                family = hc.step_path("fused", T, n, d)
                 orate, S = _oracle_point_rate(T, n, d, K, eps)
                 point_line("sweep_fused_mhc", T, n, d, ms, alg,
                            {"buffer_sets": P, "calls": ncalls, "graph": graph,
-                            "kernel_family": "register" if (small and args.path == "auto")
-                            else args.path if args.path != "auto" else "pipelined",
+                            "kernel_family": "register" if family == hc.PATH_REGISTER else "pipelined",
                             "oracle_tokens_per_s": orate, "oracle_sample_tokens": S})
                 del Hin, Hout, y, L, rl, x
                 torch.cuda.empty_cache()
@@ -849,9 +848,13 @@ def run_sweep(args):
             "fused": (lambda i: hc.write_then_read(Hs[i % P], ys[i % P], A, b, a, g, eps=eps,
                                                    out=Ho[i % P], x_next=xs[i % P]), per["fused"]),
         }
+        fam = {k: ("register" if hc.step_path(k, T, n, d) == hc.PATH_REGISTER else "pipelined")
+               for k in ("read", "write", "fused")}
+        fam["unfused_pair"] = f"write {fam['write']}, read {fam['read']}"
         for name, (fn, alg) in ops.items():
             ms = _per_call_ms(fn, max(P, 64), device, graph=True)
-            point_line("static_layer_" + name, T, n, d, ms, alg, {"buffer_sets": P})
+            point_line("static_layer_" + name, T, n, d, ms, alg,
+                       {"buffer_sets": P, "kernel_family": fam[name]})
         del Hs, Ho, ys, xs
         torch.cuda.empty_cache()
 

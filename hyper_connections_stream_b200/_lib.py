@@ -36,6 +36,7 @@ SIGNATURES = {
                             _vp, _i64, _i32, _vp, _i64, _vp, _f32, _vp], _i32),
     "hc_set_path": ([_i32], _i32),
     "hc_get_path": ([], _i32),
+    "hc_step_path": ([_i32, _i32, _i64, _i32, _i64, C.POINTER(_i32)], _i32),
     "hc_device_fault": ([C.POINTER(_i32), _vp], _i32),
     "hc_selftest_bounded_wait": ([_i32, _vp], _i32),
     "hc_mix_logits": ([_vp, _vp, _vp, _i32, _i64, _i32, _i64, _i32, _f32, _vp], _i32),
@@ -179,6 +180,18 @@ def set_path(path: int) -> None:
 
 def get_path() -> int:
     return int(lib().hc_get_path())
+
+
+STEP_OPS = {"read": 0, "write": 1, "fused": 2}
+
+
+def step_path(op: str, T: int, n: int, d: int, dtype=torch.bfloat16) -> int:
+    """The kernel family (PATH_PIPELINED or PATH_REGISTER) a read, write or
+    fused step call of these sizes takes on the current device under the
+    current set_path setting; nothing is launched."""
+    out = C.c_int(0)
+    _check(lib().hc_step_path(_DT[dtype], STEP_OPS[op], int(T), int(n), int(d), C.byref(out)))
+    return int(out.value)
 
 
 def device_fault(device=None) -> int:

@@ -192,6 +192,32 @@ hc_status hc_set_path(hc_path path) {
 
 hc_path hc_get_path(void) { return (hc_path)hc::g_path.load(std::memory_order_relaxed); }
 
+hc_status hc_step_path(hc_dtype dt, int op, int64_t T, int n, int64_t d, hc_path *path) {
+    static const char *fn = "hc_step_path";
+    g_last_error[0] = '\0';
+    if (!path) return fail(HC_ERR_INVALID_ARG, "%s: path is NULL", fn);
+    if (op < 0 || op > 2) return fail(HC_ERR_INVALID_ARG, "%s: bad op %d", fn, op);
+    const Shape s{dt, T, n, d};
+    HC_TRY(check_shape(fn, s, op != 1));
+    if (T < 1) return fail(HC_ERR_INVALID_ARG, "%s: T = %lld < 1", fn, (long long)T);
+    hc::LaunchCtx ctx{};
+    HC_TRY(launch_ctx(ctx));
+    hc::StepParams p{};
+    p.T = T;
+    p.d = d;
+    int r;
+    if (dt == HC_BF16)
+        r = op == 0   ? hc::step_path<__nv_bfloat16, hc::KIND_READ>(n, p, ctx)
+            : op == 1 ? hc::step_path<__nv_bfloat16, hc::KIND_WRITE>(n, p, ctx)
+                      : hc::step_path<__nv_bfloat16, hc::KIND_FUSED>(n, p, ctx);
+    else
+        r = op == 0   ? hc::step_path<float, hc::KIND_READ>(n, p, ctx)
+            : op == 1 ? hc::step_path<float, hc::KIND_WRITE>(n, p, ctx)
+                      : hc::step_path<float, hc::KIND_FUSED>(n, p, ctx);
+    *path = (hc_path)r;
+    return HC_OK;
+}
+
 hc_status hc_device_fault(int *code, hc_stream stream) {
     g_last_error[0] = '\0';
     if (!code) return fail(HC_ERR_INVALID_ARG, "hc_device_fault: code is NULL");

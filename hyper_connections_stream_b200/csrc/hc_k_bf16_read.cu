@@ -3,3 +3,4 @@
 
 template hc_status hc::launch_kind<__nv_bfloat16, hc::KIND_READ>(int, const hc::StepParams &,
                                                           const hc::LaunchCtx &, cudaStream_t);
+template int hc::step_path<__nv_bfloat16, hc::KIND_READ>(int, const hc::StepParams &, const hc::LaunchCtx &);

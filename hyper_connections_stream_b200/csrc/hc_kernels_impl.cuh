@@ -167,36 +167,49 @@ hc_status launch_pipe(const StepParams &p, const PipeShape &sh, int smem, const 
     return HC_OK;
 }
 
+// Which family a call takes (1 pipelined, 2 register-streaming), with the
+// pipelined geometry when that family applies. From measurements of both
+// (B200, bf16, graph-replayed calls, T = 256 ... 65536, n = 1 ... 8, d =
+// 4096, 7168). The read kind: the register-streaming family at every size
+// measured (5-39 % faster; within noise only at n = 3, 4, d = 7168). The
+// write kind: register-streaming at n <= 2 (7-38 % faster), else below ~64
+// MiB of stream traffic. The fused step: the pipeline needs enough tokens per
+// CTA to amortise its fill and the first parameter batches -- a per-n token
+// count (wider n: costlier Sinkhorn), times a factor when more than an eighth
+// of the last seven-warp tile would idle (at n = 1 such rows stay
+// register-streaming at any T: 6-10 % faster at d = 4096).
 template <int N, typename S, int KIND>
-hc_status launch_step_n(const StepParams &p, const LaunchCtx &ctx, cudaStream_t st) {
+int step_path_n(const StepParams &p, const LaunchCtx &ctx, bool &pipe_ok, bool &alt, PipeShape &sh,
+                int &smem) {
     constexpr int GWA = pipe_alt_group_warps<N, KIND>();
-    const bool alt = pipe_take_alt<N, S, KIND>(p.d, p.T);
-    PipeShape sh{};
-    int smem = 0;
-    const bool pipe_ok = alt ? pipe_shape<N, S, KIND, GWA>(p, sh, smem) : pipe_shape<N, S, KIND>(p, sh, smem);
-    if (ctx.path == 1 && !pipe_ok)
-        return set_error(HC_ERR_UNSUPPORTED, "pipelined kernels do not cover d = %lld here",
-                         (long long)p.d);
-    // Small calls (decode-sized batches) finish sooner without the pipeline's
-    // set-up. For the fused step the pipeline needs enough tokens per CTA to
-    // amortise its fill and the first parameter batches: a per-n token count
-    // (wider n: costlier Sinkhorn), times a factor when more than an eighth
-    // of the last pipelined tile would idle. Fitted to a crossover measurement
-    // of both families (B200, bf16, graph-replayed calls, T = 256 ... 8192,
-    // n in {2, 4, 5, 6, 8}, d in {4096, 7168}). The other kinds use the
-    // stream-traffic rule they were measured with: below ~64 MiB the
-    // register-streaming family wins.
+    alt = pipe_take_alt<N, S, KIND>(p.d, p.T);
+    pipe_ok = alt ? pipe_shape<N, S, KIND, GWA>(p, sh, smem) : pipe_shape<N, S, KIND>(p, sh, smem);
     bool small = p.T * (int64_t)N * p.d * (int64_t)sizeof(S) * 2 < (int64_t(64) << 20);
+    if constexpr (KIND == KIND_READ) small = true;
+    if constexpr (KIND == KIND_WRITE && N <= 2) small = true;
     if constexpr (KIND == KIND_FUSED) {
         constexpr int64_t tmin_n[9] = {0, 512, 512, 256, 256, 1024, 4096, 2048, 2048};
-        constexpr int64_t ragged_x[9] = {0, 16, 16, 4, 4, 16, 4, 4, 4};
+        constexpr int64_t ragged_x[9] = {0, int64_t(1) << 40, 64, 4, 4, 16, 4, 4, 4};
         // raggedness of the default width, which the thresholds were fitted on
         const int64_t nvec = p.d / pipe_vec_elems<N, S>();
         const int64_t slots = pipe_padded_slices<N, S>(p.d, pipe_group_warps(N));
         const bool ragged = (slots - nvec) * 8 > slots;
         small = p.T < tmin_n[N] * (ragged ? ragged_x[N] : 1);
     }
-    if (ctx.path == 2 || !pipe_ok || (ctx.path == 0 && small)) {
+    return (ctx.path == 2 || !pipe_ok || (ctx.path == 0 && small)) ? 2 : 1;
+}
+
+template <int N, typename S, int KIND>
+hc_status launch_step_n(const StepParams &p, const LaunchCtx &ctx, cudaStream_t st) {
+    constexpr int GWA = pipe_alt_group_warps<N, KIND>();
+    PipeShape sh{};
+    int smem = 0;
+    bool pipe_ok = false, alt = false;
+    const int path = step_path_n<N, S, KIND>(p, ctx, pipe_ok, alt, sh, smem);
+    if (ctx.path == 1 && !pipe_ok)
+        return set_error(HC_ERR_UNSUPPORTED, "pipelined kernels do not cover d = %lld here",
+                         (long long)p.d);
+    if (path == 2) {
         if (kind_normalises(KIND) && p.d > (int64_t)kStreamMaxThreads * 8 * StorageTraits<S>::V)
             return set_error(HC_ERR_UNSUPPORTED, "d = %lld too large", (long long)p.d);
         return launch_stream<N, S, KIND>(p, ctx, st);
@@ -261,6 +274,28 @@ hc_status launch_reduce_pipe(const ReduceWriteArgs &ra, const bool *local, const
         case 6: return launch_reduce_pipe_n<6, S>(ra, local, ctx, st, fits);
         case 7: return launch_reduce_pipe_n<7, S>(ra, local, ctx, st, fits);
         default: return launch_reduce_pipe_n<8, S>(ra, local, ctx, st, fits);
+    }
+}
+
+// The family launch_kind<S, KIND> would take for p (no launch).
+template <typename S, int KIND>
+int step_path(int n, const StepParams &p, const LaunchCtx &ctx) {
+    if constexpr (KIND >= KIND_EXPAND) {
+        return 2;
+    } else {
+        PipeShape sh{};
+        int smem = 0;
+        bool ok = false, alt = false;
+        switch (n) {
+            case 1: return step_path_n<1, S, KIND>(p, ctx, ok, alt, sh, smem);
+            case 2: return step_path_n<2, S, KIND>(p, ctx, ok, alt, sh, smem);
+            case 3: return step_path_n<3, S, KIND>(p, ctx, ok, alt, sh, smem);
+            case 4: return step_path_n<4, S, KIND>(p, ctx, ok, alt, sh, smem);
+            case 5: return step_path_n<5, S, KIND>(p, ctx, ok, alt, sh, smem);
+            case 6: return step_path_n<6, S, KIND>(p, ctx, ok, alt, sh, smem);
+            case 7: return step_path_n<7, S, KIND>(p, ctx, ok, alt, sh, smem);
+            default: return step_path_n<8, S, KIND>(p, ctx, ok, alt, sh, smem);
+        }
     }
 }
 

@@ -25,6 +25,9 @@ hc_status set_error(hc_status st, const char *fmt, ...);
 // Launch one step kind (KIND_READ / KIND_WRITE / KIND_FUSED) for n streams.
 template <typename S, int KIND>
 hc_status launch_kind(int n, const StepParams &p, const LaunchCtx &ctx, cudaStream_t st);
+// The kernel family launch_kind would take for p: 1 pipelined, 2 register-streaming.
+template <typename S, int KIND>
+int step_path(int n, const StepParams &p, const LaunchCtx &ctx);
 
 // 2-D bf16 TMA tensor map over a row-major [outer][inner] array: 128-byte
 // swizzle, zero fill out of bounds, box of box_outer rows x box_inner elements.

@@ -343,18 +343,29 @@ HC_API hc_status hc_collapse(const void *H, void *out, hc_dtype dt, int64_t T, i
 /*
  * Kernel family used by the step calls (process-wide; default HC_PATH_AUTO).
  *   HC_PATH_PIPELINED: warp-specialised kernels fed by bulk copies (TMA) into
- *     shared-memory rings; the automatic choice for calls that move 64 MiB
- *     or more of stream state, where its rings fit (for calls that normalise,
- *     two fp32 rows of d per consumer group must fit next to them: d up to
- *     9880 bf16 at n = 4). Forcing it where it does not fit returns
+ *     shared-memory rings, where its rings fit (for calls that normalise, two
+ *     fp32 rows of d per consumer group must fit next to them: d up to 9880
+ *     bf16 at n = 4). Forcing it where it does not fit returns
  *     HC_ERR_UNSUPPORTED.
- *   HC_PATH_REGISTER: register-streaming kernels (no staging); the automatic
- *     choice for smaller calls (decode-sized batches) and larger d.
+ *   HC_PATH_REGISTER: register-streaming kernels (no staging).
+ *   HC_PATH_AUTO: per call, the family measured faster for its sizes -- the
+ *     register family for hc_read_rmsnorm, for hc_write_mix at n <= 2 and
+ *     for small calls (decode-sized batches), the pipelined family for larger
+ *     fused steps and writes (hc_step_path reports the choice).
  * Both families compute bit-identical results.
  */
 typedef enum { HC_PATH_AUTO = 0, HC_PATH_PIPELINED = 1, HC_PATH_REGISTER = 2 } hc_path;
 HC_API hc_status hc_set_path(hc_path path);
 HC_API hc_path hc_get_path(void);
+/*
+ * The kernel family a step call of these sizes would take on the current
+ * device under the current hc_set_path setting; nothing is launched.
+ *   op: 0 = hc_read_rmsnorm, 1 = hc_write_mix, 2 = hc_write_then_read.
+ *   *path receives HC_PATH_PIPELINED or HC_PATH_REGISTER.
+ * dt, n and d are validated as by those calls; T >= 1. HC_ERR_INVALID_ARG for
+ * a bad op, T < 1 or a NULL path.
+ */
+HC_API hc_status hc_step_path(hc_dtype dt, int op, int64_t T, int n, int64_t d, hc_path *path);
 
 /*
  * Device-side failure report. The pipelined kernels bound every wait on

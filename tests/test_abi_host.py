@@ -121,6 +121,13 @@ _CHILD = textwrap.dedent(r"""
     call("st_lo", "hc_selftest_bounded_wait", 0, None)
     call("st_hi", "hc_selftest_bounded_wait", 1000000, None)
     call("path_bad", "hc_set_path", 7)
+    pout = C.c_int(0)
+    call("sp_null", "hc_step_path", bf, 2, T, n, d, None)
+    call("sp_op", "hc_step_path", bf, 3, T, n, d, C.byref(pout))
+    call("sp_T0", "hc_step_path", bf, 2, 0, n, d, C.byref(pout))
+    call("sp_n9", "hc_step_path", bf, 2, T, 9, d, C.byref(pout))
+    call("sp_d_ragged", "hc_step_path", bf, 0, T, n, 12, C.byref(pout))
+    call("sp_dtype", "hc_step_path", 7, 1, T, n, d, C.byref(pout))
     xb = T * d * 2
     call("ex_T0", "hc_expand", None, None, bf, 0, n, d, None)
     call("ex_n9", "hc_expand", x, H, bf, T, 9, d, None)
@@ -208,6 +215,7 @@ def test_argument_validation_statuses():
         "mis_H": MIS, "mis_x": MIS, "mis_g": MIS, "mis_A": MIS, "alias_partial": ALI,
         "alias_y": ALI, "alias_x_H": ALI, "alias_x_read": ALI, "sk_n0": INV, "sk_K0": INV,
         "sk_null": INV, "sk_alias": ALI, "sk_T0": OK, "st_lo": INV, "st_hi": INV, "path_bad": INV,
+        "sp_null": INV, "sp_op": INV, "sp_T0": INV, "sp_n9": UNS, "sp_d_ragged": UNS, "sp_dtype": INV,
         "ex_T0": OK, "ex_n9": UNS, "ex_null": INV, "ex_mis": MIS, "ex_alias": ALI,
         "er_readmode": INV, "er_null_a": INV, "er_eps": INV, "er_alias_xr_H": ALI,
         "er_alias_xr_x": ALI, "er_d_too_big": UNS, "co_null_w": INV, "co_stride": INV,

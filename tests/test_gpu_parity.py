@@ -281,6 +281,31 @@ def test_shape_sweep_mhc(hc, T, n, d):
 # Edge cases
 # ---------------------------------------------------------------------------
 
+def test_step_path_reports_the_family_choice(hc):
+    """hc_step_path reports the measured per-call choice under automatic
+    selection (register-streaming for reads, for writes at n <= 2 and for
+    small fused steps; pipelined for the workload's fused step) and the forced
+    family otherwise."""
+    P, R = hc.PATH_PIPELINED, hc.PATH_REGISTER
+    saved = hc.get_path()
+    try:
+        hc.set_path(hc.PATH_AUTO)
+        assert hc.step_path("fused", 16384, 4, 7168) == P
+        assert hc.step_path("fused", 64, 4, 7168) == R
+        assert hc.step_path("fused", 16384, 1, 4096) == R
+        assert hc.step_path("read", 16384, 4, 7168) == R
+        assert hc.step_path("read", 65536, 8, 4096) == R
+        assert hc.step_path("write", 16384, 2, 7168) == R
+        assert hc.step_path("write", 16384, 4, 7168) == P
+        assert hc.step_path("write", 64, 4, 7168) == R
+        hc.set_path(hc.PATH_PIPELINED)
+        assert hc.step_path("read", 64, 4, 7168) == P
+        hc.set_path(hc.PATH_REGISTER)
+        assert hc.step_path("fused", 16384, 4, 7168) == R
+    finally:
+        hc.set_path(saved)
+
+
 @pytest.mark.parametrize("n", [1, 2, 3, 4])
 @pytest.mark.parametrize("dt,d", [("bf16", 4096), ("bf16", 2048), ("f32", 4096)])
 def test_eight_warp_groups_every_kind(hc, n, dt, d):
